@@ -1,0 +1,368 @@
+/*
+ * yarn_oracle.c -- plain fp64 CPU oracle for YaRN-RoPE causal GQA attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline of the benchmark may load this library.  It shares no code with
+ * the CUDA path and is deliberately slow: every quantity is computed straight
+ * from its definition in double precision, with no tiling, no fusion and no
+ * online softmax.
+ *
+ * Sources (the web pages on long-context position scaling):
+ *   [P1] "LLM context window mechanics" -- sections "The memory wall,
+ *        quantified" and "The position wall: RoPE and interpolation".
+ *   [P2] "Long Context" concept page -- "Key math / How it works".
+ *   [P3] "Arch_03_Long_Context" slide deck -- the RoPE, Position
+ *        Interpolation, NTK-aware, YaRN, sliding-window and sink slides.
+ *   [P4] "Long context (engineering 100k+ tokens)" -- section 2 (RoPE
+ *        scaling tricks) and section 5 (attention sinks).
+ *   [P5] "long-context-models" -- "Position enters attention" and
+ *        "Memory grows even with efficient attention".
+ *
+ * Readings taken where the pages are silent, garbled or disagree (each is
+ * also listed with its reason in the design notes of the repository):
+ *   - YaRN band split follows [P3] YaRN slide + the steps table (alpha=1,
+ *     beta=32), with the ramp linear in r = L_train / lambda_i; [P1]'s
+ *     printed code is garbled and is not followed.
+ *   - The temperature multiplies the logits by (0.1 ln s + 1)^2 / sqrt(d)
+ *     (equivalently mscale on both rotated q and k).
+ *   - Pairs are interleaved (2i, 2i+1) as on the [P3] RoPE slide.
+ *   - Window: key n is visible to query m iff n <= m (causal) and
+ *     (m - n < W or n < n_sink); positions are absolute.
+ *   - GQA: query head h reads KV head floor(h / (Hq/Hkv)).
+ *
+ * Parity status per function:
+ *   oracle_rope_theta   pinned (closed forms, s=1 reductions, NTK worked
+ *                       number, band endpoints); the YaRN ramp INTERIOR is
+ *                       a reading of the pages: parity unpinned there.
+ *   oracle_rotate_rows  pinned (page's rotation matrix, complex-number
+ *                       form, orthogonality, relative-position invariance).
+ *   oracle_attn_rows    pinned (library SDPA special case, closed-form
+ *                       means, page's "4 + last 4096" sink count, T=1).
+ *   oracle_decode       pinned (equals the prefill row at the same position).
+ *   oracle_kv_cache_bytes pinned (the pages' ~69 GB / ~17 GB / 40 GiB).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_ROPE 0
+#define OR_PI 1
+#define OR_NTK 2
+#define OR_YARN 3
+
+static double bf16_bits_to_double(uint16_t bits)
+{
+    /* bf16 is the upper half of an IEEE binary32: widening is exact. */
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/*
+ * Per-pair rotation frequencies theta'_i (i = 0 .. d/2-1), the YaRN mscale
+ * and the softmax logit scale.
+ *   RoPE  theta_i = base^(-2i/d)                       [P1] position wall; [P3] RoPE slide
+ *   PI    theta'_i = theta_i / s                        [P1]; [P3] PI slide (angles of m/s); [P4] sec. 2
+ *   NTK   theta'_i = (base * s^(d/(d-2)))^(-2i/d)       [P3] NTK-aware slide
+ *   YaRN  r_i = L_train * theta_i / (2 pi) = L_train / lambda_i   ([P3] YaRN slide: lambda_i = 2 pi / theta_i)
+ *         gamma_i = clamp((r_i - alpha) / (beta - alpha), 0, 1)
+ *         theta'_i = gamma_i * theta_i + (1 - gamma_i) * theta_i / s
+ *         (short wavelengths unchanged, long wavelengths interpolated as PI,
+ *          linear ramp between; alpha = 1, beta = 32 per the steps table)
+ *   mscale = 0.1 ln s + 1 for YaRN, else 1             [P1] position wall; [P3] YaRN slide
+ *   softmax_scale = mscale^2 / sqrt(d)
+ * Returns 0, or -1 for an invalid argument (odd or non-positive d, s < 1,
+ * base <= 1, beta <= alpha for YaRN, L_train < 1 for YaRN).
+ */
+int oracle_rope_theta(int d, double base, int L_train, double s, int method,
+                      double alpha, double beta, double *theta,
+                      double *mscale, double *softmax_scale)
+{
+    if (d <= 0 || (d % 2) != 0) return -1;
+    if (!(s >= 1.0) || !(base > 1.0)) return -1;
+    if (method < OR_ROPE || method > OR_YARN) return -1;
+    if (method == OR_YARN && (!(beta > alpha) || L_train < 1)) return -1;
+    const int half = d / 2;
+    for (int i = 0; i < half; ++i) {
+        const double expo = -2.0 * (double)i / (double)d;
+        const double th = pow(base, expo);
+        double out = th;
+        if (method == OR_PI) {
+            out = th / s;
+        } else if (method == OR_NTK) {
+            const double base_ntk = base * pow(s, (double)d / (double)(d - 2));
+            out = pow(base_ntk, expo);
+        } else if (method == OR_YARN) {
+            const double r = (double)L_train * th / (2.0 * M_PI);
+            double g = (r - alpha) / (beta - alpha);
+            if (g < 0.0) g = 0.0;
+            if (g > 1.0) g = 1.0;
+            out = g * th + (1.0 - g) * th / s;
+        }
+        theta[i] = out;
+    }
+    const double m = (method == OR_YARN) ? 0.1 * log(s) + 1.0 : 1.0;
+    if (mscale) *mscale = m;
+    if (softmax_scale) *softmax_scale = m * m / sqrt((double)d);
+    return 0;
+}
+
+/*
+ * Rotate one d-vector x at (possibly fractional) position p:
+ *   [y_2i  ]   [cos(p theta_i)  -sin(p theta_i)] [x_2i  ]
+ *   [y_2i+1] = [sin(p theta_i)   cos(p theta_i)] [x_2i+1]
+ * [P3] RoPE slide (R_m,i on pair (2i, 2i+1)); [P5] "Position enters attention".
+ */
+static void rotate_vec(const double *x, double p, const double *theta, int d,
+                       double *y)
+{
+    for (int i = 0; i < d / 2; ++i) {
+        const double phi = p * theta[i];
+        const double c = cos(phi), sn = sin(phi);
+        const double a = x[2 * i], b = x[2 * i + 1];
+        y[2 * i] = a * c - b * sn;
+        y[2 * i + 1] = a * sn + b * c;
+    }
+}
+
+/* Rotate n rows of bf16 bits (row stride d) at positions pos[r]. */
+void oracle_rotate_rows(const uint16_t *x, long n, int d, const double *pos,
+                        const double *theta, double *out)
+{
+#pragma omp parallel
+    {
+        double *tmp = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(static)
+        for (long r = 0; r < n; ++r) {
+            for (int j = 0; j < d; ++j) tmp[j] = bf16_bits_to_double(x[r * d + j]);
+            rotate_vec(tmp, pos[r], theta, d, out + r * d);
+        }
+        free(tmp);
+    }
+}
+
+/* Same, for rows already in double precision. */
+void oracle_rotate_rows_f64(const double *x, long n, int d, const double *pos,
+                            const double *theta, double *out)
+{
+    for (long r = 0; r < n; ++r) rotate_vec(x + r * d, pos[r], theta, d, out + r * d);
+}
+
+/*
+ * Key n is visible to query m:
+ *   causal: n <= m  ([P3] ALiBi slide "only attend to past")
+ *   window W > 0: additionally m - n < W, or n < n_sink
+ *   ([P3] sliding-window and StreamingLLM slides; [P4] sec. 5
+ *    "always keep the first K tokens and the last W")
+ */
+static int visible(long m, long n, int causal, int window, int n_sink)
+{
+    if (causal && n > m) return 0;
+    if (window > 0 && !((m - n) < (long)window || n < (long)n_sink)) return 0;
+    return 1;
+}
+
+/*
+ * Exact attention for a list of query rows.
+ *   q [B,Hq,T,d], k and v [B,Hkv,T,d]: contiguous bf16 bit patterns.
+ *   rows: n_rows flat indices (b*Hq + h)*T + m, or NULL for every row.
+ *   For each row: q~ = R_m q, k~_n = R_n k_n, s_n = softmax_scale * q~.k~_n
+ *   over visible n, P = exp(s - max) / sum, O = sum_n P_n v_n,
+ *   LSE = max + ln(sum).   ([P3] "Q K^T / sqrt(d_k)" table slide; [P2]
+ *   key math; [P5] memory section: exact self-attention.)
+ *   o [n_rows, d], lse [n_rows] (nullable), q_rot [n_rows, d] (nullable).
+ * Returns 0, -1 on bad arguments, -2 on allocation failure.
+ */
+int oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                     int B, int Hq, int Hkv, int T, int d,
+                     const double *theta, double softmax_scale,
+                     int causal, int window, int n_sink,
+                     const int64_t *rows, long n_rows,
+                     double *o, double *lse, double *q_rot)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || T < 1 || d < 2 || (d % 2) || (Hq % Hkv)) return -1;
+    const int group = Hq / Hkv;
+    const long total = (long)B * Hq * T;
+    if (rows == NULL) n_rows = total;
+
+    /* Which (b, kv head) pairs are needed and up to which key. */
+    const long n_kv = (long)B * Hkv;
+    long *need = (long *)calloc((size_t)n_kv, sizeof(long));
+    if (!need) return -2;
+    for (long r = 0; r < n_rows; ++r) {
+        const long flat = rows ? (long)rows[r] : r;
+        if (flat < 0 || flat >= total) { free(need); return -1; }
+        const long m = flat % T, bh = flat / T;
+        const long b = bh / Hq, h = bh % Hq;
+        const long kv = b * Hkv + h / group;
+        const long last = causal ? m + 1 : T;
+        if (last > need[kv]) need[kv] = last;
+    }
+    /* Rotated keys k~_n = R_n k_n for the needed prefixes. */
+    double **krot = (double **)calloc((size_t)n_kv, sizeof(double *));
+    if (!krot) { free(need); return -2; }
+    int fail = 0;
+    for (long kv = 0; kv < n_kv; ++kv) {
+        if (need[kv] == 0) continue;
+        krot[kv] = (double *)malloc(sizeof(double) * (size_t)need[kv] * d);
+        if (!krot[kv]) { fail = 1; break; }
+    }
+    if (fail) {
+        for (long kv = 0; kv < n_kv; ++kv) free(krot[kv]);
+        free(krot); free(need);
+        return -2;
+    }
+    for (long kv = 0; kv < n_kv; ++kv) {
+        const long cnt = need[kv];
+        if (!cnt) continue;
+        const uint16_t *kb = k + kv * (long)T * d;
+        double *dst = krot[kv];
+#pragma omp parallel
+        {
+            double *tmp = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(static)
+            for (long n = 0; n < cnt; ++n) {
+                for (int j = 0; j < d; ++j) tmp[j] = bf16_bits_to_double(kb[n * d + j]);
+                rotate_vec(tmp, (double)n, theta, d, dst + n * d);
+            }
+            free(tmp);
+        }
+    }
+
+#pragma omp parallel
+    {
+        double *qv = (double *)malloc(sizeof(double) * (size_t)d);
+        double *qr = (double *)malloc(sizeof(double) * (size_t)d);
+        double *sc = (double *)malloc(sizeof(double) * (size_t)T);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 1)
+        for (long r = 0; r < n_rows; ++r) {
+            const long flat = rows ? (long)rows[r] : r;
+            const long m = flat % T, bh = flat / T;
+            const long b = bh / Hq, h = bh % Hq;
+            const long kv = b * Hkv + h / group;
+            const uint16_t *qrow = q + flat * d;
+            for (int j = 0; j < d; ++j) qv[j] = bf16_bits_to_double(qrow[j]);
+            rotate_vec(qv, (double)m, theta, d, qr);
+            if (q_rot) memcpy(q_rot + r * d, qr, sizeof(double) * (size_t)d);
+            const long kmax = causal ? m + 1 : T;
+            const double *kr = krot[kv];
+            const uint16_t *vb = v + kv * (long)T * d;
+            double mx = -INFINITY;
+            for (long n = 0; n < kmax; ++n) {
+                if (!visible(m, n, causal, window, n_sink)) { sc[n] = -INFINITY; continue; }
+                double dot = 0.0;
+                for (int j = 0; j < d; ++j) dot += qr[j] * kr[n * d + j];
+                sc[n] = softmax_scale * dot;
+                if (sc[n] > mx) mx = sc[n];
+            }
+            double z = 0.0;
+            for (int j = 0; j < d; ++j) acc[j] = 0.0;
+            for (long n = 0; n < kmax; ++n) {
+                if (sc[n] == -INFINITY) continue;
+                const double p = exp(sc[n] - mx);
+                z += p;
+                for (int j = 0; j < d; ++j) acc[j] += p * bf16_bits_to_double(vb[n * d + j]);
+            }
+            for (int j = 0; j < d; ++j) o[r * d + j] = acc[j] / z;
+            if (lse) lse[r] = mx + log(z);
+        }
+        free(qv); free(qr); free(sc); free(acc);
+    }
+    for (long kv = 0; kv < n_kv; ++kv) free(krot[kv]);
+    free(krot);
+    free(need);
+    return 0;
+}
+
+/*
+ * Single-token decode over a KV cache.
+ *   q_new [B,Hq,d]; k_new, v_new [B,Hkv,d]; caches [B,Hkv,T_max,d] whose
+ *   slots 0 .. L_b-1 hold keys that are already rotated (and values).
+ *   The new token sits at position L_b = cache_len[b]: q~ = R_L q_new,
+ *   k~ = R_L k_new; it attends over the L_b cached keys plus the new one,
+ *   with the visibility rule above taken at query position L_b.
+ *   ([P2] "decode is memory-bound on the cache"; [P1] memory wall.)
+ *   o [B,Hq,d]; lse [B,Hq]; k_rot_new [B,Hkv,d] and q_rot_new [B,Hq,d]
+ *   are nullable.  Returns 0, -1 on bad arguments, -2 on allocation failure.
+ */
+int oracle_decode(const uint16_t *q_new, const uint16_t *k_new, const uint16_t *v_new,
+                  const uint16_t *k_cache, const uint16_t *v_cache, int T_max,
+                  const int32_t *cache_len, int B, int Hq, int Hkv, int d,
+                  const double *theta, double softmax_scale, int window, int n_sink,
+                  double *o, double *lse, double *k_rot_new, double *q_rot_new)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || d < 2 || (d % 2) || (Hq % Hkv) || T_max < 1) return -1;
+    for (int b = 0; b < B; ++b)
+        if (cache_len[b] < 0 || cache_len[b] + 1 > T_max) return -1;
+    const int group = Hq / Hkv;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *x = (double *)malloc(sizeof(double) * (size_t)d);
+        double *qr = (double *)malloc(sizeof(double) * (size_t)d);
+        double *kn = (double *)malloc(sizeof(double) * (size_t)d);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)d);
+        double *sc = (double *)malloc(sizeof(double) * ((size_t)T_max + 1));
+        if (!x || !qr || !kn || !acc || !sc) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for collapse(2) schedule(dynamic, 1)
+        for (int b = 0; b < B; ++b) {
+            for (int h = 0; h < Hq; ++h) {
+                if (bad) continue;
+                const long L = cache_len[b];
+                const int kv = h / group;
+                const long qi = (long)b * Hq + h, ki = (long)b * Hkv + kv;
+                for (int j = 0; j < d; ++j) x[j] = bf16_bits_to_double(q_new[qi * d + j]);
+                rotate_vec(x, (double)L, theta, d, qr);
+                if (q_rot_new) memcpy(q_rot_new + qi * d, qr, sizeof(double) * (size_t)d);
+                for (int j = 0; j < d; ++j) x[j] = bf16_bits_to_double(k_new[ki * d + j]);
+                rotate_vec(x, (double)L, theta, d, kn);
+                if (k_rot_new && (h % group) == 0) memcpy(k_rot_new + ki * d, kn, sizeof(double) * (size_t)d);
+                const uint16_t *kc = k_cache + ki * (long)T_max * d;
+                const uint16_t *vc = v_cache + ki * (long)T_max * d;
+                double mx = -INFINITY;
+                for (long n = 0; n <= L; ++n) {
+                    if (!visible(L, n, 1, window, n_sink)) { sc[n] = -INFINITY; continue; }
+                    double dot = 0.0;
+                    if (n < L)
+                        for (int j = 0; j < d; ++j) dot += qr[j] * bf16_bits_to_double(kc[n * d + j]);
+                    else
+                        for (int j = 0; j < d; ++j) dot += qr[j] * kn[j];
+                    sc[n] = softmax_scale * dot;
+                    if (sc[n] > mx) mx = sc[n];
+                }
+                double z = 0.0;
+                for (int j = 0; j < d; ++j) acc[j] = 0.0;
+                for (long n = 0; n <= L; ++n) {
+                    if (sc[n] == -INFINITY) continue;
+                    const double p = exp(sc[n] - mx);
+                    z += p;
+                    if (n < L)
+                        for (int j = 0; j < d; ++j) acc[j] += p * bf16_bits_to_double(vc[n * d + j]);
+                    else
+                        for (int j = 0; j < d; ++j) acc[j] += p * bf16_bits_to_double(v_new[ki * d + j]);
+                }
+                for (int j = 0; j < d; ++j) o[qi * d + j] = acc[j] / z;
+                if (lse) lse[qi] = mx + log(z);
+            }
+        }
+        free(x); free(qr); free(kn); free(acc); free(sc);
+    }
+    return bad ? -2 : 0;
+}
+
+/*
+ * KV-cache bytes = 2 * n_layers * n_kv_heads * head_dim * seq_len * batch *
+ * dtype_bytes  ([P1] memory wall, kv_cache_gb; [P2] key math 2 L n_kv d_h s b p;
+ * [P5] M_KV = 2 L S H_kv D B).
+ */
+double oracle_kv_cache_bytes(double n_layers, double n_kv_heads, double head_dim,
+                             double seq_len, double batch, double dtype_bytes)
+{
+    return 2.0 * n_layers * n_kv_heads * head_dim * seq_len * batch * dtype_bytes;
+}
