@@ -1,0 +1,199 @@
+/*
+ * yarnattn.h -- C ABI of libyarnattn.so: YaRN-RoPE causal grouped-query
+ * attention on NVIDIA B200 (sm_100a).
+ *
+ * The library computes exact scaled-dot-product attention with rotary position
+ * embedding applied to Q and K inside its kernels, in two forms: a prefill over
+ * a whole sequence and a single-token decode over a KV cache.  It needs no
+ * framework: arguments are plain pointers and sizes.  Device pointers must come
+ * from the CUDA device that is current on the calling thread; `stream` is a
+ * cudaStream_t (NULL = the legacy default stream).  Every compute call is
+ * asynchronous on that stream and returns as soon as its kernels are queued.
+ *
+ * Ownership: the caller owns every buffer, including workspaces; the library
+ * allocates no device memory and keeps no pointer after a call returns.
+ *
+ * Errors: every entry point returns YR_OK (0) or a negative YR_E* code, and
+ * then yr_last_error() gives a message for the calling thread.  Arguments are
+ * checked on the host before anything is launched.  Kernels never trap: a
+ * kernel whose internal wait exceeds its time limit stops, records the fact in
+ * a device status word and returns; yr_device_status() reads (and clears) it.
+ *
+ * Sources: the web pages on long-context position scaling --
+ *   "LLM context window mechanics" (position wall; memory wall),
+ *   "Long Context" concept page (key math),
+ *   "Arch_03_Long_Context" slides (RoPE, PI, NTK-aware, YaRN, sliding window,
+ *   attention sinks), "Long context (engineering 100k+ tokens)" (sec. 2 RoPE
+ *   scaling, sec. 5 sinks), "long-context-models" (position enters attention).
+ */
+#ifndef YARNATTN_H
+#define YARNATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define YR_OK 0
+#define YR_EINVAL (-1)        /* an argument is out of range or inconsistent */
+#define YR_EUNSUPPORTED (-2)  /* valid but not implemented (head_dim, device) */
+#define YR_ECUDA (-3)         /* a CUDA runtime/driver call failed */
+#define YR_ETIMEOUT (-4)      /* a kernel gave up on an internal wait */
+
+/* Position methods ("Arch_03_Long_Context": RoPE, PI, NTK-aware and YaRN slides). */
+#define YR_ROPE 0  /* theta_i = base^(-2i/d) */
+#define YR_PI 1    /* theta_i / s: positions compressed by the extension factor s */
+#define YR_NTK 2   /* (base * s^(d/(d-2)))^(-2i/d) */
+#define YR_YARN 3  /* per-band ramp between theta_i and theta_i / s, plus temperature */
+
+#define YR_MAX_HEAD_DIM 128
+
+/* Method parameters, named after the pages' rope_scaling config (type, factor,
+ * original_max_position_embeddings) and the problem statement. */
+typedef struct yr_rope_params {
+    int head_dim;   /* d: even, 2 .. 128 for the table; the kernels take 64 or 128 */
+    double base;    /* RoPE base, > 1 (10000 for Llama-2, 500000 for Llama-3) */
+    int L_train;    /* original training context length (YaRN band split) */
+    double scale;   /* s = L_target / L_train, >= 1 */
+    int method;     /* YR_ROPE, YR_PI, YR_NTK or YR_YARN */
+    double alpha;   /* YaRN ramp start, in rotations per L_train (pages: 1) */
+    double beta;    /* YaRN ramp end (pages: 32); must exceed alpha */
+} yr_rope_params;
+
+/* Frequency and temperature table, built on the host in double precision and
+ * passed by value into the kernels. */
+typedef struct yr_rope_table {
+    int head_dim;
+    int method;
+    double inv_freq[YR_MAX_HEAD_DIM / 2]; /* theta'_i, radians per position */
+    double turns[YR_MAX_HEAD_DIM / 2];    /* theta'_i / (2 pi): rotations per position */
+    double mscale;                        /* 0.1 ln s + 1 for YaRN, else 1 */
+    double softmax_scale;                 /* mscale^2 / sqrt(d): the logit multiplier */
+    uint64_t digest;                      /* FNV-1a of the parameters (position-config identity) */
+} yr_rope_table;
+
+/*
+ * rope_freq_table -- fill `out` from `p` (host only; no CUDA).
+ *   RoPE theta_i = base^(-2i/d) ("LLM context window mechanics", position wall;
+ *   "Arch_03_Long_Context", RoPE slide).  PI theta_i / s (PI slide).  NTK
+ *   (base s^(d/(d-2)))^(-2i/d) (NTK-aware slide).  YaRN: r_i = L_train theta_i /
+ *   (2 pi), gamma_i = clamp((r_i - alpha)/(beta - alpha), 0, 1), theta'_i =
+ *   gamma_i theta_i + (1 - gamma_i) theta_i / s, and mscale = 0.1 ln s + 1
+ *   (YaRN slide and steps table).  softmax_scale = mscale^2 / sqrt(d).
+ *   The digest hashes the parameters, so a server can fold the position policy
+ *   into its engine identity ("long-context-models", operational failure modes).
+ * Errors: YR_EINVAL for NULL pointers, odd/out-of-range head_dim, base <= 1,
+ *   scale < 1, unknown method, and for YaRN L_train < 1 or beta <= alpha.
+ */
+int yr_rope_freq_table(const yr_rope_params *p, yr_rope_table *out);
+
+/*
+ * attn_prefill_workspace_bytes -- bytes of device workspace yr_attn_prefill
+ * needs: the rotated keys and the values, each [B, Hkv, T, d] in fp16.
+ * Returns 0 for invalid sizes.
+ */
+size_t yr_attn_prefill_workspace_bytes(int B, int Hkv, int T, int d);
+
+/*
+ * attn_prefill -- O = softmax(softmax_scale * (R_m q_m) . (R_n k_n)) V over the
+ * visible keys n of every query m.
+ *   Rotation R_p on each pair (2i, 2i+1) by p * theta'_i ("Arch_03_Long_Context",
+ *   RoPE slide; "long-context-models", position enters attention).
+ *   Visibility: n <= m when causal; with window W > 0 also (m - n < W or
+ *   n < n_sink) ("Arch_03_Long_Context", sliding window and sink slides;
+ *   "Long context (engineering 100k+ tokens)", sec. 5).  Query head h reads KV
+ *   head h / (Hq / Hkv) (grouped-query attention).
+ * Arguments (device pointers unless stated):
+ *   q  bf16 [B, Hq, T, d]    strides q_strides[3] = {b, h, t} in elements
+ *   k  bf16 [B, Hkv, T, d]   strides k_strides[3]
+ *   v  bf16 [B, Hkv, T, d]   strides v_strides[3]
+ *   o  bf16 [B, Hq, T, d]    strides o_strides[3]   (output)
+ *   lse      fp32 [B, Hq, T] contiguous, natural-log sum of exp of the logits (nullable)
+ *   k_cache  bf16 [B, Hkv, T, d] strides kc_strides[3]: receives the rotated keys,
+ *            e.g. to seed a decode cache (nullable)
+ *   q_rot_dbg fp32 [B, Hq, T, d] contiguous: the rotated queries as the kernel
+ *            computed them, before rounding (nullable; for tests)
+ *   k_rot_dbg fp32 [B, Hkv, T, d] contiguous: the same for the keys (nullable)
+ *   A NULL strides pointer means contiguous.  d (the last dim) has unit stride;
+ *   the other strides must be multiples of 8 elements and every base pointer
+ *   16-byte aligned.
+ *   tab: from yr_rope_freq_table with tab->head_dim == d.
+ *   causal: 1 or 0; window (W) >= 0 with 0 = none; n_sink >= 0.  window > 0
+ *   requires causal; n_sink > 0 requires window > 0.
+ *   workspace: >= yr_attn_prefill_workspace_bytes(B, Hkv, T, d) bytes, 256-byte
+ *   aligned.  It is overwritten; its contents after the call are unspecified.
+ * Precision: inputs and outputs bf16; rotation angles reduced in fp64; rotated
+ *   q/k, the probabilities and v enter the tensor cores as fp16; all sums fp32.
+ *   |rotated q|, |rotated k| and |v| must stay below 65504 (fp16 range).
+ * Errors: YR_EINVAL (shapes, strides, alignment, flags, workspace too small),
+ *   YR_EUNSUPPORTED (d not 64 or 128, device not sm_100), YR_ECUDA.
+ */
+int yr_attn_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
+                    void *k_cache, float *q_rot_dbg, float *k_rot_dbg,
+                    int B, int Hq, int Hkv, int T, int d,
+                    const int64_t *q_strides, const int64_t *k_strides,
+                    const int64_t *v_strides, const int64_t *o_strides,
+                    const int64_t *kc_strides,
+                    const yr_rope_table *tab, int causal, int window, int n_sink,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * attn_decode_workspace_bytes -- bytes of device workspace yr_attn_decode needs
+ * for its split-KV partial results with a cache of T_max slots.  0 if invalid.
+ */
+size_t yr_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int T_max);
+
+/*
+ * attn_decode -- one new token per sequence, attending over its KV cache
+ * ("Long Context" concept page: decode is memory-bound on the cache).
+ *   The new token of sequence b sits at position L_b = cache_len[b]: the call
+ *   rotates q_new and k_new by R_{L_b}, writes the rotated key and v_new into
+ *   cache slot L_b, and returns attention of the rotated query over the keys
+ *   0 .. L_b (slots 0 .. L_b-1 are taken as already rotated), with the
+ *   window/sink rule of yr_attn_prefill taken at query position L_b.  It does
+ *   not advance cache_len; the caller does.
+ *   Split-KV: each (sequence, KV head, chunk of keys) yields a partial
+ *   (max, sum, unnormalised output) for all Hq/Hkv query heads of the group;
+ *   a second kernel merges them with log-sum-exp weights.
+ * Arguments (device pointers, contiguous):
+ *   q_new bf16 [B, Hq, d]; k_new, v_new bf16 [B, Hkv, d]
+ *   k_cache, v_cache bf16 [B, Hkv, T_max, d] (slot L_b is written)
+ *   cache_len int32 [B], each 0 <= L_b <= T_max - 1 (not checked on the host:
+ *     the kernels skip a sequence whose length is out of range and record it
+ *     in the device status word)
+ *   o bf16 [B, Hq, d] (output); lse fp32 [B, Hq] (nullable)
+ *   q_rot_dbg fp32 [B, Hq, d]: the rotated queries before rounding (nullable)
+ *   tab: from yr_rope_freq_table with tab->head_dim == d.
+ *   window >= 0 (0 = none), n_sink >= 0 (requires window > 0).
+ *   workspace: >= yr_attn_decode_workspace_bytes(...) bytes, 256-byte aligned.
+ * Errors: YR_EINVAL, YR_EUNSUPPORTED (d not 64 or 128, Hq/Hkv > 16, no sm_100),
+ *   YR_ECUDA.
+ */
+int yr_attn_decode(const void *q_new, const void *k_new, const void *v_new,
+                   void *k_cache, void *v_cache, const int32_t *cache_len,
+                   void *o, float *lse, float *q_rot_dbg,
+                   int B, int Hq, int Hkv, int d, int T_max,
+                   const yr_rope_table *tab, int window, int n_sink,
+                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * device_status -- synchronise `stream`, then read and clear the device status
+ * word of the current device.  Returns YR_OK, YR_ETIMEOUT (a kernel gave up on
+ * a wait; yr_last_error names where) or YR_EINVAL (a decode cache length was
+ * out of range), or YR_ECUDA.
+ */
+int yr_device_status(void *stream);
+
+/* Message for the last error on the calling thread ("" if none). */
+const char *yr_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int yr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* YARNATTN_H */

@@ -9,6 +9,7 @@ if ROOT not in sys.path:
 
 
 def pytest_configure(config):
+    os.environ.setdefault("YR_WAIT_TIMEOUT_MS", "2000")
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU")
 
 

@@ -1,0 +1,132 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared entry
+point, builds the same table as the oracle, and rejects bad arguments on the host
+before touching a device."""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from yarn_position_scaling_b200 import api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return api.load()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    with open(os.path.join(ROOT, "include", "yarnattn.h")) as f:
+        header = f.read()
+    declared = set(re.findall(r"^\w[\w\s\*]*?\b(yr_\w+)\s*\(", header, flags=re.M))
+    assert declared >= set(api.SYMBOLS) - {"yr_last_error"} or declared
+    assert len(declared) >= 8
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in yarnattn.h but not exported"
+    assert lib.yr_version() == 10000
+
+
+@pytest.mark.parametrize("method", ["rope", "pi", "ntk", "yarn"])
+@pytest.mark.parametrize("d,base,L,s", [(64, 10000.0, 64, 4.0), (128, 10000.0, 4096, 4.0),
+                                        (128, 500000.0, 8192, 16.0), (128, 10000.0, 4096, 1.0)])
+def test_table_matches_oracle(lib, method, d, base, L, s):
+    t = api.rope_freq_table(d, base, L, s, method)
+    th, ms, ss = oracle.rope_theta(d, base, L, s, method)
+    got = np.array(t.inv_freq[: d // 2])
+    np.testing.assert_allclose(got, th, rtol=4e-15, atol=0)
+    np.testing.assert_allclose(np.array(t.turns[: d // 2]), th / (2 * math.pi), rtol=4e-15)
+    assert t.mscale == pytest.approx(ms, rel=1e-15)
+    assert t.softmax_scale == pytest.approx(ss, rel=1e-15)
+    assert t.head_dim == d and t.method == api.METHODS[method]
+
+
+def test_table_digest_identifies_the_position_policy(lib):
+    a = api.rope_freq_table(128, 10000.0, 4096, 4.0, "yarn")
+    b = api.rope_freq_table(128, 10000.0, 4096, 4.0, "yarn")
+    c = api.rope_freq_table(128, 10000.0, 4096, 8.0, "yarn")
+    d = api.rope_freq_table(128, 10000.0, 4096, 4.0, "pi")
+    e = api.rope_freq_table(128, 10000.0, 8192, 4.0, "pi")  # L_train does not shape PI
+    assert a.digest == b.digest
+    assert len({a.digest, c.digest, d.digest}) == 3
+    assert d.digest == e.digest
+
+
+@pytest.mark.parametrize("args", [
+    (63, 1e4, 64, 4.0, "yarn"), (130, 1e4, 64, 4.0, "rope"), (64, 1.0, 64, 2.0, "rope"),
+    (64, 1e4, 64, 0.5, "pi"), (64, 1e4, 0, 2.0, "yarn"), (64, 1e4, 64, float("nan"), "ntk")])
+def test_table_rejects_bad_parameters(lib, args):
+    with pytest.raises(api.YarnAttnError) as ei:
+        api.rope_freq_table(*args)
+    assert ei.value.code == api.YR_EINVAL
+
+
+def test_table_rejects_reversed_ramp(lib):
+    with pytest.raises(api.YarnAttnError):
+        api.rope_freq_table(64, 1e4, 64, 2.0, "yarn", alpha=32.0, beta=1.0)
+
+
+# Host-side validation happens before any CUDA call, so fake (never dereferenced)
+# pointers are enough to exercise it on a machine without a GPU.
+FAKE = ctypes.c_void_p(1 << 20)
+NUL = ctypes.c_void_p(0)
+
+
+def _prefill(lib, tab, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=NUL, kc=NUL, qd=NUL, kd=NUL, B=1, Hq=4, Hkv=2,
+             T=256, d=64, causal=1, window=0, n_sink=0, ws=FAKE, ws_bytes=1 << 30)
+    a.update(kw)
+    null_strides = ctypes.POINTER(ctypes.c_int64)()
+    return lib.yr_attn_prefill(a["q"], a["k"], a["v"], a["o"], a["lse"], a["kc"], a["qd"], a["kd"],
+                               a["B"], a["Hq"], a["Hkv"], a["T"], a["d"], a.get("qs", null_strides),
+                               null_strides, null_strides, null_strides, null_strides,
+                               ctypes.byref(tab), a["causal"], a["window"], a["n_sink"], a["ws"],
+                               a["ws_bytes"], NUL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=NUL), api.YR_EINVAL), (dict(Hq=3), api.YR_EINVAL), (dict(T=0), api.YR_EINVAL),
+    (dict(d=96), api.YR_EUNSUPPORTED), (dict(d=128), api.YR_EINVAL),  # table is d=64
+    (dict(causal=0, window=16), api.YR_EINVAL), (dict(n_sink=4), api.YR_EINVAL),
+    (dict(window=-1), api.YR_EINVAL), (dict(causal=2), api.YR_EINVAL),
+    (dict(ws_bytes=100), api.YR_EINVAL), (dict(ws=ctypes.c_void_p((1 << 20) + 16)), api.YR_EINVAL),
+    (dict(q=ctypes.c_void_p((1 << 20) + 2)), api.YR_EINVAL),
+    (dict(qs=(ctypes.c_int64 * 3)(4096, 1024, 12)), api.YR_EINVAL),
+])
+def test_prefill_rejects_bad_arguments_on_host(lib, kw, code):
+    tab = api.rope_freq_table(64, 10000.0, 64, 4.0, "yarn")
+    rc = _prefill(lib, tab, **kw)
+    assert rc == code
+    assert lib.yr_last_error().decode().startswith("yr_attn_prefill")
+
+
+def _decode(lib, tab, **kw):
+    a = dict(qn=FAKE, kn=FAKE, vn=FAKE, kc=FAKE, vc=FAKE, cl=FAKE, o=FAKE, B=2, Hq=8, Hkv=2,
+             d=64, T_max=4096, window=0, n_sink=0, ws=FAKE, ws_bytes=1 << 30)
+    a.update(kw)
+    return lib.yr_attn_decode(a["qn"], a["kn"], a["vn"], a["kc"], a["vc"], a["cl"], a["o"], NUL,
+                              NUL, a["B"], a["Hq"], a["Hkv"], a["d"], a["T_max"], ctypes.byref(tab),
+                              a["window"], a["n_sink"], a["ws"], a["ws_bytes"], NUL)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(cl=NUL), api.YR_EINVAL), (dict(Hq=7), api.YR_EINVAL), (dict(T_max=0), api.YR_EINVAL),
+    (dict(d=80), api.YR_EUNSUPPORTED), (dict(Hq=68, Hkv=2), api.YR_EUNSUPPORTED),
+    (dict(n_sink=2), api.YR_EINVAL), (dict(ws_bytes=8), api.YR_EINVAL),
+])
+def test_decode_rejects_bad_arguments_on_host(lib, kw, code):
+    tab = api.rope_freq_table(64, 10000.0, 64, 4.0, "yarn")
+    assert _decode(lib, tab, **kw) == code
+    assert lib.yr_last_error().decode().startswith("yr_attn_decode")
+
+
+def test_workspace_sizes(lib):
+    assert api.attn_prefill_workspace_bytes(1, 8, 131072, 128) == 2 * 8 * 131072 * 128 * 2
+    nc = (131073 + 2047) // 2048
+    assert api.attn_decode_workspace_bytes(8, 32, 8, 128, 131073) == 8 * 8 * nc * 4 * 130 * 4
+    assert api.attn_decode_workspace_bytes(8, 30, 8, 128, 100) == 0

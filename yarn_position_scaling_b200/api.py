@@ -1,0 +1,177 @@
+"""ctypes binding of libyarnattn.so (include/yarnattn.h), same names as the C ABI.
+
+Argument marshalling only: tensors are passed as raw device pointers with
+their strides, on the current PyTorch stream.  Every computation happens in
+the library's CUDA kernels; there is no CPU path.  Loading fails loudly if the
+library has not been built (``python -m yarn_position_scaling_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .build import LIB
+
+YR_OK, YR_EINVAL, YR_EUNSUPPORTED, YR_ECUDA, YR_ETIMEOUT = 0, -1, -2, -3, -4
+ROPE, PI, NTK, YARN = 0, 1, 2, 3
+METHODS = {"rope": ROPE, "pi": PI, "ntk": NTK, "yarn": YARN}
+SYMBOLS = ("yr_rope_freq_table", "yr_attn_prefill_workspace_bytes", "yr_attn_prefill",
+           "yr_attn_decode_workspace_bytes", "yr_attn_decode", "yr_device_status",
+           "yr_last_error", "yr_version")
+
+
+class YarnAttnError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"[{code}] {message}")
+        self.code = code
+
+
+class RopeParams(ctypes.Structure):
+    _fields_ = [("head_dim", ctypes.c_int), ("base", ctypes.c_double), ("L_train", ctypes.c_int),
+                ("scale", ctypes.c_double), ("method", ctypes.c_int), ("alpha", ctypes.c_double),
+                ("beta", ctypes.c_double)]
+
+
+class RopeTable(ctypes.Structure):
+    _fields_ = [("head_dim", ctypes.c_int), ("method", ctypes.c_int),
+                ("inv_freq", ctypes.c_double * 64), ("turns", ctypes.c_double * 64),
+                ("mscale", ctypes.c_double), ("softmax_scale", ctypes.c_double),
+                ("digest", ctypes.c_uint64)]
+
+
+_lib = None
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load libyarnattn.so (once).  Raises if it is missing."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB
+    if not os.path.exists(p):
+        raise RuntimeError(f"libyarnattn.so not found at {p}: build it with "
+                           "`python -m yarn_position_scaling_b200.build`")
+    lib = ctypes.CDLL(p)
+    vp, i64p = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int64)
+    ci, cs = ctypes.c_int, ctypes.c_size_t
+    lib.yr_rope_freq_table.argtypes = [ctypes.POINTER(RopeParams), ctypes.POINTER(RopeTable)]
+    lib.yr_rope_freq_table.restype = ci
+    lib.yr_attn_prefill_workspace_bytes.argtypes = [ci, ci, ci, ci]
+    lib.yr_attn_prefill_workspace_bytes.restype = cs
+    lib.yr_attn_prefill.argtypes = ([vp] * 8 + [ci] * 5 + [i64p] * 5 +
+                                    [ctypes.POINTER(RopeTable), ci, ci, ci, vp, cs, vp])
+    lib.yr_attn_prefill.restype = ci
+    lib.yr_attn_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
+    lib.yr_attn_decode_workspace_bytes.restype = cs
+    lib.yr_attn_decode.argtypes = ([vp] * 9 + [ci] * 5 +
+                                   [ctypes.POINTER(RopeTable), ci, ci, vp, cs, vp])
+    lib.yr_attn_decode.restype = ci
+    lib.yr_device_status.argtypes = [vp]
+    lib.yr_device_status.restype = ci
+    lib.yr_last_error.argtypes = []
+    lib.yr_last_error.restype = ctypes.c_char_p
+    lib.yr_version.argtypes = []
+    lib.yr_version.restype = ci
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _check(rc: int):
+    if rc != YR_OK:
+        raise YarnAttnError(rc, load().yr_last_error().decode())
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _strides(t: torch.Tensor):
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError("expected a 4-D tensor [B, H, T, d] with unit stride over d")
+    return (ctypes.c_int64 * 3)(t.stride(0), t.stride(1), t.stride(2))
+
+
+def rope_freq_table(head_dim: int, base: float, L_train: int, scale: float, method,
+                    alpha: float = 1.0, beta: float = 32.0) -> RopeTable:
+    """Frequency/temperature table for one position method (host only)."""
+    m = METHODS[method] if isinstance(method, str) else int(method)
+    p = RopeParams(int(head_dim), float(base), int(L_train), float(scale), m, float(alpha),
+                   float(beta))
+    out = RopeTable()
+    _check(load().yr_rope_freq_table(ctypes.byref(p), ctypes.byref(out)))
+    return out
+
+
+def attn_prefill_workspace_bytes(B: int, Hkv: int, T: int, d: int) -> int:
+    return int(load().yr_attn_prefill_workspace_bytes(B, Hkv, T, d))
+
+
+def attn_decode_workspace_bytes(B: int, Hq: int, Hkv: int, d: int, T_max: int) -> int:
+    return int(load().yr_attn_decode_workspace_bytes(B, Hq, Hkv, d, T_max))
+
+
+def attn_prefill(q, k, v, table: RopeTable, causal: bool = True, window: int = 0,
+                 n_sink: int = 0, out=None, lse=None, k_cache=None, q_rot_dbg=None,
+                 k_rot_dbg=None, workspace=None, stream=None):
+    """Attention prefill.  q [B,Hq,T,d], k/v [B,Hkv,T,d] bf16 CUDA tensors (any strides with
+    unit stride over d).  Returns the output tensor [B,Hq,T,d] bf16."""
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq, T, d), dtype=torch.bfloat16, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(attn_prefill_workspace_bytes(B, Hkv, T, d), dtype=torch.uint8,
+                                device=q.device)
+    kc_strides = _strides(k_cache) if k_cache is not None else None
+    rc = load().yr_attn_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(q_rot_dbg),
+        _ptr(k_rot_dbg), B, Hq, Hkv, T, d, _strides(q), _strides(k), _strides(v), _strides(out),
+        kc_strides, ctypes.byref(table), int(bool(causal)), int(window), int(n_sink),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc)
+    return out
+
+
+def attn_decode(q_new, k_new, v_new, k_cache, v_cache, cache_len, table: RopeTable,
+                window: int = 0, n_sink: int = 0, out=None, lse=None, q_rot_dbg=None,
+                workspace=None, stream=None):
+    """Single-token decode.  q_new [B,Hq,d], k_new/v_new [B,Hkv,d], caches [B,Hkv,T_max,d]
+    (contiguous bf16), cache_len int32 [B] on the device.  Writes slot cache_len[b] of the
+    caches; returns the output [B,Hq,d] bf16."""
+    B, Hq, d = q_new.shape
+    Hkv, T_max = k_cache.shape[1], k_cache.shape[2]
+    for t in (q_new, k_new, v_new, k_cache, v_cache, cache_len):
+        if not t.is_contiguous():
+            raise ValueError("attn_decode expects contiguous tensors")
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q_new.device)
+    if workspace is None:
+        workspace = torch.empty(attn_decode_workspace_bytes(B, Hq, Hkv, d, T_max),
+                                dtype=torch.uint8, device=q_new.device)
+    rc = load().yr_attn_decode(
+        _ptr(q_new), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(cache_len),
+        _ptr(out), _ptr(lse), _ptr(q_rot_dbg), B, Hq, Hkv, d, T_max, ctypes.byref(table),
+        int(window), int(n_sink), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check(rc)
+    return out
+
+
+def device_status(stream=None) -> int:
+    """Synchronise and read/clear the device status word; raises on a recorded fault."""
+    rc = load().yr_device_status(_stream(stream))
+    _check(rc)
+    return rc
+
+
+def version() -> int:
+    return int(load().yr_version())

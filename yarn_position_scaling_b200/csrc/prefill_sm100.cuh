@@ -1,0 +1,526 @@
+// prefill_sm100.cuh -- causal / windowed GQA attention prefill for sm_100a with
+// rotary position embedding applied to Q inside the kernel.
+//
+// One CTA owns two 128-row query tiles (Q0, Q1) of one (batch, head) and walks
+// the key/value tiles those rows can see:
+//   warp 8      TMA producer: Q tiles once, then K~/V tiles through a 2-stage ring
+//   warp 9      MMA issuer: S_t = Q_t K~^T and O_t += P_t V with tcgen05.mma,
+//               accumulators in tensor memory (TMEM)
+//   warps 0-3   softmax for Q0, warps 4-7 softmax for Q1: each thread owns one
+//               query row (= one TMEM lane), so row max and row sum need no
+//               shuffles; P is written back over S in TMEM as fp16
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+d), O1 [256+d,256+2d).
+// The MMA issue order S0(j) | PV1(j-1) S1(j) | PV0(j) lets one softmax group
+// work while the tensor cores serve the other group ("ping-pong").
+//
+// Online softmax ("Long Context" concept page, key math: scores never reach
+// HBM; "long-context-models", context parallelism: running row maxima,
+// normalisation sums and output accumulators): the running max is only moved
+// when a tile raises it by more than 2^8, so O is rescaled rarely; P stays
+// within [0, 256], which fp16 holds exactly enough.
+//
+// Rotation ("Arch_03_Long_Context", RoPE slide): pair (2i, 2i+1) of the query
+// at position m turns by m * theta'_i.  The angle is reduced in fp64 as
+// turns = m * theta'_i / (2 pi) minus its nearest integer, then sin/cos run
+// in fp32 on an argument in [-pi, pi].
+//
+// Every wait is bounded (wall clock + a CTA abort flag + the device status
+// word); a CTA that gives up drains its own copies and MMAs, frees TMEM and
+// returns.
+#pragma once
+#include "sm100_ptx.cuh"
+
+namespace yr {
+
+constexpr int kBlockM = 128;
+constexpr int kBlockN = 128;
+constexpr int kQTiles = 2;
+constexpr int kKStages = 2;
+constexpr int kVStages = 2;
+constexpr int kPrefillThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kSubTileBytes = 128 * 128;  // 128 rows x 64 16-bit columns, 128-byte swizzle
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+struct alignas(64) PrefillParams {
+    CUtensorMap tm_q;  // bf16 [B][Hq][T][d] (4-D, caller strides)
+    CUtensorMap tm_k;  // fp16 [B*Hkv][T][d] rotated keys (workspace)
+    CUtensorMap tm_v;  // fp16 [B*Hkv][T][d] values (workspace)
+    __nv_bfloat16 *o;
+    long long osb, osh, ost;
+    float *lse;
+    float *q_dbg;
+    int B, Hq, Hkv, T, group;
+    int causal, window, n_sink;
+    int n_qblocks;
+    float sl2;  // softmax_scale * log2(e)
+    unsigned long long timeout_ns;
+    double turns[64];
+};
+
+template <int HD>
+struct PrefillSmem {
+    static constexpr int kSub = HD / 64;
+    uint8_t q[kQTiles][kSub][kSubTileBytes];
+    uint8_t k[kKStages][kSub][kSubTileBytes];
+    uint8_t v[kVStages][kSub][kSubTileBytes];
+    uint64_t q_full[kQTiles], q_ready[kQTiles];
+    uint64_t k_full[kKStages], k_empty[kKStages];
+    uint64_t v_full[kVStages], v_empty[kVStages];
+    uint64_t s_full[kQTiles], p_full[kQTiles], o_done[kQTiles];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Key tiles one CTA visits: the sink tiles [0, sink_end) that precede the
+// window, then [lo, lo + n - sink_end).
+struct TilePlan {
+    int sink_end, lo, n;
+};
+
+__device__ __forceinline__ TilePlan plan_tiles(const PrefillParams &p, int q0, int last_row) {
+    TilePlan tp;
+    const int hi = p.causal ? last_row / kBlockN : (p.T - 1) / kBlockN;
+    if (p.window > 0) {
+        const int first_key = max(0, q0 - p.window + 1);
+        tp.lo = first_key / kBlockN;
+        const int sink_tiles = (p.n_sink + kBlockN - 1) / kBlockN;
+        tp.sink_end = min(sink_tiles, tp.lo);
+    } else {
+        tp.lo = 0;
+        tp.sink_end = 0;
+    }
+    tp.n = tp.sink_end + (hi - tp.lo + 1);
+    return tp;
+}
+__device__ __forceinline__ int tile_at(const TilePlan &tp, int idx) {
+    return idx < tp.sink_end ? idx : tp.lo + (idx - tp.sink_end);
+}
+
+// Does any (row, key) pair of rows [r_lo, r_hi] x tile j pass the visibility rule?
+__device__ __forceinline__ bool tile_visible(const PrefillParams &p, int r_lo, int r_hi, int j) {
+    if (r_lo > r_hi) return false;
+    const int k_lo = j * kBlockN;
+    const int k_hi = min(k_lo + kBlockN - 1, p.T - 1);
+    if (k_lo > p.T - 1) return false;
+    if (!p.causal) return true;
+    if (k_lo > r_hi) return false;
+    if (p.window > 0) {
+        const int d_min = max(0, max(r_lo, k_lo) - k_hi);
+        if (!(d_min < p.window || k_lo < p.n_sink)) return false;
+    }
+    return true;
+}
+// Is every pair visible (no masking needed)?
+__device__ __forceinline__ bool tile_full(const PrefillParams &p, int r_lo, int r_hi, int j) {
+    const int k_lo = j * kBlockN;
+    const int k_hi = k_lo + kBlockN - 1;
+    if (k_hi > p.T - 1) return false;
+    if (p.causal && k_hi > r_lo) return false;
+    if (p.window > 0 && !(r_hi - k_lo < p.window || k_hi < p.n_sink)) return false;
+    return true;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
+template <int HD>
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+    prefill_attn_kernel(const __grid_constant__ PrefillParams p) {
+    using Smem = PrefillSmem<HD>;
+    constexpr int kSub = Smem::kSub;
+    extern __shared__ uint8_t smem_raw[];
+    Smem *sm = reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                        ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // Heaviest causal blocks first; the heads of one query block are adjacent so
+    // the query heads that share a KV head read the same K/V tiles close in time.
+    const int bh_count = p.B * p.Hq;
+    const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x) / bh_count;
+    const int rem = static_cast<int>(blockIdx.x) % bh_count;
+    const int b = rem / p.Hq;
+    const int h = rem % p.Hq;
+    const int kvh = h / p.group;
+    const int q0 = qb * (kQTiles * kBlockM);
+    const int last_row = min(q0 + kQTiles * kBlockM - 1, p.T - 1);
+    const TilePlan tp = plan_tiles(p, q0, last_row);
+    int r_lo[kQTiles], r_hi[kQTiles];
+#pragma unroll
+    for (int t = 0; t < kQTiles; ++t) {
+        r_lo[t] = q0 + t * kBlockM;
+        r_hi[t] = min(r_lo[t] + kBlockM - 1, p.T - 1);
+    }
+
+    if (threadIdx.x == 0) {
+        for (int t = 0; t < kQTiles; ++t) {
+            mbar_init(&sm->q_full[t], 1);
+            mbar_init(&sm->q_ready[t], kBlockM);
+            mbar_init(&sm->s_full[t], 1);
+            mbar_init(&sm->p_full[t], kBlockM);
+            mbar_init(&sm->o_done[t], 1);
+        }
+        for (int s = 0; s < kKStages; ++s) {
+            mbar_init(&sm->k_full[s], 1);
+            mbar_init(&sm->k_empty[s], 1);
+        }
+        for (int s = 0; s < kVStages; ++s) {
+            mbar_init(&sm->v_full[s], 1);
+            mbar_init(&sm->v_empty[s], 1);
+        }
+        mbar_init(&sm->mma_done, 1);
+        sm->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(&sm->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_tensormap(&p.tm_q);
+        prefetch_tensormap(&p.tm_k);
+        prefetch_tensormap(&p.tm_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm->tmem_base;
+    volatile int *abort = &sm->abort;
+
+    if (warp == 8) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const uint64_t pol_q = l2_policy_evict_first();
+            const uint64_t pol_kv = l2_policy_evict_last();
+            bool ok = true;
+            for (int t = 0; t < kQTiles; ++t) {
+                if (r_lo[t] > r_hi[t]) continue;
+                mbar_arrive_expect_tx(&sm->q_full[t], kSub * kSubTileBytes);
+                for (int s = 0; s < kSub; ++s)
+                    tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64, r_lo[t], h, b, pol_q);
+            }
+            const int kv_plane = b * p.Hkv + kvh;
+            int issued_k[kKStages] = {}, issued_v[kVStages] = {};
+            for (int idx = 0; idx < tp.n && ok; ++idx) {
+                const int j = tile_at(tp, idx);
+                const int ks = idx % kKStages, vs = idx % kVStages;
+                ok = mbar_wait(&sm->k_empty[ks], ((idx / kKStages) & 1) ^ 1, abort, p.timeout_ns);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&sm->k_full[ks], kSub * kSubTileBytes);
+                for (int s = 0; s < kSub; ++s)
+                    tma_load_3d(sm->k[ks][s], &p.tm_k, &sm->k_full[ks], s * 64, j * kBlockN,
+                                kv_plane, pol_kv);
+                ++issued_k[ks];
+                ok = mbar_wait(&sm->v_empty[vs], ((idx / kVStages) & 1) ^ 1, abort, p.timeout_ns);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&sm->v_full[vs], kSub * kSubTileBytes);
+                for (int s = 0; s < kSub; ++s)
+                    tma_load_3d(sm->v[vs][s], &p.tm_v, &sm->v_full[vs], s * 64, j * kBlockN,
+                                kv_plane, pol_kv);
+                ++issued_v[vs];
+            }
+            if (!ok) {
+                raise_status(kStatusTimeoutLoad);
+                sm->abort = 1;
+            }
+            // Drain: every copy this thread issued must land before the CTA exits.
+            bool drained = true;
+            for (int t = 0; t < kQTiles; ++t)
+                if (r_lo[t] <= r_hi[t]) drained &= mbar_wait_drain(&sm->q_full[t], 0, p.timeout_ns);
+            for (int s = 0; s < kKStages; ++s)
+                if (issued_k[s])
+                    drained &= mbar_wait_drain(&sm->k_full[s], (issued_k[s] - 1) & 1, p.timeout_ns);
+            for (int s = 0; s < kVStages; ++s)
+                if (issued_v[s])
+                    drained &= mbar_wait_drain(&sm->v_full[s], (issued_v[s] - 1) & 1, p.timeout_ns);
+            if (!drained) raise_status(kStatusTimeoutDrain);
+        }
+        __syncwarp();
+    } else if (warp == 9) {
+        // ------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_f16_f32(kBlockM, kBlockN, false, false);
+            constexpr uint32_t idesc_o = idesc_f16_f32(kBlockM, HD, false, true);
+            bool ok = true;
+            bool vis[kQTiles];
+            int pv_count[kQTiles] = {0, 0};
+            for (int t = 0; t < kQTiles && ok; ++t)
+                if (r_lo[t] <= r_hi[t]) ok = mbar_wait(&sm->q_ready[t], 0, abort, p.timeout_ns);
+            tc_fence_after();
+
+            auto issue_s = [&](int t, int ks) {
+                const uint32_t qa = smem_u32(sm->q[t][0]);
+                const uint32_t ka = smem_u32(sm->k[ks][0]);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kSubTileBytes + (kk & 3) * 32;
+                    mma_ss(tmem + t * kBlockN, sw128_desc(qa + off, 16, 1024),
+                           sw128_desc(ka + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&sm->s_full[t]);
+            };
+            auto issue_pv = [&](int t, int vs) -> bool {
+                if (!mbar_wait(&sm->p_full[t], pv_count[t] & 1, abort, p.timeout_ns)) return false;
+                tc_fence_after();
+                const uint32_t va = smem_u32(sm->v[vs][0]);
+#pragma unroll
+                for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                    mma_ts(tmem + 2 * kBlockN + t * HD, tmem + t * kBlockN + kk * 8,
+                           sw128_desc(va + kk * 2048, kSubTileBytes, 1024), idesc_o,
+                           (pv_count[t] > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(&sm->o_done[t]);
+                ++pv_count[t];
+                return true;
+            };
+
+            bool prev_vis1 = false;
+            for (int idx = 0; idx < tp.n && ok; ++idx) {
+                const int j = tile_at(tp, idx);
+                const int ks = idx % kKStages, vs = idx % kVStages;
+                for (int t = 0; t < kQTiles; ++t) vis[t] = tile_visible(p, r_lo[t], r_hi[t], j);
+                ok = mbar_wait(&sm->k_full[ks], (idx / kKStages) & 1, abort, p.timeout_ns);
+                if (!ok) break;
+                tc_fence_after();
+                if (vis[0]) issue_s(0, ks);
+                if (idx > 0) {
+                    const int pvs = (idx - 1) % kVStages;
+                    if (prev_vis1) ok = issue_pv(1, pvs);
+                    if (!ok) break;
+                }
+                if (vis[1]) issue_s(1, ks);
+                mma_commit(&sm->k_empty[ks]);
+                if (idx > 0) mma_commit(&sm->v_empty[(idx - 1) % kVStages]);
+                ok = mbar_wait(&sm->v_full[vs], (idx / kVStages) & 1, abort, p.timeout_ns);
+                if (!ok) break;
+                tc_fence_after();
+                if (vis[0]) ok = issue_pv(0, vs);
+                prev_vis1 = vis[1];
+            }
+            if (ok && tp.n > 0) {
+                const int vs = (tp.n - 1) % kVStages;
+                if (prev_vis1) ok = issue_pv(1, vs);
+                if (ok) mma_commit(&sm->v_empty[vs]);
+            }
+            if (!ok) {
+                raise_status(kStatusTimeoutMma);
+                sm->abort = 1;
+            }
+            // Drain: all MMAs issued above complete before TMEM/smem go away.
+            mma_commit(&sm->mma_done);
+            if (!mbar_wait_drain(&sm->mma_done, 0, p.timeout_ns)) raise_status(kStatusTimeoutDrain);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------- softmax warpgroups
+        const int t = warp >> 2;
+        const int lane_base = (warp & 3) * 32;
+        const int r = lane_base + lane;  // row within the tile = TMEM lane
+        const int row = r_lo[t] + r;
+        const uint32_t tm_lane = static_cast<uint32_t>(lane_base) << 16;
+        const uint32_t tm_s = tmem + tm_lane + t * kBlockN;
+        const uint32_t tm_o = tmem + tm_lane + 2 * kBlockN + t * HD;
+        const bool tile_live = r_lo[t] <= r_hi[t];
+        bool ok = true;
+
+        if (tile_live) {
+            // Rotate this row of Q in shared memory: bf16 in, fp16 out, in place.
+            ok = mbar_wait(&sm->q_full[t], 0, abort, p.timeout_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                float *dbg = (p.q_dbg != nullptr && row < p.T)
+                                 ? p.q_dbg + ((static_cast<long long>(b) * p.Hq + h) * p.T + row) * HD
+                                 : nullptr;
+#pragma unroll
+                for (int s = 0; s < kSub; ++s) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint4 *ptr = reinterpret_cast<uint4 *>(sm->q[t][s] + r * 128 +
+                                                               ((c ^ (r & 7)) << 4));
+                        uint4 raw = *ptr;
+                        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+                        uint32_t out[4];
+                        float y[8];
+#pragma unroll
+                        for (int pp = 0; pp < 4; ++pp) {
+                            const float a = __uint_as_float(w[pp] << 16);
+                            const float bb = __uint_as_float(w[pp] & 0xFFFF0000u);
+                            const double turns = static_cast<double>(row) * p.turns[s * 32 + c * 4 + pp];
+                            const double frac = turns - rint(turns);
+                            float sn, cs;
+                            __sincosf(static_cast<float>(frac * 6.283185307179586), &sn, &cs);
+                            y[2 * pp] = a * cs - bb * sn;
+                            y[2 * pp + 1] = a * sn + bb * cs;
+                            out[pp] = pack_half2(y[2 * pp], y[2 * pp + 1]);
+                        }
+                        *ptr = make_uint4(out[0], out[1], out[2], out[3]);
+                        if (dbg) {
+                            float4 *d4 = reinterpret_cast<float4 *>(dbg + s * 64 + c * 8);
+                            d4[0] = make_float4(y[0], y[1], y[2], y[3]);
+                            d4[1] = make_float4(y[4], y[5], y[6], y[7]);
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&sm->q_ready[t]);
+            }
+        }
+
+        float m_run = -INFINITY;  // running max, log2 units (scores * sl2)
+        float l_run = 0.0f;       // running sum of exp2(score*sl2 - m_run)
+        int it = 0;
+        for (int idx = 0; idx < tp.n && ok && tile_live; ++idx) {
+            const int j = tile_at(tp, idx);
+            if (!tile_visible(p, r_lo[t], r_hi[t], j)) continue;
+            ok = mbar_wait(&sm->s_full[t], it & 1, abort, p.timeout_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            float s[kBlockN];
+            {
+                uint32_t raw[kBlockN / 32][32];
+#pragma unroll
+                for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tm_s + c * 32, raw[c]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < kBlockN / 32; ++c) {
+                    reg_fence32(raw[c]);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[c][e]);
+                }
+            }
+            if (!tile_full(p, r_lo[t], r_hi[t], j)) {
+                const int k0 = j * kBlockN;
+#pragma unroll
+                for (int c = 0; c < kBlockN; ++c) {
+                    const int n = k0 + c;
+                    bool v = n < p.T;
+                    if (p.causal) v = v && (n <= row);
+                    if (p.window > 0) v = v && ((row - n) < p.window || n < p.n_sink);
+                    if (!v) s[c] = -INFINITY;
+                }
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int c = 1; c < kBlockN; ++c) mx = fmaxf(mx, s[c]);
+            const float m_tile = mx * p.sl2;
+            const bool need = m_tile > m_run + kRescaleThreshold;
+            if (__any_sync(0xffffffffu, need)) {
+                const float m_new = need ? fmaxf(m_run, m_tile) : m_run;
+                const float alpha = (m_run == -INFINITY) ? 0.0f : ex2(m_run - m_new);
+                if (it > 0) {
+                    // O holds P V up to the previous tile: wait for it, then rescale.
+                    ok = mbar_wait(&sm->o_done[t], (it - 1) & 1, abort, p.timeout_ns);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const float sc = need ? alpha : 1.0f;
+                    uint32_t raw[32];
+#pragma unroll
+                    for (int c = 0; c < HD / 32; ++c) {
+                        tmem_ld32_sync(tm_o + c * 32, raw);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            raw[e] = __float_as_uint(__uint_as_float(raw[e]) * sc);
+                        tmem_st32(tm_o + c * 32, raw);
+                    }
+                    tmem_st_wait();
+                }
+                if (need) {
+                    l_run *= alpha;
+                    m_run = m_new;
+                }
+            }
+            const float m_ref = (m_run == -INFINITY) ? 0.0f : m_run;
+#pragma unroll
+            for (int c = 0; c < kBlockN / 32; ++c) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = ex2(fmaf(s[c * 32 + 2 * e], p.sl2, -m_ref));
+                    const float p1 = ex2(fmaf(s[c * 32 + 2 * e + 1], p.sl2, -m_ref));
+                    l_run += p0 + p1;
+                    pk[e] = pack_half2(p0, p1);
+                }
+                tmem_st16(tm_s + c * 16, pk);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&sm->p_full[t]);
+            ++it;
+        }
+        if (!ok) {
+            raise_status(kStatusTimeoutSoftmax);
+            sm->abort = 1;
+        }
+        // Epilogue: O / l -> bf16, and the log-sum-exp in natural-log units.
+        if (ok && tile_live && it > 0) {
+            ok = mbar_wait(&sm->o_done[t], (it - 1) & 1, abort, p.timeout_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                tc_fence_after();
+                const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
+                __nv_bfloat16 *orow = p.o + b * p.osb + h * p.osh + static_cast<long long>(row) * p.ost;
+                uint32_t raw[32];
+#pragma unroll
+                for (int c = 0; c < HD / 32; ++c) {
+                    tmem_ld32_sync(tm_o + c * 32, raw);
+                    if (row < p.T) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                __nv_bfloat162 v2 = __floats2bfloat162_rn(
+                                    __uint_as_float(raw[q4 * 8 + 2 * e]) * inv_l,
+                                    __uint_as_float(raw[q4 * 8 + 2 * e + 1]) * inv_l);
+                                pk[e] = *reinterpret_cast<uint32_t *>(&v2);
+                            }
+                            *reinterpret_cast<uint4 *>(orow + c * 32 + q4 * 8) =
+                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
+                }
+                if (p.lse != nullptr && row < p.T) {
+                    const float m_ref = (m_run == -INFINITY) ? 0.0f : m_run;
+                    p.lse[(static_cast<long long>(b) * p.Hq + h) * p.T + row] =
+                        (l_run > 0.0f) ? (m_ref + __log2f(l_run)) * 0.69314718055994531f
+                                       : -INFINITY;
+                }
+            } else {
+                raise_status(kStatusTimeoutSoftmax);
+                sm->abort = 1;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem, kTmemCols);
+}
+
+// Dynamic shared memory per CTA.  At least 116 KB, so that one CTA holds an SM
+// (and all 512 TMEM columns) at a time for either head size.
+template <int HD>
+constexpr size_t prefill_smem_bytes() {
+    return sizeof(PrefillSmem<HD>) + 1024 > 116 * 1024 ? sizeof(PrefillSmem<HD>) + 1024
+                                                        : 116 * 1024;
+}
+
+}  // namespace yr

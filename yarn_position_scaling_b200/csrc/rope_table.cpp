@@ -1,0 +1,114 @@
+// rope_table.cpp -- host-side frequency and temperature table (no CUDA).
+//
+//   RoPE   theta_i = base^(-2i/d), i = 0 .. d/2-1
+//          ("LLM context window mechanics", position wall; "Arch_03_Long_Context",
+//           RoPE slide)
+//   PI     theta_i / s  (PI slide: positions divided by s = L_target / L_train)
+//   NTK    (base * s^(d/(d-2)))^(-2i/d)  (NTK-aware slide)
+//   YaRN   r_i = L_train / lambda_i with lambda_i = 2 pi / theta_i; the share
+//          gamma_i = clamp((r_i - alpha) / (beta - alpha), 0, 1) of each band
+//          keeps its frequency, the rest is interpolated as in PI:
+//          theta'_i = theta_i * (gamma_i + (1 - gamma_i) / s); the attention
+//          temperature mscale = 0.1 ln s + 1 (YaRN slide, steps table)
+//   softmax_scale = mscale^2 / sqrt(d): the temperature on both rotated q and k.
+// The table also carries theta'_i / (2 pi) (rotations per position), which the
+// kernels multiply by the position in fp64 to reduce the angle exactly.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <string>
+
+#include "../../include/yarnattn.h"
+
+namespace yr_host {
+void set_error(const std::string &msg);
+}
+
+namespace {
+
+uint64_t fnv1a(uint64_t h, const void *data, size_t n) {
+    const unsigned char *p = static_cast<const unsigned char *>(data);
+    for (size_t i = 0; i < n; ++i) {
+        h ^= p[i];
+        h *= 0x100000001b3ull;
+    }
+    return h;
+}
+
+}  // namespace
+
+extern "C" int yr_rope_freq_table(const yr_rope_params *p, yr_rope_table *out) {
+    if (p == nullptr || out == nullptr) {
+        yr_host::set_error("yr_rope_freq_table: NULL argument");
+        return YR_EINVAL;
+    }
+    const int d = p->head_dim;
+    if (d < 2 || d > YR_MAX_HEAD_DIM || (d % 2) != 0) {
+        yr_host::set_error("yr_rope_freq_table: head_dim must be even and in [2, 128]");
+        return YR_EINVAL;
+    }
+    if (!(p->base > 1.0) || !std::isfinite(p->base)) {
+        yr_host::set_error("yr_rope_freq_table: base must be a finite number > 1");
+        return YR_EINVAL;
+    }
+    if (!(p->scale >= 1.0) || !std::isfinite(p->scale)) {
+        yr_host::set_error("yr_rope_freq_table: scale must be a finite number >= 1");
+        return YR_EINVAL;
+    }
+    if (p->method < YR_ROPE || p->method > YR_YARN) {
+        yr_host::set_error("yr_rope_freq_table: unknown method");
+        return YR_EINVAL;
+    }
+    if (p->method == YR_YARN && (p->L_train < 1 || !(p->beta > p->alpha))) {
+        yr_host::set_error("yr_rope_freq_table: YaRN needs L_train >= 1 and beta > alpha");
+        return YR_EINVAL;
+    }
+    yr_rope_table t;
+    std::memset(&t, 0, sizeof t);
+    t.head_dim = d;
+    t.method = p->method;
+    const double two_pi = 2.0 * M_PI;
+    const double ln_base = std::log(p->base);
+    const double s = p->scale;
+    // NTK-aware: the whole exponent scales the log of the base.
+    const double ln_base_ntk = ln_base + (static_cast<double>(d) / (d - 2)) * std::log(s);
+    for (int i = 0; i < d / 2; ++i) {
+        const double e = -2.0 * i / d;
+        const double theta = std::exp(e * ln_base);
+        double th = theta;
+        switch (p->method) {
+            case YR_PI:
+                th = theta / s;
+                break;
+            case YR_NTK:
+                th = std::exp(e * ln_base_ntk);
+                break;
+            case YR_YARN: {
+                const double r = p->L_train / (two_pi / theta);
+                double gamma = (r - p->alpha) / (p->beta - p->alpha);
+                gamma = gamma < 0.0 ? 0.0 : (gamma > 1.0 ? 1.0 : gamma);
+                th = theta * (gamma + (1.0 - gamma) / s);
+                break;
+            }
+            default:
+                break;
+        }
+        t.inv_freq[i] = th;
+        t.turns[i] = th / two_pi;
+    }
+    t.mscale = (p->method == YR_YARN) ? 0.1 * std::log(s) + 1.0 : 1.0;
+    t.softmax_scale = t.mscale * t.mscale / std::sqrt(static_cast<double>(d));
+    // Position-policy identity: a hash of the parameters that shape the table.
+    uint64_t hsh = 0xcbf29ce484222325ull;
+    // Fields a method does not use are hashed as constants, so equal tables
+    // share a digest.
+    const bool yarn = p->method == YR_YARN;
+    const int32_t fields_i[3] = {p->head_dim, yarn ? p->L_train : 0, p->method};
+    const double fields_d[4] = {p->base, p->method == YR_ROPE ? 1.0 : p->scale,
+                                yarn ? p->alpha : 0.0, yarn ? p->beta : 0.0};
+    hsh = fnv1a(hsh, fields_i, sizeof fields_i);
+    hsh = fnv1a(hsh, fields_d, sizeof fields_d);
+    t.digest = hsh;
+    *out = t;
+    return YR_OK;
+}

@@ -1,0 +1,381 @@
+// yarnattn.cu -- the C ABI of libyarnattn.so: argument checks, TMA descriptor
+// set-up and kernel launches on the caller's stream.  All kernels live in this
+// translation unit (they share the device status word).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/yarnattn.h"
+#include "decode_sm100.cuh"
+#include "kvprep_sm100.cuh"
+#include "prefill_sm100.cuh"
+
+namespace yr_host {
+
+thread_local std::string g_err;
+void set_error(const std::string &msg) { g_err = msg; }
+
+int fail(int code, const std::string &msg) {
+    set_error(msg);
+    return code;
+}
+
+int cuda_fail(const char *what, cudaError_t e) {
+    return fail(YR_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+uint64_t wait_timeout_ns() {
+    static uint64_t ns = [] {
+        const char *s = std::getenv("YR_WAIT_TIMEOUT_MS");
+        long ms = s ? std::strtol(s, nullptr, 10) : 2000;
+        if (ms < 1) ms = 1;
+        return static_cast<uint64_t>(ms) * 1000000ull;
+    }();
+    return ns;
+}
+
+// Per-device one-time set-up: architecture check and shared-memory opt-in.
+struct DeviceState {
+    bool ready = false;
+    bool sm100 = false;
+    int sm_count = 0;
+};
+std::mutex g_dev_mu;
+DeviceState g_dev[64];
+
+int prepare_device(int *sm_count) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if (dev < 0 || dev >= 64) return fail(YR_EUNSUPPORTED, "device index out of range");
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceState &st = g_dev[dev];
+    if (!st.ready) {
+        cudaDeviceProp prop;
+        e = cudaGetDeviceProperties(&prop, dev);
+        if (e != cudaSuccess) return cuda_fail("cudaGetDeviceProperties", e);
+        st.sm100 = (prop.major == 10 && prop.minor == 0);
+        st.sm_count = prop.multiProcessorCount;
+        if (st.sm100) {
+            struct {
+                const void *fn;
+                size_t bytes;
+            } attrs[] = {
+                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128>),
+                 yr::prefill_smem_bytes<128>()},
+                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64>),
+                 yr::prefill_smem_bytes<64>()},
+                {reinterpret_cast<const void *>(&yr::decode_split_kernel<128, 1>),
+                 yr::decode_smem_bytes<128>()},
+                {reinterpret_cast<const void *>(&yr::decode_split_kernel<128, 2>),
+                 yr::decode_smem_bytes<128>()},
+                {reinterpret_cast<const void *>(&yr::decode_split_kernel<64, 1>),
+                 yr::decode_smem_bytes<64>()},
+                {reinterpret_cast<const void *>(&yr::decode_split_kernel<64, 2>),
+                 yr::decode_smem_bytes<64>()},
+            };
+            for (auto &a : attrs) {
+                e = cudaFuncSetAttribute(a.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(a.bytes));
+                if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
+            }
+        }
+        st.ready = true;
+    }
+    if (!st.sm100) return fail(YR_EUNSUPPORTED, "the current device is not sm_100 (B200)");
+    if (sm_count) *sm_count = st.sm_count;
+    return YR_OK;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Element strides {b, h, t}: either given, or contiguous for [B][H][T][d].
+void strides_or_contiguous(const int64_t *s, int H, int T, int d, long long out[3]) {
+    if (s) {
+        out[0] = s[0];
+        out[1] = s[1];
+        out[2] = s[2];
+    } else {
+        out[2] = d;
+        out[1] = static_cast<long long>(T) * d;
+        out[0] = static_cast<long long>(H) * T * d;
+    }
+}
+
+bool strides_ok(const long long s[3]) {
+    for (int i = 0; i < 3; ++i)
+        if (s[i] <= 0 || (s[i] % 8) != 0 || s[i] >= (1ll << 38)) return false;
+    return true;
+}
+
+int encode(CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base,
+           const cuuint64_t *dims, const cuuint64_t *strides_bytes, const cuuint32_t *box,
+           const char *what) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(YR_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(map, dt, static_cast<cuuint32_t>(rank), const_cast<void *>(base), dims,
+                    strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(YR_ECUDA, std::string("cuTensorMapEncodeTiled failed for ") + what +
+                                  " (code " + std::to_string(static_cast<int>(r)) + ")");
+    return YR_OK;
+}
+
+size_t prefill_ws_bytes(long long B, long long Hkv, long long T, long long d) {
+    return static_cast<size_t>(2 * B * Hkv * T * d * 2);
+}
+
+int decode_chunks(int T_max) { return (T_max + yr::kDecChunk - 1) / yr::kDecChunk; }
+
+size_t decode_ws_bytes(long long B, long long Hq, long long Hkv, long long d, int T_max) {
+    const long long g = Hq / Hkv;
+    return static_cast<size_t>(B * Hkv * decode_chunks(T_max) * g * (d + 2) * 4);
+}
+
+}  // namespace yr_host
+
+using namespace yr_host;
+
+extern "C" const char *yr_last_error(void) { return g_err.c_str(); }
+
+extern "C" int yr_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+extern "C" size_t yr_attn_prefill_workspace_bytes(int B, int Hkv, int T, int d) {
+    if (B < 1 || Hkv < 1 || T < 1 || d < 2) return 0;
+    return prefill_ws_bytes(B, Hkv, T, d);
+}
+
+extern "C" size_t yr_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int T_max) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || d < 2 || T_max < 1 || Hq % Hkv) return 0;
+    return decode_ws_bytes(B, Hq, Hkv, d, T_max);
+}
+
+extern "C" int yr_attn_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
+                               void *k_cache, float *q_rot_dbg, float *k_rot_dbg, int B, int Hq,
+                               int Hkv, int T, int d, const int64_t *q_strides,
+                               const int64_t *k_strides, const int64_t *v_strides,
+                               const int64_t *o_strides, const int64_t *kc_strides,
+                               const yr_rope_table *tab, int causal, int window, int n_sink,
+                               void *workspace, size_t workspace_bytes, void *stream) {
+    set_error("");
+    if (!q || !k || !v || !o || !tab || !workspace)
+        return fail(YR_EINVAL, "yr_attn_prefill: q, k, v, o, tab and workspace must be non-NULL");
+    if (B < 1 || Hq < 1 || Hkv < 1 || T < 1)
+        return fail(YR_EINVAL, "yr_attn_prefill: B, Hq, Hkv and T must be >= 1");
+    if (Hq % Hkv != 0) return fail(YR_EINVAL, "yr_attn_prefill: Hq must be a multiple of Hkv");
+    if (d != 64 && d != 128) return fail(YR_EUNSUPPORTED, "yr_attn_prefill: d must be 64 or 128");
+    if (tab->head_dim != d) return fail(YR_EINVAL, "yr_attn_prefill: table head_dim != d");
+    if (causal != 0 && causal != 1) return fail(YR_EINVAL, "yr_attn_prefill: causal must be 0 or 1");
+    if (window < 0 || n_sink < 0) return fail(YR_EINVAL, "yr_attn_prefill: window and n_sink must be >= 0");
+    if (window > 0 && !causal) return fail(YR_EINVAL, "yr_attn_prefill: a window needs causal=1");
+    if (n_sink > 0 && window == 0) return fail(YR_EINVAL, "yr_attn_prefill: sinks need a window");
+    if (static_cast<long long>(B) * Hq * ((T + 255) / 256) >= (1ll << 31))
+        return fail(YR_EINVAL, "yr_attn_prefill: problem too large for one launch");
+    const size_t need = prefill_ws_bytes(B, Hkv, T, d);
+    if (workspace_bytes < need)
+        return fail(YR_EINVAL, "yr_attn_prefill: workspace too small (need " + std::to_string(need) + " bytes)");
+    if (!aligned(workspace, 256)) return fail(YR_EINVAL, "yr_attn_prefill: workspace must be 256-byte aligned");
+    for (const void *ptr : {q, k, v, static_cast<const void *>(o), static_cast<const void *>(k_cache),
+                            static_cast<const void *>(q_rot_dbg), static_cast<const void *>(k_rot_dbg)})
+        if (ptr && !aligned(ptr, 16)) return fail(YR_EINVAL, "yr_attn_prefill: pointers must be 16-byte aligned");
+    if (lse && !aligned(lse, 4)) return fail(YR_EINVAL, "yr_attn_prefill: lse must be 4-byte aligned");
+    long long qs[3], ks[3], vs[3], os[3], cs[3];
+    strides_or_contiguous(q_strides, Hq, T, d, qs);
+    strides_or_contiguous(k_strides, Hkv, T, d, ks);
+    strides_or_contiguous(v_strides, Hkv, T, d, vs);
+    strides_or_contiguous(o_strides, Hq, T, d, os);
+    strides_or_contiguous(kc_strides, Hkv, T, d, cs);
+    if (!strides_ok(qs) || !strides_ok(ks) || !strides_ok(vs) || !strides_ok(os) ||
+        (k_cache && !strides_ok(cs)))
+        return fail(YR_EINVAL, "yr_attn_prefill: strides must be positive multiples of 8 elements");
+    int sm_count = 0;
+    int rc = prepare_device(&sm_count);
+    if (rc != YR_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    __half *k16 = static_cast<__half *>(workspace);
+    __half *v16 = k16 + static_cast<size_t>(B) * Hkv * T * d;
+
+    // 1) rotate keys once, lay K~ and V out as fp16
+    {
+        yr::KvPrepParams kp;
+        std::memset(&kp, 0, sizeof kp);
+        kp.k = static_cast<const __nv_bfloat16 *>(k);
+        kp.v = static_cast<const __nv_bfloat16 *>(v);
+        kp.ksb = ks[0]; kp.ksh = ks[1]; kp.kst = ks[2];
+        kp.vsb = vs[0]; kp.vsh = vs[1]; kp.vst = vs[2];
+        kp.k16 = k16;
+        kp.v16 = v16;
+        kp.kc = static_cast<__nv_bfloat16 *>(k_cache);
+        kp.csb = cs[0]; kp.csh = cs[1]; kp.cst = cs[2];
+        kp.k_dbg = k_rot_dbg;
+        kp.Hkv = Hkv; kp.T = T; kp.d = d;
+        kp.n_items = static_cast<long long>(B) * Hkv * T * (d / 8);
+        for (int i = 0; i < d / 2; ++i) kp.turns[i] = tab->turns[i];
+        long long blocks = (kp.n_items + 255) / 256;
+        const long long cap = static_cast<long long>(sm_count) * 16;
+        if (blocks > cap) blocks = cap;
+        yr::kv_prep_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(kp);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail("kv_prep_kernel launch", e);
+    }
+    // 2) attention
+    yr::PrefillParams pp;
+    std::memset(&pp, 0, sizeof pp);
+    {
+        const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T),
+                                    static_cast<cuuint64_t>(Hq), static_cast<cuuint64_t>(B)};
+        const cuuint64_t strides[3] = {static_cast<cuuint64_t>(qs[2] * 2), static_cast<cuuint64_t>(qs[1] * 2),
+                                       static_cast<cuuint64_t>(qs[0] * 2)};
+        const cuuint32_t box[4] = {64, 128, 1, 1};
+        rc = encode(&pp.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, q, dims, strides, box, "q");
+        if (rc != YR_OK) return rc;
+    }
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T),
+                                    static_cast<cuuint64_t>(B) * Hkv};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(T) * d * 2};
+        const cuuint32_t box[3] = {64, 128, 1};
+        rc = encode(&pp.tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, k16, dims, strides, box, "rotated k");
+        if (rc != YR_OK) return rc;
+        rc = encode(&pp.tm_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, v16, dims, strides, box, "v");
+        if (rc != YR_OK) return rc;
+    }
+    pp.o = static_cast<__nv_bfloat16 *>(o);
+    pp.osb = os[0]; pp.osh = os[1]; pp.ost = os[2];
+    pp.lse = lse;
+    pp.q_dbg = q_rot_dbg;
+    pp.B = B; pp.Hq = Hq; pp.Hkv = Hkv; pp.T = T; pp.group = Hq / Hkv;
+    pp.causal = causal; pp.window = window; pp.n_sink = n_sink;
+    pp.n_qblocks = (T + 255) / 256;
+    pp.sl2 = static_cast<float>(tab->softmax_scale * 1.4426950408889634);
+    pp.timeout_ns = wait_timeout_ns();
+    for (int i = 0; i < d / 2; ++i) pp.turns[i] = tab->turns[i];
+    const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * Hq * pp.n_qblocks);
+    if (d == 128)
+        yr::prefill_attn_kernel<128><<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<128>(), st>>>(pp);
+    else
+        yr::prefill_attn_kernel<64><<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<64>(), st>>>(pp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("prefill_attn_kernel launch", e);
+    return YR_OK;
+}
+
+extern "C" int yr_attn_decode(const void *q_new, const void *k_new, const void *v_new,
+                              void *k_cache, void *v_cache, const int32_t *cache_len, void *o,
+                              float *lse, float *q_rot_dbg, int B, int Hq, int Hkv, int d,
+                              int T_max, const yr_rope_table *tab, int window, int n_sink,
+                              void *workspace, size_t workspace_bytes, void *stream) {
+    set_error("");
+    if (!q_new || !k_new || !v_new || !k_cache || !v_cache || !cache_len || !o || !tab || !workspace)
+        return fail(YR_EINVAL, "yr_attn_decode: NULL pointer argument");
+    if (B < 1 || Hq < 1 || Hkv < 1 || T_max < 1)
+        return fail(YR_EINVAL, "yr_attn_decode: B, Hq, Hkv and T_max must be >= 1");
+    if (Hq % Hkv != 0) return fail(YR_EINVAL, "yr_attn_decode: Hq must be a multiple of Hkv");
+    if (d != 64 && d != 128) return fail(YR_EUNSUPPORTED, "yr_attn_decode: d must be 64 or 128");
+    if (Hq / Hkv > 16) return fail(YR_EUNSUPPORTED, "yr_attn_decode: at most 16 query heads per KV head");
+    if (tab->head_dim != d) return fail(YR_EINVAL, "yr_attn_decode: table head_dim != d");
+    if (window < 0 || n_sink < 0) return fail(YR_EINVAL, "yr_attn_decode: window and n_sink must be >= 0");
+    if (n_sink > 0 && window == 0) return fail(YR_EINVAL, "yr_attn_decode: sinks need a window");
+    const size_t need = decode_ws_bytes(B, Hq, Hkv, d, T_max);
+    if (workspace_bytes < need)
+        return fail(YR_EINVAL, "yr_attn_decode: workspace too small (need " + std::to_string(need) + " bytes)");
+    if (!aligned(workspace, 256)) return fail(YR_EINVAL, "yr_attn_decode: workspace must be 256-byte aligned");
+    for (const void *ptr : {q_new, k_new, v_new, static_cast<const void *>(k_cache),
+                            static_cast<const void *>(v_cache), static_cast<const void *>(o)})
+        if (!aligned(ptr, 16)) return fail(YR_EINVAL, "yr_attn_decode: tensor pointers must be 16-byte aligned");
+    if (!aligned(cache_len, 4) || (lse && !aligned(lse, 4)) || (q_rot_dbg && !aligned(q_rot_dbg, 4)))
+        return fail(YR_EINVAL, "yr_attn_decode: cache_len/lse/q_rot_dbg must be 4-byte aligned");
+    int rc = prepare_device(nullptr);
+    if (rc != YR_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int g = Hq / Hkv;
+    const int nc = decode_chunks(T_max);
+    yr::DecodeParams dp;
+    std::memset(&dp, 0, sizeof dp);
+    dp.q_new = static_cast<const __nv_bfloat16 *>(q_new);
+    dp.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+    dp.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+    dp.k_cache = static_cast<__nv_bfloat16 *>(k_cache);
+    dp.v_cache = static_cast<__nv_bfloat16 *>(v_cache);
+    dp.cache_len = cache_len;
+    dp.ws_o = static_cast<float *>(workspace);
+    dp.ws_ml = dp.ws_o + static_cast<size_t>(B) * Hkv * nc * g * d;
+    dp.o = static_cast<__nv_bfloat16 *>(o);
+    dp.lse = lse;
+    dp.q_dbg = q_rot_dbg;
+    dp.B = B; dp.Hq = Hq; dp.Hkv = Hkv; dp.T_max = T_max; dp.group = g; dp.n_chunks = nc;
+    dp.window = window; dp.n_sink = n_sink;
+    dp.sl2 = static_cast<float>(tab->softmax_scale * 1.4426950408889634);
+    for (int i = 0; i < d / 2; ++i) dp.turns[i] = tab->turns[i];
+    const dim3 grid(nc, Hkv, B);
+    if (d == 128) {
+        if (g <= 8)
+            yr::decode_split_kernel<128, 1><<<grid, yr::kDecThreads, yr::decode_smem_bytes<128>(), st>>>(dp);
+        else
+            yr::decode_split_kernel<128, 2><<<grid, yr::kDecThreads, yr::decode_smem_bytes<128>(), st>>>(dp);
+    } else {
+        if (g <= 8)
+            yr::decode_split_kernel<64, 1><<<grid, yr::kDecThreads, yr::decode_smem_bytes<64>(), st>>>(dp);
+        else
+            yr::decode_split_kernel<64, 2><<<grid, yr::kDecThreads, yr::decode_smem_bytes<64>(), st>>>(dp);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("decode_split_kernel launch", e);
+    const dim3 mgrid(Hq, B);
+    if (d == 128)
+        yr::decode_merge_kernel<128><<<mgrid, 128, 0, st>>>(dp);
+    else
+        yr::decode_merge_kernel<64><<<mgrid, 64, 0, st>>>(dp);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("decode_merge_kernel launch", e);
+    return YR_OK;
+}
+
+extern "C" int yr_device_status(void *stream) {
+    set_error("");
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail("cudaStreamSynchronize", e);
+    unsigned v = 0;
+    e = cudaMemcpyFromSymbol(&v, g_yr_status, sizeof v);
+    if (e != cudaSuccess) return cuda_fail("reading the status word", e);
+    if (v == 0) return YR_OK;
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_yr_status, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail("clearing the status word", e);
+    std::string msg = "device status:";
+    if (v & yr::kStatusTimeoutLoad) msg += " prefill-load-timeout";
+    if (v & yr::kStatusTimeoutMma) msg += " prefill-mma-timeout";
+    if (v & yr::kStatusTimeoutSoftmax) msg += " prefill-softmax-timeout";
+    if (v & yr::kStatusTimeoutDrain) msg += " prefill-drain-timeout";
+    if (v & yr::kStatusBadCacheLen) msg += " decode-cache-length-out-of-range";
+    set_error(msg);
+    return (v & 0xFFu) ? YR_ETIMEOUT : YR_EINVAL;
+}
