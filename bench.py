@@ -1,0 +1,474 @@
+#!/usr/bin/env python
+"""Benchmark of the YaRN-RoPE attention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl yarn|reference]
+
+One step is one prefill of the Llama-2-7B-shaped workload (B=1, Hq=Hkv=32,
+d=128, T=16384, causal, YaRN base 1e4, L_train 4096, s=4): the rotated-key pass
+plus the attention kernel, inputs resident in HBM.  The headline is prefill
+TFLOP/s with causal FLOPs counted (4 d Hq B sum_m |visible(m)|).  The same run
+times the single-token decode workload (B=8, Hq=32, Hkv=8, d=128, cache
+lengths U[32768,131072]) and reports it as KV-read GB/s under "decode".
+
+For N > 1 (launched with torch.distributed.run) every rank runs the same
+workload as an independent replica; NCCL carries only the barrier and the
+max-over-ranks of the timings.  --impl reference times the fp64 CPU oracle on
+a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from yarn_position_scaling_b200 import metrics, synth  # noqa: E402
+
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["yarn", "reference"], default="yarn")
+    ap.add_argument("--decode-steps", type=int, default=None)
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="sequences in the decode workload (default 8; smaller for profiling)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the last ncu capture, or None when the kernel
+    sources changed since that capture (profiles/traffic.json keeps their hash)."""
+    import glob
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        h = hashlib.sha256()
+        for src in sorted(glob.glob(os.path.join(ROOT, "yarn_position_scaling_b200", "csrc", "*"))):
+            with open(src, "rb") as f:
+                h.update(f.read())
+        if h.hexdigest()[:16] != t["source_sha"] or kernel not in t:
+            return None
+        return float(t[kernel]["dram_read"] + t[kernel]["dram_write"])
+    except Exception:
+        return None
+
+
+class Dist:
+    """One process per GPU (torch.distributed.run).  The collective carries only the
+    barrier and the max of the timings: the replicas share no data."""
+
+    def __init__(self, n_gpus: int, backend: str = "nccl"):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        if self.world != n_gpus:
+            raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={self.world}: launch N>1 with "
+                             "torch.distributed.run")
+        self.pg = None
+        self.device = "cuda" if backend == "nccl" else "cpu"
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            kw = {}
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+                kw["device_id"] = torch.device("cuda", self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+            self.dist = dist
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            self.dist.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+            self.pg = None
+
+
+def throughput(units_per_step: float, steps: int, max_ms: float, world: int, scale: float):
+    """Whole-job rate: the units every rank processed over the slowest rank's time."""
+    return world * units_per_step * steps / (max_ms * 1e-3) / scale
+
+
+class Clocks:
+    """nvidia-smi samples of this GPU during a timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        self.file.close()
+        os.unlink(self.file.name)
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                power.append(float(r[3]))
+            except (ValueError, IndexError):
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        loaded = [s for s, p in zip(sm, power) if p > 300.0] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+def time_events(fn, steps, stream):
+    """Run fn(step) `steps` times; fn returns a list of (start, end) event pairs per kernel."""
+    starts = torch.cuda.Event(enable_timing=True)
+    ends = torch.cuda.Event(enable_timing=True)
+    per_kernel = []
+    torch.cuda.synchronize()
+    starts.record(stream)
+    for i in range(steps):
+        per_kernel.append(fn(i))
+    ends.record(stream)
+    torch.cuda.synchronize()
+    total = starts.elapsed_time(ends)
+    kernel_ms = [sum(a.elapsed_time(b) for a, b in ev) for ev in zip(*per_kernel)]
+    return total, kernel_ms
+
+
+# ------------------------------------------------------------------ CPU oracle
+_CPU_INPUTS = {}
+
+
+def _cpu_inputs(w):
+    if w.name not in _CPU_INPUTS:
+        q, k, v = synth.prefill_inputs(w, "cpu")
+        _CPU_INPUTS[w.name] = tuple(t.view(torch.int16).numpy().view(np.uint16) for t in (q, k, v))
+    return _CPU_INPUTS[w.name]
+
+
+def oracle_sample(w, seconds: float, seed: int = 0):
+    """Time the fp64 oracle on query rows of workload w drawn until ~`seconds` of CPU work;
+    returns (flops_done, wall_s, threads, description)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    T, d = w.T, w.d
+    qb, kb, vb = _cpu_inputs(w)
+    th, _, ss = oracle.rope_theta(d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta)
+    counts = metrics.visible_counts(T, w.causal, w.window, w.n_sink)
+    done_flops, done_rows, wall = 0.0, 0, 0.0
+    batch = 16
+    while wall < seconds:
+        h = int(rng.integers(0, w.Hq))
+        ms = rng.integers(0, T, size=batch)
+        rows = (h * T + ms).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attn_rows(qb, kb, vb, th, ss, w.causal, w.window, w.n_sink, rows=rows)
+        wall += time.perf_counter() - t0
+        done_flops += float(4.0 * d * counts[ms].sum())
+        done_rows += batch
+        batch = min(batch * 2, 256)
+    threads = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+    desc = (f"{done_rows} query rows of {w.name} drawn uniformly over positions, "
+            f"one head per batch of rows; keys rotated on the fly by the oracle; "
+            f"FLOPs counted as 4*d*|visible(m)| per row")
+    return done_flops, wall, threads, desc
+
+
+def reference_arm(args, dist: Dist):
+    w = synth.LLAMA2_16K
+    line = {"impl": "reference"}
+    if dist.rank != 0:
+        return None
+    steps, warm = args.steps, args.warmup
+    per_step = min(max(0.2, 120.0 / max(1, steps + warm)), 20.0)
+    for _ in range(warm):
+        oracle_sample(w, min(per_step, 2.0), seed=1)
+    flops, wall = 0.0, 0.0
+    desc, threads = "", 0
+    for s in range(steps):
+        f, t, threads, desc = oracle_sample(w, per_step, seed=100 + s)
+        flops += f
+        wall += t
+    value = flops / wall / 1e12
+    line.update({
+        "metric": "causal YaRN-RoPE attention prefill TFLOP/s", "value": value, "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": steps, "warmup": warm, "ms_per_step": wall / steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic N(0,1) bf16 inputs, seeded",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T,
+                   "method": w.method, "base": w.base, "L_train": w.L_train, "scale": w.scale,
+                   "causal": True, "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"each step ~{per_step:.1f}s of oracle work: {desc}"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    })
+    return line
+
+
+# ------------------------------------------------------------------- GPU arm
+def prefill_bench(w, steps, warmup, stream):
+    from yarn_position_scaling_b200 import api
+    q, k, v = synth.prefill_inputs(w, "cuda")
+    tab = api.rope_freq_table(w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta)
+    ws = torch.empty(api.attn_prefill_workspace_bytes(w.B, w.Hkv, w.T, w.d), dtype=torch.uint8,
+                     device="cuda")
+    o = torch.empty_like(q)
+
+    def step(_):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        api.prefill_prepare_kv(k, v, tab, ws, stream=stream)
+        e[1].record(stream)
+        api.prefill_attend(q, w.Hkv, tab, ws, w.causal, w.window, w.n_sink, out=o, stream=stream)
+        e[2].record(stream)
+        return [(e[0], e[1]), (e[1], e[2])]
+
+    for i in range(warmup):
+        step(i)
+    api.device_status(stream)
+    return step, (q, k, v, o, ws, tab)
+
+
+def decode_bench(w, steps, warmup, stream):
+    from yarn_position_scaling_b200 import api
+    qn, kn, vn, kc, vc, lens = synth.decode_inputs(w, "cuda")
+    cl = lens.cuda()
+    tab = api.rope_freq_table(w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta)
+    ws = torch.empty(api.attn_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.d, w.T),
+                     dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(qn)
+
+    def step(_):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(stream)
+        api.attn_decode(qn, kn, vn, kc, vc, cl, tab, out=o, workspace=ws, stream=stream)
+        e[1].record(stream)
+        return [(e[0], e[1])]
+
+    for i in range(warmup):
+        step(i)
+    api.device_status(stream)
+    return step, lens.tolist()
+
+
+def e2e_prefill(w, steps, warmup, stream):
+    """Through the public API with host buffers: pinned H2D of q, k, v, the call, D2H of o."""
+    from yarn_position_scaling_b200 import api
+    qh, kh, vh = [t.pin_memory() for t in synth.prefill_inputs(w, "cpu")]
+    oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
+    qd, kd, vd = [torch.empty_like(t, device="cuda") for t in (qh, kh, vh)]
+    tab = api.rope_freq_table(w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta)
+    ws = torch.empty(api.attn_prefill_workspace_bytes(w.B, w.Hkv, w.T, w.d), dtype=torch.uint8,
+                     device="cuda")
+    od = torch.empty_like(qd)
+
+    def step(_):
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        api.attn_prefill(qd, kd, vd, tab, w.causal, w.window, w.n_sink, out=od, workspace=ws,
+                         stream=stream)
+        oh.copy_(od, non_blocking=True)
+        return []
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size()
+    return step, h2d, d2h
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        # CPU only: rank 0 runs the oracle, the other ranks exit at once without a
+        # process group (nothing to synchronise).
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+
+        class _Solo:
+            rank = 0
+        line = reference_arm(args, _Solo())
+        print(json.dumps(line), flush=True)
+        return
+    dist = Dist(args.gpus)
+    if not torch.cuda.is_available():
+        raise SystemExit("no CUDA device: the benchmark needs a B200")
+    from yarn_position_scaling_b200 import api
+    api.load()
+    torch.cuda.set_device(dist.local)
+    stream = torch.cuda.current_stream()
+    peaks, peak_src = load_peaks()
+    n = dist.world
+    wp, wd = synth.LLAMA2_16K, synth.DECODE
+    if args.decode_batch:
+        import dataclasses
+        wd = dataclasses.replace(wd, B=args.decode_batch)
+    steps, warm = args.steps, max(3, args.warmup)
+    dsteps = args.decode_steps or steps
+    esteps = args.e2e_steps or max(3, min(steps // 10, 30))
+
+    # ---------------- prefill (headline)
+    pstep, keep = prefill_bench(wp, steps, warm, stream)
+    flops_step = metrics.prefill_flops(wp.B, wp.Hq, wp.T, wp.d, wp.causal, wp.window, wp.n_sink)
+    clocks = Clocks(torch.cuda.current_device())
+    clocks.start()
+    dist.barrier()
+    total_ms, (prep_ms, attn_ms) = time_events(pstep, steps, stream)
+    dist.barrier()
+    clk = clocks.stop()
+    api.device_status(stream)
+    total_ms = dist.max(total_ms)
+    attn_ms_max = dist.max(attn_ms)
+    prep_ms_max = dist.max(prep_ms)
+    ms_per_step = total_ms / steps
+    value = throughput(flops_step, steps, total_ms, n, 1e12)
+    attn_tflops = flops_step / (attn_ms_max / steps * 1e-3) / 1e12
+    peak_t = peaks["bf16_tflops"]
+    del keep, pstep
+    torch.cuda.empty_cache()
+
+    # ---------------- decode
+    dstep, lens = decode_bench(wd, dsteps, warm, stream)
+    dbytes = metrics.decode_kv_bytes(lens, wd.Hkv, wd.d)
+    dist.barrier()
+    dtotal_ms, (dcall_ms,) = time_events(dstep, dsteps, stream)
+    dist.barrier()
+    api.device_status(stream)
+    dtotal_ms = dist.max(dtotal_ms)
+    dcall_ms = dist.max(dcall_ms)
+    d_gbs = throughput(dbytes, dsteps, dtotal_ms, n, 1e9)
+    d_call_gbs = dbytes / (dcall_ms / dsteps * 1e-3) / 1e9
+    del dstep
+    torch.cuda.empty_cache()
+
+    # ---------------- end to end through the API with host buffers
+    estep, h2d, d2h = e2e_prefill(wp, esteps, 2, stream)
+    dist.barrier()
+    etotal_ms, _ = time_events(estep, esteps, stream)
+    dist.barrier()
+    etotal_ms = dist.max(etotal_ms)
+    e2e_value = throughput(flops_step, esteps, etotal_ms, n, 1e12)
+
+    # ---------------- CPU oracle baseline (rank 0, N=1 only)
+    cpu = None
+    if dist.rank == 0 and n == 1 and not args.no_cpu_baseline:
+        f, t, threads, desc = oracle_sample(wp, args.cpu_seconds)
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": desc}
+
+    line = {
+        "metric": "causal YaRN-RoPE attention prefill TFLOP/s", "value": value,
+        "unit": "TFLOP/s", "n_gpus": n, "steps": steps, "warmup": warm,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp16",
+        "data": "synthetic: seeded i.i.d. N(0,1) inputs rounded to bf16",
+        "config": {"workload": wp.name, "B": wp.B, "Hq": wp.Hq, "Hkv": wp.Hkv, "d": wp.d,
+                   "T": wp.T, "method": wp.method, "base": wp.base, "L_train": wp.L_train,
+                   "scale": wp.scale, "causal": True, "io_dtype": "bf16",
+                   "mma_operands": "fp16", "accumulate": "fp32",
+                   "parallelism": f"replicas x{n}",
+                   "l2": "no flush: q+k+v+o = %.0f MB per step > 126 MB L2" %
+                         (4 * wp.B * wp.Hq * wp.T * wp.d * 2 / 2 ** 20),
+                   "step": "yr_prefill_prepare_kv + yr_prefill_attend (= yr_attn_prefill)"},
+        "roofline": {"bound": "tensor", "kernel": "prefill_attn_kernel<128>",
+                     "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": attn_tflops / peak_t, "peak_source": f"{peak_src} bf16 burst "
+                     "(fp16 tensor rate equals bf16)",
+                     "traffic": ncu_traffic("prefill_attn_kernel<128>"),
+                     "algorithmic_flops_per_launch": flops_step,
+                     "kernel_ms": attn_ms_max / steps,
+                     "kv_prep_ms": prep_ms_max / steps},
+        "decode": {
+            "metric": "decode KV-read GB/s", "value": d_gbs, "unit": "GB/s", "steps": dsteps,
+            "ms_per_step": dtotal_ms / dsteps, "workload": wd.name,
+            "config": {"B": wd.B, "Hq": wd.Hq, "Hkv": wd.Hkv, "d": wd.d, "T_max": wd.T,
+                       "cache_len": lens, "chunk_keys": 2048,
+                       "l2": "no flush: %.2f GB of K/V read per step > 126 MB L2" % (dbytes / 1e9)},
+            "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<128,1> + merge",
+                         "achieved": d_call_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": d_call_gbs / peaks["hbm_gbs"],
+                         "peak_source": f"{peak_src} HBM copy",
+                         "traffic": ncu_traffic("decode_split_kernel<128,1>"),
+                         "algorithmic_bytes_per_launch": dbytes,
+                         "timed_over": "the whole decode call (split + merge launches)"}},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": esteps},
+        "cpu_baseline": cpu,
+        "gpu_launches": 2 * steps,
+        "clocks": clk,
+    }
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+if __name__ == "__main__":
+    main()

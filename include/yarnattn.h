@@ -140,6 +140,35 @@ int yr_attn_prefill(const void *q, const void *k, const void *v, void *o, float 
                     void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * prefill_prepare_kv -- first half of yr_attn_prefill: rotate every key by its
+ * position (k~_n = R_n k_n, "Arch_03_Long_Context", RoPE slide) and lay the
+ * rotated keys and the values out in `workspace` as fp16 [B, Hkv, T, d].
+ * Optionally also writes the rotated keys as bf16 to k_cache (caller strides)
+ * and as fp32 to k_rot_dbg (contiguous).  Arguments, alignment and errors as in
+ * yr_attn_prefill.  Useful on its own when several query blocks attend to the
+ * same keys: prepare once, then call yr_prefill_attend per block.
+ */
+int yr_prefill_prepare_kv(const void *k, const void *v, void *k_cache, float *k_rot_dbg,
+                          int B, int Hkv, int T, int d,
+                          const int64_t *k_strides, const int64_t *v_strides,
+                          const int64_t *kc_strides, const yr_rope_table *tab,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * prefill_attend -- second half of yr_attn_prefill: rotate the queries inside
+ * the attention kernel and attend over the keys and values that
+ * yr_prefill_prepare_kv left in `workspace` (which must have been prepared with
+ * the same B, Hkv, T, d and table, on this stream or with the ordering made
+ * explicit by the caller).  Arguments, alignment and errors as in
+ * yr_attn_prefill; `workspace` is only read.
+ */
+int yr_prefill_attend(const void *q, void *o, float *lse, float *q_rot_dbg,
+                      int B, int Hq, int Hkv, int T, int d,
+                      const int64_t *q_strides, const int64_t *o_strides,
+                      const yr_rope_table *tab, int causal, int window, int n_sink,
+                      const void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * attn_decode_workspace_bytes -- bytes of device workspace yr_attn_decode needs
  * for its split-KV partial results with a cache of T_max slots.  0 if invalid.
  */

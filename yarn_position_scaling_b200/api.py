@@ -18,8 +18,8 @@ YR_OK, YR_EINVAL, YR_EUNSUPPORTED, YR_ECUDA, YR_ETIMEOUT = 0, -1, -2, -3, -4
 ROPE, PI, NTK, YARN = 0, 1, 2, 3
 METHODS = {"rope": ROPE, "pi": PI, "ntk": NTK, "yarn": YARN}
 SYMBOLS = ("yr_rope_freq_table", "yr_attn_prefill_workspace_bytes", "yr_attn_prefill",
-           "yr_attn_decode_workspace_bytes", "yr_attn_decode", "yr_device_status",
-           "yr_last_error", "yr_version")
+           "yr_prefill_prepare_kv", "yr_prefill_attend", "yr_attn_decode_workspace_bytes",
+           "yr_attn_decode", "yr_device_status", "yr_last_error", "yr_version")
 
 
 class YarnAttnError(RuntimeError):
@@ -63,6 +63,12 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.yr_attn_prefill.argtypes = ([vp] * 8 + [ci] * 5 + [i64p] * 5 +
                                     [ctypes.POINTER(RopeTable), ci, ci, ci, vp, cs, vp])
     lib.yr_attn_prefill.restype = ci
+    lib.yr_prefill_prepare_kv.argtypes = ([vp] * 4 + [ci] * 4 + [i64p] * 3 +
+                                          [ctypes.POINTER(RopeTable), vp, cs, vp])
+    lib.yr_prefill_prepare_kv.restype = ci
+    lib.yr_prefill_attend.argtypes = ([vp] * 4 + [ci] * 5 + [i64p] * 2 +
+                                      [ctypes.POINTER(RopeTable), ci, ci, ci, vp, cs, vp])
+    lib.yr_prefill_attend.restype = ci
     lib.yr_attn_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
     lib.yr_attn_decode_workspace_bytes.restype = cs
     lib.yr_attn_decode.argtypes = ([vp] * 9 + [ci] * 5 +
@@ -136,6 +142,34 @@ def attn_prefill(q, k, v, table: RopeTable, causal: bool = True, window: int = 0
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(q_rot_dbg),
         _ptr(k_rot_dbg), B, Hq, Hkv, T, d, _strides(q), _strides(k), _strides(v), _strides(out),
         kc_strides, ctypes.byref(table), int(bool(causal)), int(window), int(n_sink),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc)
+    return out
+
+
+def prefill_prepare_kv(k, v, table: RopeTable, workspace, k_cache=None, k_rot_dbg=None,
+                       stream=None):
+    """First half of attn_prefill: rotated keys and values (fp16) into `workspace`."""
+    B, Hkv, T, d = k.shape
+    kc_strides = _strides(k_cache) if k_cache is not None else None
+    rc = load().yr_prefill_prepare_kv(
+        _ptr(k), _ptr(v), _ptr(k_cache), _ptr(k_rot_dbg), B, Hkv, T, d, _strides(k),
+        _strides(v), kc_strides, ctypes.byref(table), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc)
+    return workspace
+
+
+def prefill_attend(q, Hkv: int, table: RopeTable, workspace, causal: bool = True,
+                   window: int = 0, n_sink: int = 0, out=None, lse=None, q_rot_dbg=None,
+                   stream=None):
+    """Second half of attn_prefill: attention over a workspace from prefill_prepare_kv."""
+    B, Hq, T, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, T, d), dtype=torch.bfloat16, device=q.device)
+    rc = load().yr_prefill_attend(
+        _ptr(q), _ptr(out), _ptr(lse), _ptr(q_rot_dbg), B, Hq, Hkv, T, d, _strides(q),
+        _strides(out), ctypes.byref(table), int(bool(causal)), int(window), int(n_sink),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc)
     return out

@@ -177,82 +177,111 @@ extern "C" size_t yr_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, 
     return decode_ws_bytes(B, Hq, Hkv, d, T_max);
 }
 
-extern "C" int yr_attn_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
-                               void *k_cache, float *q_rot_dbg, float *k_rot_dbg, int B, int Hq,
-                               int Hkv, int T, int d, const int64_t *q_strides,
-                               const int64_t *k_strides, const int64_t *v_strides,
-                               const int64_t *o_strides, const int64_t *kc_strides,
-                               const yr_rope_table *tab, int causal, int window, int n_sink,
-                               void *workspace, size_t workspace_bytes, void *stream) {
-    set_error("");
-    if (!q || !k || !v || !o || !tab || !workspace)
-        return fail(YR_EINVAL, "yr_attn_prefill: q, k, v, o, tab and workspace must be non-NULL");
-    if (B < 1 || Hq < 1 || Hkv < 1 || T < 1)
-        return fail(YR_EINVAL, "yr_attn_prefill: B, Hq, Hkv and T must be >= 1");
-    if (Hq % Hkv != 0) return fail(YR_EINVAL, "yr_attn_prefill: Hq must be a multiple of Hkv");
-    if (d != 64 && d != 128) return fail(YR_EUNSUPPORTED, "yr_attn_prefill: d must be 64 or 128");
-    if (tab->head_dim != d) return fail(YR_EINVAL, "yr_attn_prefill: table head_dim != d");
-    if (causal != 0 && causal != 1) return fail(YR_EINVAL, "yr_attn_prefill: causal must be 0 or 1");
-    if (window < 0 || n_sink < 0) return fail(YR_EINVAL, "yr_attn_prefill: window and n_sink must be >= 0");
-    if (window > 0 && !causal) return fail(YR_EINVAL, "yr_attn_prefill: a window needs causal=1");
-    if (n_sink > 0 && window == 0) return fail(YR_EINVAL, "yr_attn_prefill: sinks need a window");
-    if (static_cast<long long>(B) * Hq * ((T + 255) / 256) >= (1ll << 31))
-        return fail(YR_EINVAL, "yr_attn_prefill: problem too large for one launch");
+namespace yr_host {
+
+int check_common(const char *fn, int B, int Hkv, int T, int d, const yr_rope_table *tab,
+                 const void *workspace, size_t workspace_bytes) {
+    const std::string f(fn);
+    if (!tab || !workspace) return fail(YR_EINVAL, f + ": tab and workspace must be non-NULL");
+    if (B < 1 || Hkv < 1 || T < 1) return fail(YR_EINVAL, f + ": B, Hkv and T must be >= 1");
+    if (d != 64 && d != 128) return fail(YR_EUNSUPPORTED, f + ": d must be 64 or 128");
+    if (tab->head_dim != d) return fail(YR_EINVAL, f + ": table head_dim != d");
     const size_t need = prefill_ws_bytes(B, Hkv, T, d);
     if (workspace_bytes < need)
-        return fail(YR_EINVAL, "yr_attn_prefill: workspace too small (need " + std::to_string(need) + " bytes)");
-    if (!aligned(workspace, 256)) return fail(YR_EINVAL, "yr_attn_prefill: workspace must be 256-byte aligned");
-    for (const void *ptr : {q, k, v, static_cast<const void *>(o), static_cast<const void *>(k_cache),
-                            static_cast<const void *>(q_rot_dbg), static_cast<const void *>(k_rot_dbg)})
-        if (ptr && !aligned(ptr, 16)) return fail(YR_EINVAL, "yr_attn_prefill: pointers must be 16-byte aligned");
-    if (lse && !aligned(lse, 4)) return fail(YR_EINVAL, "yr_attn_prefill: lse must be 4-byte aligned");
-    long long qs[3], ks[3], vs[3], os[3], cs[3];
-    strides_or_contiguous(q_strides, Hq, T, d, qs);
+        return fail(YR_EINVAL, f + ": workspace too small (need " + std::to_string(need) + " bytes)");
+    if (!aligned(workspace, 256)) return fail(YR_EINVAL, f + ": workspace must be 256-byte aligned");
+    return YR_OK;
+}
+
+int check_prepare(const void *k, const void *v, const void *k_cache, const float *k_rot_dbg,
+                  int B, int Hkv, int T, int d, const int64_t *k_strides, const int64_t *v_strides,
+                  const int64_t *kc_strides, const yr_rope_table *tab, const void *workspace,
+                  size_t workspace_bytes, const char *fn, long long ks[3], long long vs[3],
+                  long long cs[3]) {
+    if (!k || !v) return fail(YR_EINVAL, std::string(fn) + ": k and v must be non-NULL");
+    int rc = check_common(fn, B, Hkv, T, d, tab, workspace, workspace_bytes);
+    if (rc != YR_OK) return rc;
+    for (const void *ptr : {k, v, k_cache, static_cast<const void *>(k_rot_dbg)})
+        if (ptr && !aligned(ptr, 16))
+            return fail(YR_EINVAL, std::string(fn) + ": pointers must be 16-byte aligned");
     strides_or_contiguous(k_strides, Hkv, T, d, ks);
     strides_or_contiguous(v_strides, Hkv, T, d, vs);
-    strides_or_contiguous(o_strides, Hq, T, d, os);
     strides_or_contiguous(kc_strides, Hkv, T, d, cs);
-    if (!strides_ok(qs) || !strides_ok(ks) || !strides_ok(vs) || !strides_ok(os) ||
-        (k_cache && !strides_ok(cs)))
-        return fail(YR_EINVAL, "yr_attn_prefill: strides must be positive multiples of 8 elements");
-    int sm_count = 0;
-    int rc = prepare_device(&sm_count);
-    if (rc != YR_OK) return rc;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (!strides_ok(ks) || !strides_ok(vs) || (k_cache && !strides_ok(cs)))
+        return fail(YR_EINVAL, std::string(fn) + ": strides must be positive multiples of 8 elements");
+    return YR_OK;
+}
 
+int check_attend(const void *q, const void *o, const float *lse, const float *q_rot_dbg, int B,
+                 int Hq, int Hkv, int T, int d, const int64_t *q_strides, const int64_t *o_strides,
+                 const yr_rope_table *tab, int causal, int window, int n_sink,
+                 const void *workspace, size_t workspace_bytes, const char *fn, long long qs[3],
+                 long long os[3]) {
+    const std::string f(fn);
+    if (!q || !o) return fail(YR_EINVAL, f + ": q and o must be non-NULL");
+    if (Hq < 1) return fail(YR_EINVAL, f + ": B, Hq, Hkv and T must be >= 1");
+    int rc = check_common(fn, B, Hkv, T, d, tab, workspace, workspace_bytes);
+    if (rc != YR_OK) return rc;
+    if (Hq % Hkv != 0) return fail(YR_EINVAL, f + ": Hq must be a multiple of Hkv");
+    if (causal != 0 && causal != 1) return fail(YR_EINVAL, f + ": causal must be 0 or 1");
+    if (window < 0 || n_sink < 0) return fail(YR_EINVAL, f + ": window and n_sink must be >= 0");
+    if (window > 0 && !causal) return fail(YR_EINVAL, f + ": a window needs causal=1");
+    if (n_sink > 0 && window == 0) return fail(YR_EINVAL, f + ": sinks need a window");
+    if (static_cast<long long>(B) * Hq * ((T + 255) / 256) >= (1ll << 31))
+        return fail(YR_EINVAL, f + ": problem too large for one launch");
+    for (const void *ptr : {q, o, static_cast<const void *>(q_rot_dbg)})
+        if (ptr && !aligned(ptr, 16)) return fail(YR_EINVAL, f + ": pointers must be 16-byte aligned");
+    if (lse && !aligned(lse, 4)) return fail(YR_EINVAL, f + ": lse must be 4-byte aligned");
+    strides_or_contiguous(q_strides, Hq, T, d, qs);
+    strides_or_contiguous(o_strides, Hq, T, d, os);
+    if (!strides_ok(qs) || !strides_ok(os))
+        return fail(YR_EINVAL, f + ": strides must be positive multiples of 8 elements");
+    return YR_OK;
+}
+
+int launch_prepare(const void *k, const void *v, void *k_cache, float *k_rot_dbg, int B, int Hkv,
+                   int T, int d, const long long ks[3], const long long vs[3],
+                   const long long cs[3], const yr_rope_table *tab, void *workspace,
+                   int sm_count, cudaStream_t st) {
     __half *k16 = static_cast<__half *>(workspace);
     __half *v16 = k16 + static_cast<size_t>(B) * Hkv * T * d;
+    yr::KvPrepParams kp;
+    std::memset(&kp, 0, sizeof kp);
+    kp.k = static_cast<const __nv_bfloat16 *>(k);
+    kp.v = static_cast<const __nv_bfloat16 *>(v);
+    kp.ksb = ks[0]; kp.ksh = ks[1]; kp.kst = ks[2];
+    kp.vsb = vs[0]; kp.vsh = vs[1]; kp.vst = vs[2];
+    kp.k16 = k16;
+    kp.v16 = v16;
+    kp.kc = static_cast<__nv_bfloat16 *>(k_cache);
+    kp.csb = cs[0]; kp.csh = cs[1]; kp.cst = cs[2];
+    kp.k_dbg = k_rot_dbg;
+    kp.Hkv = Hkv; kp.T = T; kp.d = d;
+    kp.n_items = static_cast<long long>(B) * Hkv * T * (d / 8);
+    for (int i = 0; i < d / 2; ++i) kp.turns[i] = tab->turns[i];
+    long long blocks = (kp.n_items + 255) / 256;
+    const long long cap = static_cast<long long>(sm_count) * 16;
+    if (blocks > cap) blocks = cap;
+    yr::kv_prep_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(kp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("kv_prep_kernel launch", e);
+    return YR_OK;
+}
 
-    // 1) rotate keys once, lay K~ and V out as fp16
-    {
-        yr::KvPrepParams kp;
-        std::memset(&kp, 0, sizeof kp);
-        kp.k = static_cast<const __nv_bfloat16 *>(k);
-        kp.v = static_cast<const __nv_bfloat16 *>(v);
-        kp.ksb = ks[0]; kp.ksh = ks[1]; kp.kst = ks[2];
-        kp.vsb = vs[0]; kp.vsh = vs[1]; kp.vst = vs[2];
-        kp.k16 = k16;
-        kp.v16 = v16;
-        kp.kc = static_cast<__nv_bfloat16 *>(k_cache);
-        kp.csb = cs[0]; kp.csh = cs[1]; kp.cst = cs[2];
-        kp.k_dbg = k_rot_dbg;
-        kp.Hkv = Hkv; kp.T = T; kp.d = d;
-        kp.n_items = static_cast<long long>(B) * Hkv * T * (d / 8);
-        for (int i = 0; i < d / 2; ++i) kp.turns[i] = tab->turns[i];
-        long long blocks = (kp.n_items + 255) / 256;
-        const long long cap = static_cast<long long>(sm_count) * 16;
-        if (blocks > cap) blocks = cap;
-        yr::kv_prep_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(kp);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail("kv_prep_kernel launch", e);
-    }
-    // 2) attention
+int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, int Hq, int Hkv,
+                  int T, int d, const long long qs[3], const long long os[3],
+                  const yr_rope_table *tab, int causal, int window, int n_sink,
+                  const void *workspace, cudaStream_t st) {
+    const __half *k16 = static_cast<const __half *>(workspace);
+    const __half *v16 = k16 + static_cast<size_t>(B) * Hkv * T * d;
     yr::PrefillParams pp;
     std::memset(&pp, 0, sizeof pp);
+    int rc;
     {
         const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T),
                                     static_cast<cuuint64_t>(Hq), static_cast<cuuint64_t>(B)};
-        const cuuint64_t strides[3] = {static_cast<cuuint64_t>(qs[2] * 2), static_cast<cuuint64_t>(qs[1] * 2),
+        const cuuint64_t strides[3] = {static_cast<cuuint64_t>(qs[2] * 2),
+                                       static_cast<cuuint64_t>(qs[1] * 2),
                                        static_cast<cuuint64_t>(qs[0] * 2)};
         const cuuint32_t box[4] = {64, 128, 1, 1};
         rc = encode(&pp.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, q, dims, strides, box, "q");
@@ -261,9 +290,11 @@ extern "C" int yr_attn_prefill(const void *q, const void *k, const void *v, void
     {
         const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T),
                                     static_cast<cuuint64_t>(B) * Hkv};
-        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(T) * d * 2};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                       static_cast<cuuint64_t>(T) * d * 2};
         const cuuint32_t box[3] = {64, 128, 1};
-        rc = encode(&pp.tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, k16, dims, strides, box, "rotated k");
+        rc = encode(&pp.tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, k16, dims, strides, box,
+                    "rotated k");
         if (rc != YR_OK) return rc;
         rc = encode(&pp.tm_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, v16, dims, strides, box, "v");
         if (rc != YR_OK) return rc;
@@ -280,12 +311,78 @@ extern "C" int yr_attn_prefill(const void *q, const void *k, const void *v, void
     for (int i = 0; i < d / 2; ++i) pp.turns[i] = tab->turns[i];
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * Hq * pp.n_qblocks);
     if (d == 128)
-        yr::prefill_attn_kernel<128><<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<128>(), st>>>(pp);
+        yr::prefill_attn_kernel<128>
+            <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<128>(), st>>>(pp);
     else
-        yr::prefill_attn_kernel<64><<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<64>(), st>>>(pp);
+        yr::prefill_attn_kernel<64>
+            <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<64>(), st>>>(pp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("prefill_attn_kernel launch", e);
     return YR_OK;
+}
+
+}  // namespace yr_host
+
+extern "C" int yr_prefill_prepare_kv(const void *k, const void *v, void *k_cache,
+                                     float *k_rot_dbg, int B, int Hkv, int T, int d,
+                                     const int64_t *k_strides, const int64_t *v_strides,
+                                     const int64_t *kc_strides, const yr_rope_table *tab,
+                                     void *workspace, size_t workspace_bytes, void *stream) {
+    set_error("");
+    long long ks[3], vs[3], cs[3];
+    int rc = check_prepare(k, v, k_cache, k_rot_dbg, B, Hkv, T, d, k_strides, v_strides,
+                           kc_strides, tab, workspace, workspace_bytes, "yr_prefill_prepare_kv",
+                           ks, vs, cs);
+    if (rc != YR_OK) return rc;
+    int sm_count = 0;
+    rc = prepare_device(&sm_count);
+    if (rc != YR_OK) return rc;
+    return launch_prepare(k, v, k_cache, k_rot_dbg, B, Hkv, T, d, ks, vs, cs, tab, workspace,
+                          sm_count, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int yr_prefill_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B,
+                                 int Hq, int Hkv, int T, int d, const int64_t *q_strides,
+                                 const int64_t *o_strides, const yr_rope_table *tab, int causal,
+                                 int window, int n_sink, const void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+    set_error("");
+    long long qs[3], os[3];
+    int rc = check_attend(q, o, lse, q_rot_dbg, B, Hq, Hkv, T, d, q_strides, o_strides, tab,
+                          causal, window, n_sink, workspace, workspace_bytes, "yr_prefill_attend",
+                          qs, os);
+    if (rc != YR_OK) return rc;
+    rc = prepare_device(nullptr);
+    if (rc != YR_OK) return rc;
+    return launch_attend(q, o, lse, q_rot_dbg, B, Hq, Hkv, T, d, qs, os, tab, causal, window,
+                         n_sink, workspace, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int yr_attn_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
+                               void *k_cache, float *q_rot_dbg, float *k_rot_dbg, int B, int Hq,
+                               int Hkv, int T, int d, const int64_t *q_strides,
+                               const int64_t *k_strides, const int64_t *v_strides,
+                               const int64_t *o_strides, const int64_t *kc_strides,
+                               const yr_rope_table *tab, int causal, int window, int n_sink,
+                               void *workspace, size_t workspace_bytes, void *stream) {
+    set_error("");
+    long long qs[3], os[3], ks[3], vs[3], cs[3];
+    int rc = check_attend(q, o, lse, q_rot_dbg, B, Hq, Hkv, T, d, q_strides, o_strides, tab,
+                          causal, window, n_sink, workspace, workspace_bytes, "yr_attn_prefill",
+                          qs, os);
+    if (rc != YR_OK) return rc;
+    rc = check_prepare(k, v, k_cache, k_rot_dbg, B, Hkv, T, d, k_strides, v_strides, kc_strides,
+                       tab, workspace, workspace_bytes, "yr_attn_prefill", ks, vs, cs);
+    if (rc != YR_OK) return rc;
+    int sm_count = 0;
+    rc = prepare_device(&sm_count);
+    if (rc != YR_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = launch_prepare(k, v, k_cache, k_rot_dbg, B, Hkv, T, d, ks, vs, cs, tab, workspace,
+                        sm_count, st);
+    if (rc != YR_OK) return rc;
+    return launch_attend(q, o, lse, q_rot_dbg, B, Hq, Hkv, T, d, qs, os, tab, causal, window,
+                         n_sink, workspace, st);
 }
 
 extern "C" int yr_attn_decode(const void *q_new, const void *k_new, const void *v_new,
