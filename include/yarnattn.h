@@ -208,6 +208,35 @@ int yr_attn_decode(const void *q_new, const void *k_new, const void *v_new,
                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * attn_decode_noalloc -- yr_attn_decode for callers that cannot allocate device
+ * memory.  The pages have no counterpart: this is an interface for embedding.
+ * Some callers cannot call cudaMalloc: a plugin inside a host application that
+ * owns every byte of device memory and hands its plugins no scratch allocator,
+ * or a latency-bound serving loop that may not allocate once it is running
+ * (cudaMalloc can synchronise the device).  This entry point allocates nothing:
+ * the caller still passes inputs, caches and outputs, and the split-KV partial
+ * results go to a fixed scratch array inside the library instead of a workspace.
+ *   Limit: the scratch is YR_DECODE_NOALLOC_SCRATCH_BYTES (16 MiB) per device,
+ *   held by every GPU that loads the library until the process exits.  A call
+ *   that needs more -- yr_attn_decode_workspace_bytes(B, Hq, Hkv, d, T_max)
+ *   bytes -- returns YR_EINVAL without launching anything (e.g. 16 sequences of
+ *   32768 slots with 128 query and 8 KV heads of d=128 need just over 16 MiB).
+ *   The first call on each device looks up the scratch address for that device
+ *   with the CUDA runtime; make that first call before any stream capture.
+ *   Every call shares the one array, which keeps the last call's contents: calls
+ *   that overlap on the GPU (other streams, other host threads) race on it, so
+ *   order them.  Nothing in it needs to start at zero, because each call writes
+ *   every partial result it reads back.
+ * Other arguments, results and errors as yr_attn_decode.
+ */
+#define YR_DECODE_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+int yr_attn_decode_noalloc(const void *q_new, const void *k_new, const void *v_new,
+                           void *k_cache, void *v_cache, const int32_t *cache_len,
+                           void *o, float *lse, float *q_rot_dbg,
+                           int B, int Hq, int Hkv, int d, int T_max,
+                           const yr_rope_table *tab, int window, int n_sink, void *stream);
+
+/*
  * device_status -- synchronise `stream`, then read and clear the device status
  * word of the current device.  Returns YR_OK, YR_ETIMEOUT (a kernel gave up on
  * a wait; yr_last_error names where) or YR_EINVAL (a decode cache length was

@@ -19,7 +19,8 @@ ROPE, PI, NTK, YARN = 0, 1, 2, 3
 METHODS = {"rope": ROPE, "pi": PI, "ntk": NTK, "yarn": YARN}
 SYMBOLS = ("yr_rope_freq_table", "yr_attn_prefill_workspace_bytes", "yr_attn_prefill",
            "yr_prefill_prepare_kv", "yr_prefill_attend", "yr_attn_decode_workspace_bytes",
-           "yr_attn_decode", "yr_device_status", "yr_last_error", "yr_version")
+           "yr_attn_decode", "yr_attn_decode_noalloc", "yr_device_status", "yr_last_error",
+           "yr_version")
 
 
 class YarnAttnError(RuntimeError):
@@ -74,6 +75,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.yr_attn_decode.argtypes = ([vp] * 9 + [ci] * 5 +
                                    [ctypes.POINTER(RopeTable), ci, ci, vp, cs, vp])
     lib.yr_attn_decode.restype = ci
+    lib.yr_attn_decode_noalloc.argtypes = ([vp] * 9 + [ci] * 5 +
+                                           [ctypes.POINTER(RopeTable), ci, ci, vp])
+    lib.yr_attn_decode_noalloc.restype = ci
     lib.yr_device_status.argtypes = [vp]
     lib.yr_device_status.restype = ci
     lib.yr_last_error.argtypes = []
@@ -196,6 +200,27 @@ def attn_decode(q_new, k_new, v_new, k_cache, v_cache, cache_len, table: RopeTab
         _ptr(out), _ptr(lse), _ptr(q_rot_dbg), B, Hq, Hkv, d, T_max, ctypes.byref(table),
         int(window), int(n_sink), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream))
+    _check(rc)
+    return out
+
+
+def attn_decode_noalloc(q_new, k_new, v_new, k_cache, v_cache, cache_len, table: RopeTable,
+                        window: int = 0, n_sink: int = 0, out=None, lse=None, q_rot_dbg=None,
+                        stream=None):
+    """attn_decode with the library's fixed scratch instead of a workspace: the library
+    allocates nothing (for callers that cannot allocate device memory).  `out` must be given
+    by such callers; it is allocated here only as a convenience when omitted."""
+    B, Hq, d = q_new.shape
+    Hkv, T_max = k_cache.shape[1], k_cache.shape[2]
+    for t in (q_new, k_new, v_new, k_cache, v_cache, cache_len):
+        if not t.is_contiguous():
+            raise ValueError("attn_decode_noalloc expects contiguous tensors")
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q_new.device)
+    rc = load().yr_attn_decode_noalloc(
+        _ptr(q_new), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(cache_len),
+        _ptr(out), _ptr(lse), _ptr(q_rot_dbg), B, Hq, Hkv, d, T_max, ctypes.byref(table),
+        int(window), int(n_sink), _stream(stream))
     _check(rc)
     return out
 

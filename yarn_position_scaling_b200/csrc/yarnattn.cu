@@ -456,6 +456,63 @@ extern "C" int yr_attn_decode(const void *q_new, const void *k_new, const void *
     return YR_OK;
 }
 
+// ------------------------------------------------------------------------------
+// Decode without a caller-supplied workspace.  The split-KV partial results go to
+// this fixed array instead; every GPU that loads the library holds it until exit.
+// In host code `g_decode_noalloc_scratch` is only a stand-in for the symbol, not a
+// device address: the address is looked up per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[YR_DECODE_NOALLOC_SCRATCH_BYTES];
+
+namespace yr_host {
+std::mutex g_scratch_mu;
+void *g_scratch_ptr[64] = {};
+
+// Set-up, once per device, with that device current.
+int noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if (dev < 0 || dev >= 64) return fail(YR_EUNSUPPORTED, "device index out of range");
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_decode_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress(decode scratch)", e);
+        g_scratch_ptr[dev] = ptr;
+    }
+    *out = g_scratch_ptr[dev];
+    return YR_OK;
+}
+}  // namespace yr_host
+
+extern "C" int yr_attn_decode_noalloc(const void *q_new, const void *k_new, const void *v_new,
+                                      void *k_cache, void *v_cache, const int32_t *cache_len,
+                                      void *o, float *lse, float *q_rot_dbg, int B, int Hq,
+                                      int Hkv, int d, int T_max, const yr_rope_table *tab,
+                                      int window, int n_sink, void *stream) {
+    set_error("");
+    const size_t need = yr_attn_decode_workspace_bytes(B, Hq, Hkv, d, T_max);
+    if (need == 0)
+        return fail(YR_EINVAL, "yr_attn_decode_noalloc: invalid sizes (B, Hq, Hkv, d, T_max)");
+    if (need > static_cast<size_t>(YR_DECODE_NOALLOC_SCRATCH_BYTES))
+        return fail(YR_EINVAL, "yr_attn_decode_noalloc: this call needs " + std::to_string(need) +
+                                   " bytes of scratch, more than the fixed " +
+                                   std::to_string(YR_DECODE_NOALLOC_SCRATCH_BYTES) +
+                                   " bytes; use yr_attn_decode with a workspace");
+    void *scratch = nullptr;
+    int rc = noalloc_scratch(&scratch);
+    if (rc != YR_OK) return rc;
+    rc = yr_attn_decode(q_new, k_new, v_new, k_cache, v_cache, cache_len, o, lse, q_rot_dbg, B,
+                        Hq, Hkv, d, T_max, tab, window, n_sink, scratch,
+                        YR_DECODE_NOALLOC_SCRATCH_BYTES, stream);
+    if (rc != YR_OK) {
+        std::string m = g_err;
+        if (m.rfind("yr_attn_decode:", 0) == 0) m = "yr_attn_decode_noalloc:" + m.substr(15);
+        set_error(m);
+    }
+    return rc;
+}
+
 extern "C" int yr_device_status(void *stream) {
     set_error("");
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
