@@ -128,6 +128,12 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -329,13 +335,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     } else {
         // ------------------------------------------------- softmax warpgroups
         const int t = warp >> 2;
+        const int my_lo = t == 0 ? r_lo[0] : r_lo[1];
+        const int my_hi = t == 0 ? r_hi[0] : r_hi[1];
         const int lane_base = (warp & 3) * 32;
         const int r = lane_base + lane;  // row within the tile = TMEM lane
-        const int row = r_lo[t] + r;
+        const int row = my_lo + r;
         const uint32_t tm_lane = static_cast<uint32_t>(lane_base) << 16;
         const uint32_t tm_s = tmem + tm_lane + t * kBlockN;
         const uint32_t tm_o = tmem + tm_lane + 2 * kBlockN + t * HD;
-        const bool tile_live = r_lo[t] <= r_hi[t];
+        const bool tile_live = my_lo <= my_hi;
         bool ok = true;
 
         if (tile_live) {
@@ -381,12 +389,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
         }
 
-        float m_run = -INFINITY;  // running max, log2 units (scores * sl2)
-        float l_run = 0.0f;       // running sum of exp2(score*sl2 - m_run)
+        float m_run = -INFINITY;  // reference max of this row, log2 units (score * sl2)
+        float l_run = 0.0f;       // sum of exp2(score * sl2 - m_run) so far
         int it = 0;
+        const float sl2 = p.sl2;
+        const float2 sl2_2 = make_float2(sl2, sl2);
         for (int idx = 0; idx < tp.n && ok && tile_live; ++idx) {
             const int j = tile_at(tp, idx);
-            if (!tile_visible(p, r_lo[t], r_hi[t], j)) continue;
+            if (!tile_visible(p, my_lo, my_hi, j)) continue;
             ok = mbar_wait(&sm->s_full[t], it & 1, abort, p.timeout_ns);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
@@ -404,7 +414,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[c][e]);
                 }
             }
-            if (!tile_full(p, r_lo[t], r_hi[t], j)) {
+            if (!tile_full(p, my_lo, my_hi, j)) {
                 const int k0 = j * kBlockN;
 #pragma unroll
                 for (int c = 0; c < kBlockN; ++c) {
@@ -415,50 +425,75 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     if (!v) s[c] = -INFINITY;
                 }
             }
-            float mx = s[0];
+            // Tile max in four independent chains of three-input max.
+            float m4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-            for (int c = 1; c < kBlockN; ++c) mx = fmaxf(mx, s[c]);
-            const float m_tile = mx * p.sl2;
-            const bool need = m_tile > m_run + kRescaleThreshold;
-            if (__any_sync(0xffffffffu, need)) {
-                const float m_new = need ? fmaxf(m_run, m_tile) : m_run;
-                const float alpha = (m_run == -INFINITY) ? 0.0f : ex2(m_run - m_new);
+            for (int c = 4; c < kBlockN; c += 8) {
+                m4[0] = fmax3(m4[0], s[c], s[c + 1]);
+                m4[1] = fmax3(m4[1], s[c + 2], s[c + 3]);
+                m4[2] = fmax3(m4[2], s[c + 4], s[c + 5]);
+                m4[3] = fmax3(m4[3], s[c + 6], s[c + 7]);
+            }
+            const float m_tile = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * sl2;
+            // Once a row has a reference max, its exponentials need not wait for this
+            // tile's max: they are taken against the reference, and redone only when the
+            // tile raises the max by more than 2^kRescaleThreshold (then P would not fit).
+            const float m_use = (m_run == -INFINITY) ? m_tile : m_run;
+            auto exps_to_tmem = [&](float m_ref_in) -> float {
+                const float m_ref = (m_ref_in == -INFINITY) ? 0.0f : m_ref_in;
+                const float2 neg = make_float2(-m_ref, -m_ref);
+                float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                 make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+                for (int c = 0; c < kBlockN / 32; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float2 x = __ffma2_rn(
+                            make_float2(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]), sl2_2, neg);
+                        const float p0 = ex2(x.x), p1 = ex2(x.y);
+                        acc[e & 3] = __fadd2_rn(acc[e & 3], make_float2(p0, p1));
+                        pk[e] = pack_half2(p0, p1);
+                    }
+                    tmem_st16(tm_s + c * 16, pk);
+                }
+                const float2 a01 = __fadd2_rn(acc[0], acc[1]);
+                const float2 a23 = __fadd2_rn(acc[2], acc[3]);
+                const float2 a = __fadd2_rn(a01, a23);
+                return a.x + a.y;
+            };
+            float l_tile = exps_to_tmem(m_use);
+            const bool over = (m_run != -INFINITY) && (m_tile > m_run + kRescaleThreshold);
+            if (__any_sync(0xffffffffu, over)) {
+                // Rare: move the reference of the rows that overflowed and redo P.
+                const float m_new = over ? m_tile : m_use;
+                const float alpha = over ? ex2(m_run - m_new) : 1.0f;
+                tmem_st_wait();
+                l_tile = exps_to_tmem(m_new);
                 if (it > 0) {
                     // O holds P V up to the previous tile: wait for it, then rescale.
                     ok = mbar_wait(&sm->o_done[t], (it - 1) & 1, abort, p.timeout_ns);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
                     tc_fence_after();
-                    const float sc = need ? alpha : 1.0f;
                     uint32_t raw[32];
 #pragma unroll
                     for (int c = 0; c < HD / 32; ++c) {
                         tmem_ld32_sync(tm_o + c * 32, raw);
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
-                            raw[e] = __float_as_uint(__uint_as_float(raw[e]) * sc);
+                            raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
                         tmem_st32(tm_o + c * 32, raw);
                     }
-                    tmem_st_wait();
                 }
-                if (need) {
-                    l_run *= alpha;
-                    m_run = m_new;
-                }
+                l_run *= alpha;
+                m_run = m_new;
+            } else {
+                // Rows seen for the first time adopt this tile's max; their O and l are
+                // still zero, so nothing needs rescaling.
+                m_run = m_use;
             }
-            const float m_ref = (m_run == -INFINITY) ? 0.0f : m_run;
-#pragma unroll
-            for (int c = 0; c < kBlockN / 32; ++c) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2(fmaf(s[c * 32 + 2 * e], p.sl2, -m_ref));
-                    const float p1 = ex2(fmaf(s[c * 32 + 2 * e + 1], p.sl2, -m_ref));
-                    l_run += p0 + p1;
-                    pk[e] = pack_half2(p0, p1);
-                }
-                tmem_st16(tm_s + c * 16, pk);
-            }
+            l_run += l_tile;
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&sm->p_full[t]);
