@@ -15,9 +15,9 @@
 //
 // Online softmax ("Long Context" concept page, key math: scores never reach
 // HBM; "long-context-models", context parallelism: running row maxima,
-// normalisation sums and output accumulators): the running max is only moved
-// when a tile raises it by more than 2^8, so O is rescaled rarely; P stays
-// within [0, 256], which fp16 holds exactly enough.
+// normalisation sums and output accumulators): a row's reference max only
+// moves when its probabilities against the current reference would not fit
+// fp16 (some p > 2^15), so O is rescaled rarely and most tiles need no row max.
 //
 // Rotation ("Arch_03_Long_Context", RoPE slide): pair (2i, 2i+1) of the query
 // at position m turns by m * theta'_i.  The angle is reduced in fp64 as
@@ -35,12 +35,23 @@ namespace yr {
 constexpr int kBlockM = 128;
 constexpr int kBlockN = 128;
 constexpr int kQTiles = 2;
-constexpr int kKStages = 2;
+#ifndef YR_PREFILL_KSTAGES
+#define YR_PREFILL_KSTAGES 2
+#endif
+constexpr int kKStages = YR_PREFILL_KSTAGES;  // 2 or 3 (3 fits 227 KB only at d=128 with 2 V stages)
 constexpr int kVStages = 2;
-constexpr int kPrefillThreads = 320;
+constexpr int kPrefillThreads = 384;  // 3 warpgroups: softmax Q0, softmax Q1, load/MMA
+// Register split (setmaxnreg): the softmax warpgroups grow, the load/MMA one
+// shrinks.  256 * 216 + 128 * 64 = 63488 <= 384 * 168 registers at launch; the
+// host checks the launched count before the first launch.
+constexpr int kRegsSoftmax = 216;
+constexpr int kRegsOther = 64;
+constexpr int kMinLaunchRegs = (256 * kRegsSoftmax + 128 * kRegsOther + 383) / 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSubTileBytes = 128 * 128;  // 128 rows x 64 16-bit columns, 128-byte swizzle
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Upper bound on a row's probabilities within one tile before its reference max
+// must move: P is stored as fp16 (max 65504), so 2^15 leaves a factor of two.
+constexpr float kPBound = 32768.0f;
 
 struct alignas(64) PrefillParams {
     CUtensorMap tm_q;  // bf16 [B][Hq][T][d] (4-D, caller strides)
@@ -176,9 +187,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (threadIdx.x == 0) {
         for (int t = 0; t < kQTiles; ++t) {
             mbar_init(&sm->q_full[t], 1);
-            mbar_init(&sm->q_ready[t], kBlockM);
+            mbar_init(&sm->q_ready[t], kBlockM / 32);  // one arrival per softmax warp
             mbar_init(&sm->s_full[t], 1);
-            mbar_init(&sm->p_full[t], kBlockM);
+            mbar_init(&sm->p_full[t], kBlockM / 32);
             mbar_init(&sm->o_done[t], 1);
         }
         for (int s = 0; s < kKStages; ++s) {
@@ -208,7 +219,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint32_t tmem = sm->tmem_base;
     volatile int *abort = &sm->abort;
 
-    if (warp == 8) {
+    if (warp >= 8) {
+      // load/MMA warpgroup (warps 8-11; 10 and 11 have no role): shrink first
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+      if (warp == 8) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint64_t pol_q = l2_policy_evict_first();
@@ -332,8 +346,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             if (!mbar_wait_drain(&sm->mma_done, 0, p.timeout_ns)) raise_status(kStatusTimeoutDrain);
         }
         __syncwarp();
+      }
     } else {
         // ------------------------------------------------- softmax warpgroups
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
         const int t = warp >> 2;
         const int my_lo = t == 0 ? r_lo[0] : r_lo[1];
         const int my_hi = t == 0 ? r_hi[0] : r_hi[1];
@@ -385,7 +401,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     }
                 }
                 fence_proxy_async_smem();
-                mbar_arrive(&sm->q_ready[t]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm->q_ready[t]);
             }
         }
 
@@ -393,7 +410,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         float l_run = 0.0f;       // sum of exp2(score * sl2 - m_run) so far
         int it = 0;
         const float sl2 = p.sl2;
-        const float2 sl2_2 = make_float2(sl2, sl2);
         for (int idx = 0; idx < tp.n && ok && tile_live; ++idx) {
             const int j = tile_at(tp, idx);
             if (!tile_visible(p, my_lo, my_hi, j)) continue;
@@ -425,52 +441,60 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     if (!v) s[c] = -INFINITY;
                 }
             }
-            // Tile max in four independent chains of three-input max.
-            float m4[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-            for (int c = 4; c < kBlockN; c += 8) {
-                m4[0] = fmax3(m4[0], s[c], s[c + 1]);
-                m4[1] = fmax3(m4[1], s[c + 2], s[c + 3]);
-                m4[2] = fmax3(m4[2], s[c + 4], s[c + 5]);
-                m4[3] = fmax3(m4[3], s[c + 6], s[c + 7]);
-            }
-            const float m_tile = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * sl2;
-            // Once a row has a reference max, its exponentials need not wait for this
-            // tile's max: they are taken against the reference, and redone only when the
-            // tile raises the max by more than 2^kRescaleThreshold (then P would not fit).
-            const float m_use = (m_run == -INFINITY) ? m_tile : m_run;
             auto exps_to_tmem = [&](float m_ref_in) -> float {
+                // Scalar FMA and adds throughout: measured on sm_100a, a packed f32x2
+                // FMA feeding the scalar ex2 costs about twice as many cycles per
+                // element as two scalar FMAs.
                 const float m_ref = (m_ref_in == -INFINITY) ? 0.0f : m_ref_in;
-                const float2 neg = make_float2(-m_ref, -m_ref);
-                float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                                 make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                const float neg_m = -m_ref;
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int c = 0; c < kBlockN / 32; ++c) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float2 x = __ffma2_rn(
-                            make_float2(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]), sl2_2, neg);
-                        const float p0 = ex2(x.x), p1 = ex2(x.y);
-                        acc[e & 3] = __fadd2_rn(acc[e & 3], make_float2(p0, p1));
+                        const float p0 = ex2(fmaf(s[c * 32 + 2 * e], sl2, neg_m));
+                        const float p1 = ex2(fmaf(s[c * 32 + 2 * e + 1], sl2, neg_m));
+                        acc[(2 * e) & 7] += p0;
+                        acc[(2 * e + 1) & 7] += p1;
                         pk[e] = pack_half2(p0, p1);
                     }
                     tmem_st16(tm_s + c * 16, pk);
                 }
-                const float2 a01 = __fadd2_rn(acc[0], acc[1]);
-                const float2 a23 = __fadd2_rn(acc[2], acc[3]);
-                const float2 a = __fadd2_rn(a01, a23);
-                return a.x + a.y;
+                return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
             };
-            float l_tile = exps_to_tmem(m_use);
-            const bool over = (m_run != -INFINITY) && (m_tile > m_run + kRescaleThreshold);
+            // A row with a reference max takes its exponentials against it without
+            // looking at this tile's max: P only has to fit fp16, and since every
+            // p <= l_tile, l_tile <= kPBound proves it does.  Rows with no reference
+            // yet, and warps where some row fails the test, take the tile max, move
+            // the reference of those rows to it and redo P (rare after a row's first
+            // tile: the running max of a row grows slowly).
+            const bool have_ref = __all_sync(0xffffffffu, m_run != -INFINITY);
+            float l_tile = 0.0f;
+            bool over = true;
+            if (have_ref) {
+                l_tile = exps_to_tmem(m_run);
+                over = !(l_tile <= kPBound);
+            }
             if (__any_sync(0xffffffffu, over)) {
-                // Rare: move the reference of the rows that overflowed and redo P.
-                const float m_new = over ? m_tile : m_use;
-                const float alpha = over ? ex2(m_run - m_new) : 1.0f;
+                // Tile max in four independent chains of three-input max.
+                float m4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+                for (int c = 4; c < kBlockN; c += 8) {
+                    m4[0] = fmax3(m4[0], s[c], s[c + 1]);
+                    m4[1] = fmax3(m4[1], s[c + 2], s[c + 3]);
+                    m4[2] = fmax3(m4[2], s[c + 4], s[c + 5]);
+                    m4[3] = fmax3(m4[3], s[c + 6], s[c + 7]);
+                }
+                const float m_tile = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * sl2;
+                const bool first = m_run == -INFINITY;
+                const bool move = first || (have_ref && over && m_tile > m_run);
+                const float m_new = move ? fmaxf(m_run, m_tile) : m_run;
+                const bool rescale = !first && m_new > m_run;
+                const float alpha = rescale ? ex2(m_run - m_new) : 1.0f;
                 tmem_st_wait();
                 l_tile = exps_to_tmem(m_new);
-                if (it > 0) {
+                if (it > 0 && __any_sync(0xffffffffu, rescale)) {
                     // O holds P V up to the previous tile: wait for it, then rescale.
                     ok = mbar_wait(&sm->o_done[t], (it - 1) & 1, abort, p.timeout_ns);
                     ok = __all_sync(0xffffffffu, ok);
@@ -486,17 +510,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         tmem_st32(tm_o + c * 32, raw);
                     }
                 }
+                // Rows seen for the first time have O = 0 and l = 0: nothing to rescale.
                 l_run *= alpha;
                 m_run = m_new;
-            } else {
-                // Rows seen for the first time adopt this tile's max; their O and l are
-                // still zero, so nothing needs rescaling.
-                m_run = m_use;
             }
             l_run += l_tile;
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&sm->p_full[t]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm->p_full[t]);
             ++it;
         }
         if (!ok) {

@@ -62,6 +62,7 @@ uint64_t wait_timeout_ns() {
 struct DeviceState {
     bool ready = false;
     bool sm100 = false;
+    bool prefill_regs_ok = false;  // launched register count covers the setmaxnreg split
     int sm_count = 0;
 };
 std::mutex g_dev_mu;
@@ -102,6 +103,16 @@ int prepare_device(int *sm_count) {
                 e = cudaFuncSetAttribute(a.fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(a.bytes));
                 if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
+            }
+            // The prefill kernel re-splits its registers between warpgroups
+            // (setmaxnreg); that only works if the launch reserves enough of them.
+            st.prefill_regs_ok = true;
+            for (const void *fn : {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128>),
+                                   reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64>)}) {
+                cudaFuncAttributes fa;
+                e = cudaFuncGetAttributes(&fa, fn);
+                if (e != cudaSuccess) return cuda_fail("cudaFuncGetAttributes", e);
+                if (fa.numRegs < yr::kMinLaunchRegs) st.prefill_regs_ok = false;
             }
         }
         st.ready = true;
@@ -268,10 +279,20 @@ int launch_prepare(const void *k, const void *v, void *k_cache, float *k_rot_dbg
     return YR_OK;
 }
 
+int prefill_regs_ok() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    return g_dev[dev].prefill_regs_ok ? 1 : 0;
+}
+
 int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, int Hq, int Hkv,
                   int T, int d, const long long qs[3], const long long os[3],
                   const yr_rope_table *tab, int causal, int window, int n_sink,
                   const void *workspace, cudaStream_t st) {
+    if (!prefill_regs_ok())
+        return fail(YR_EUNSUPPORTED, "prefill kernel was built with too few registers per thread "
+                                     "for its warpgroup register split");
     const __half *k16 = static_cast<const __half *>(workspace);
     const __half *v16 = k16 + static_cast<size_t>(B) * Hkv * T * d;
     yr::PrefillParams pp;
