@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the 128K and sweep prefill workloads")
+    ap.add_argument("--other-steps", type=int, default=3)
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="sequences in the decode workload (default 8; smaller for profiling)")
     return ap.parse_args()
@@ -317,6 +320,26 @@ def decode_bench(w, steps, warmup, stream):
     return step, lens.tolist()
 
 
+def workload_prefill(w, steps, stream, dist, peak_t):
+    """Prefill of one more workload: attention-kernel TFLOP/s with causal (and window/sink)
+    FLOPs counted, and the whole step (rotated-key pass + attention)."""
+    step, keep = prefill_bench(w, steps, 2, stream)
+    flops = metrics.prefill_flops(w.B, w.Hq, w.T, w.d, w.causal, w.window, w.n_sink)
+    dist.barrier()
+    total_ms, (prep_ms, attn_ms) = time_events(step, steps, stream)
+    dist.barrier()
+    from yarn_position_scaling_b200 import api
+    api.device_status(stream)
+    total_ms, attn_ms = dist.max(total_ms), dist.max(attn_ms)
+    attn = flops / (attn_ms / steps * 1e-3) / 1e12
+    del keep, step
+    return {"method": w.method, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "window": w.window,
+            "n_sink": w.n_sink, "flops_per_step": flops, "steps": steps,
+            "step_tflops": throughput(flops, steps, total_ms, dist.world, 1e12),
+            "attn_kernel_tflops": attn, "attn_kernel_ms": attn_ms / steps,
+            "frac_of_peak": attn / peak_t}
+
+
 def e2e_prefill(w, steps, warmup, stream):
     """Through the public API with host buffers: pinned H2D of q, k, v, the call, D2H of o."""
     from yarn_position_scaling_b200 import api
@@ -409,6 +432,13 @@ def main():
     del dstep
     torch.cuda.empty_cache()
 
+    # ---------------- the other prefill workloads (128K, method/structure sweep)
+    others = {}
+    if not args.no_other_workloads:
+        for w in [synth.LLAMA3_128K] + synth.SWEEP:
+            others[w.name] = workload_prefill(w, args.other_steps, stream, dist, peak_t)
+            torch.cuda.empty_cache()
+
     # ---------------- end to end through the API with host buffers
     estep, h2d, d2h = e2e_prefill(wp, esteps, 2, stream)
     dist.barrier()
@@ -461,6 +491,7 @@ def main():
                          "timed_over": "the whole decode call (split + merge launches)"}},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": esteps},
+        "other_workloads": others,
         "cpu_baseline": cpu,
         "gpu_launches": 2 * steps,
         "clocks": clk,

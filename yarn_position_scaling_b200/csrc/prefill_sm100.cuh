@@ -5,7 +5,8 @@
 // the key/value tiles those rows can see:
 //   warp 8      TMA producer: Q tiles once, then K~/V tiles through a 2-stage ring
 //   warp 9      MMA issuer: S_t = Q_t K~^T and O_t += P_t V with tcgen05.mma,
-//               accumulators in tensor memory (TMEM)
+//               accumulators in tensor memory (TMEM); the whole warp runs the
+//               loop and one elected lane issues
 //   warps 0-3   softmax for Q0, warps 4-7 softmax for Q1: each thread owns one
 //               query row (= one TMEM lane), so row max and row sum need no
 //               shuffles; P is written back over S in TMEM as fp16
@@ -42,10 +43,10 @@ constexpr int kKStages = YR_PREFILL_KSTAGES;  // 2 or 3 (3 fits 227 KB only at d
 constexpr int kVStages = 2;
 constexpr int kPrefillThreads = 384;  // 3 warpgroups: softmax Q0, softmax Q1, load/MMA
 // Register split (setmaxnreg): the softmax warpgroups grow, the load/MMA one
-// shrinks.  256 * 216 + 128 * 64 = 63488 <= 384 * 168 registers at launch; the
+// shrinks.  256 * 200 + 128 * 96 = 63488 <= 384 * 168 registers at launch; the
 // host checks the launched count before the first launch.
-constexpr int kRegsSoftmax = 216;
-constexpr int kRegsOther = 64;
+constexpr int kRegsSoftmax = 200;
+constexpr int kRegsOther = 96;
 constexpr int kMinLaunchRegs = (256 * kRegsSoftmax + 128 * kRegsOther + 383) / 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSubTileBytes = 128 * 128;  // 128 rows x 64 16-bit columns, 128-byte swizzle
@@ -273,79 +274,101 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         __syncwarp();
     } else if (warp == 9) {
         // ------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_f16_f32(kBlockM, kBlockN, false, false);
-            constexpr uint32_t idesc_o = idesc_f16_f32(kBlockM, HD, false, true);
-            bool ok = true;
-            bool vis[kQTiles];
-            int pv_count[kQTiles] = {0, 0};
-            for (int t = 0; t < kQTiles && ok; ++t)
-                if (r_lo[t] <= r_hi[t]) ok = mbar_wait(&sm->q_ready[t], 0, abort, p.timeout_ns);
-            tc_fence_after();
+        // The whole warp runs this loop, so its control flow and every operand
+        // descriptor are warp-uniform; one elected lane issues the tcgen05.mma
+        // and tcgen05.commit instructions.
+        const bool leader = elect_one();
+        constexpr uint32_t idesc_s = idesc_f16_f32(kBlockM, kBlockN, false, false);
+        constexpr uint32_t idesc_o = idesc_f16_f32(kBlockM, HD, false, true);
+        constexpr uint32_t kStageBytes = kSub * kSubTileBytes;
+        const uint64_t desc_q0 = sw128_desc(smem_u32(sm->q[0][0]), 16, 1024);
+        const uint64_t desc_q1 = sw128_desc(smem_u32(sm->q[1][0]), 16, 1024);
+        const uint64_t desc_k = sw128_desc(smem_u32(sm->k[0][0]), 16, 1024);
+        const uint64_t desc_v = sw128_desc(smem_u32(sm->v[0][0]), kSubTileBytes, 1024);
+        bool ok = true;
+        bool vis[kQTiles];
+        int pv_count[kQTiles] = {0, 0};
+        for (int t = 0; t < kQTiles; ++t)
+            if (ok && r_lo[t] <= r_hi[t])
+                ok = __all_sync(0xffffffffu, mbar_wait(&sm->q_ready[t], 0, abort, p.timeout_ns));
+        tc_fence_after();
 
-            auto issue_s = [&](int t, int ks) {
-                const uint32_t qa = smem_u32(sm->q[t][0]);
-                const uint32_t ka = smem_u32(sm->k[ks][0]);
+        // Descriptors advance by (byte offset >> 4) in their start-address field.
+        auto issue_s = [&](int t, int ks) {
+            const uint64_t da = t == 0 ? desc_q0 : desc_q1;
+            const uint64_t db = desc_k + ((ks * kStageBytes) >> 4);
+            if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kSubTileBytes + (kk & 3) * 32;
-                    mma_ss(tmem + t * kBlockN, sw128_desc(qa + off, 16, 1024),
-                           sw128_desc(ka + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                    const uint32_t off = ((kk >> 2) * kSubTileBytes + (kk & 3) * 32) >> 4;
+                    mma_ss(tmem + t * kBlockN, da + off, db + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&sm->s_full[t]);
-            };
-            auto issue_pv = [&](int t, int vs) -> bool {
-                if (!mbar_wait(&sm->p_full[t], pv_count[t] & 1, abort, p.timeout_ns)) return false;
-                tc_fence_after();
-                const uint32_t va = smem_u32(sm->v[vs][0]);
+            }
+            __syncwarp();
+        };
+        auto issue_pv = [&](int t, int vs) -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm->p_full[t], pv_count[t] & 1, abort, p.timeout_ns)))
+                return false;
+            tc_fence_after();
+            const uint64_t db = desc_v + ((vs * kStageBytes) >> 4);
+            const uint32_t first = pv_count[t] > 0 ? 1u : 0u;
+            if (leader) {
 #pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                for (int kk = 0; kk < kBlockN / 16; ++kk)
                     mma_ts(tmem + 2 * kBlockN + t * HD, tmem + t * kBlockN + kk * 8,
-                           sw128_desc(va + kk * 2048, kSubTileBytes, 1024), idesc_o,
-                           (pv_count[t] > 0 || kk > 0) ? 1u : 0u);
-                }
+                           db + ((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : first);
                 mma_commit(&sm->o_done[t]);
-                ++pv_count[t];
-                return true;
-            };
+            }
+            __syncwarp();
+            ++pv_count[t];
+            return true;
+        };
 
-            bool prev_vis1 = false;
-            for (int idx = 0; idx < tp.n && ok; ++idx) {
-                const int j = tile_at(tp, idx);
-                const int ks = idx % kKStages, vs = idx % kVStages;
-                for (int t = 0; t < kQTiles; ++t) vis[t] = tile_visible(p, r_lo[t], r_hi[t], j);
-                ok = mbar_wait(&sm->k_full[ks], (idx / kKStages) & 1, abort, p.timeout_ns);
+        bool prev_vis1 = false;
+        for (int idx = 0; idx < tp.n && ok; ++idx) {
+            const int j = tile_at(tp, idx);
+            const int ks = idx % kKStages, vs = idx % kVStages;
+            for (int t = 0; t < kQTiles; ++t) vis[t] = tile_visible(p, r_lo[t], r_hi[t], j);
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(&sm->k_full[ks], (idx / kKStages) & 1, abort, p.timeout_ns));
+            if (!ok) break;
+            tc_fence_after();
+            if (vis[0]) issue_s(0, ks);
+            if (idx > 0 && prev_vis1) {
+                ok = issue_pv(1, (idx - 1) % kVStages);
                 if (!ok) break;
-                tc_fence_after();
-                if (vis[0]) issue_s(0, ks);
-                if (idx > 0) {
-                    const int pvs = (idx - 1) % kVStages;
-                    if (prev_vis1) ok = issue_pv(1, pvs);
-                    if (!ok) break;
-                }
-                if (vis[1]) issue_s(1, ks);
+            }
+            if (vis[1]) issue_s(1, ks);
+            if (leader) {
                 mma_commit(&sm->k_empty[ks]);
                 if (idx > 0) mma_commit(&sm->v_empty[(idx - 1) % kVStages]);
-                ok = mbar_wait(&sm->v_full[vs], (idx / kVStages) & 1, abort, p.timeout_ns);
-                if (!ok) break;
-                tc_fence_after();
-                if (vis[0]) ok = issue_pv(0, vs);
-                prev_vis1 = vis[1];
             }
-            if (ok && tp.n > 0) {
-                const int vs = (tp.n - 1) % kVStages;
-                if (prev_vis1) ok = issue_pv(1, vs);
-                if (ok) mma_commit(&sm->v_empty[vs]);
-            }
-            if (!ok) {
+            __syncwarp();
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(&sm->v_full[vs], (idx / kVStages) & 1, abort, p.timeout_ns));
+            if (!ok) break;
+            tc_fence_after();
+            if (vis[0]) ok = issue_pv(0, vs);
+            prev_vis1 = vis[1];
+        }
+        if (ok && tp.n > 0) {
+            const int vs = (tp.n - 1) % kVStages;
+            if (prev_vis1) ok = issue_pv(1, vs);
+            if (ok && leader) mma_commit(&sm->v_empty[vs]);
+            __syncwarp();
+        }
+        if (!ok) {
+            if (leader) {
                 raise_status(kStatusTimeoutMma);
                 sm->abort = 1;
             }
-            // Drain: all MMAs issued above complete before TMEM/smem go away.
-            mma_commit(&sm->mma_done);
-            if (!mbar_wait_drain(&sm->mma_done, 0, p.timeout_ns)) raise_status(kStatusTimeoutDrain);
         }
+        // Drain: all MMAs issued above complete before TMEM/smem go away.
+        if (leader) mma_commit(&sm->mma_done);
         __syncwarp();
+        if (!__all_sync(0xffffffffu, mbar_wait_drain(&sm->mma_done, 0, p.timeout_ns)) && leader)
+            raise_status(kStatusTimeoutDrain);
       }
     } else {
         // ------------------------------------------------- softmax warpgroups
