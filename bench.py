@@ -66,21 +66,34 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def ncu_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the last ncu capture, or None when the kernel
-    sources changed since that capture (profiles/traffic.json keeps their hash)."""
-    import glob
+KERNEL_SOURCES = {
+    "prefill_attn_kernel<128>": ["prefill_sm100.cuh"],
+    "kv_prep_kernel": ["kvprep_sm100.cuh"],
+    "decode_split_kernel<128,1>": ["decode_sm100.cuh"],
+}
+
+
+def kernel_source_sha(kernel: str) -> str:
+    """Hash of the sources that define `kernel` (its own header plus the shared PTX and
+    status helpers)."""
     import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel] + ["sm100_ptx.cuh", "yr_status.cuh"]:
+        with open(os.path.join(ROOT, "yarn_position_scaling_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the last ncu capture of it, or None when its
+    sources changed since that capture (profiles/traffic.json keeps their hash)."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
-        h = hashlib.sha256()
-        for src in sorted(glob.glob(os.path.join(ROOT, "yarn_position_scaling_b200", "csrc", "*"))):
-            with open(src, "rb") as f:
-                h.update(f.read())
-        if h.hexdigest()[:16] != t["source_sha"] or kernel not in t:
+        rec = t[kernel]
+        if rec["source_sha"] != kernel_source_sha(kernel):
             return None
-        return float(t[kernel]["dram_read"] + t[kernel]["dram_write"])
+        return float(rec["dram_read"] + rec["dram_write"])
     except Exception:
         return None
 
@@ -472,6 +485,8 @@ def main():
                      "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": attn_tflops / peak_t, "peak_source": f"{peak_src} bf16 burst "
                      "(fp16 tensor rate equals bf16)",
+                     "peak_sustained": peaks["bf16_tflops_sustained"],
+                     "frac_of_sustained": attn_tflops / peaks["bf16_tflops_sustained"],
                      "traffic": ncu_traffic("prefill_attn_kernel<128>"),
                      "algorithmic_flops_per_launch": flops_step,
                      "kernel_ms": attn_ms_max / steps,

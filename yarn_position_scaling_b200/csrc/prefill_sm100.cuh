@@ -65,6 +65,7 @@ struct alignas(64) PrefillParams {
     int B, Hq, Hkv, T, group;
     int causal, window, n_sink;
     int n_qblocks;
+    int kv_major;  // CTA order: 1 = by KV head first (grouped heads), 0 = by query block
     float sl2;  // softmax_scale * log2(e)
     unsigned long long timeout_ns;
     double turns[64];
@@ -167,13 +168,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Heaviest causal blocks first; the heads of one query block are adjacent so
-    // the query heads that share a KV head read the same K/V tiles close in time.
-    const int bh_count = p.B * p.Hq;
-    const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x) / bh_count;
-    const int rem = static_cast<int>(blockIdx.x) % bh_count;
-    const int b = rem / p.Hq;
-    const int h = rem % p.Hq;
+    int qb, b, h;
+    if (p.kv_major) {
+        // Grouped heads: one (batch, KV head) after another, its query blocks
+        // heaviest first and the query heads of its group adjacent, so the CTAs
+        // resident at any time read the K/V of one or two KV heads, which stay in L2.
+        const int per_kv = p.n_qblocks * p.group;
+        const int bk = static_cast<int>(blockIdx.x) / per_kv;
+        const int rem = static_cast<int>(blockIdx.x) % per_kv;
+        qb = p.n_qblocks - 1 - rem / p.group;
+        b = bk / p.Hkv;
+        h = (bk % p.Hkv) * p.group + rem % p.group;
+    } else {
+        // Heaviest causal blocks first, the heads of one query block adjacent.
+        const int bh_count = p.B * p.Hq;
+        qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x) / bh_count;
+        const int rem = static_cast<int>(blockIdx.x) % bh_count;
+        b = rem / p.Hq;
+        h = rem % p.Hq;
+    }
     const int kvh = h / p.group;
     const int q0 = qb * (kQTiles * kBlockM);
     const int last_row = min(q0 + kQTiles * kBlockM - 1, p.T - 1);

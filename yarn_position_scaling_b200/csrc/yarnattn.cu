@@ -327,6 +327,9 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     pp.B = B; pp.Hq = Hq; pp.Hkv = Hkv; pp.T = T; pp.group = Hq / Hkv;
     pp.causal = causal; pp.window = window; pp.n_sink = n_sink;
     pp.n_qblocks = (T + 255) / 256;
+    // Grouped query heads read each K/V tile several times: order the CTAs by KV head
+    // so that re-reads hit L2 (measured: +2.7% at the 128K GQA workload, neutral for MHA).
+    pp.kv_major = pp.group > 1 ? 1 : 0;
     pp.sl2 = static_cast<float>(tab->softmax_scale * 1.4426950408889634);
     pp.timeout_ns = wait_timeout_ns();
     for (int i = 0; i < d / 2; ++i) pp.turns[i] = tab->turns[i];
