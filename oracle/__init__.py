@@ -23,7 +23,9 @@ import threading
 import numpy as np
 
 ROPE, PI, NTK, YARN = 0, 1, 2, 3
-METHODS = {"rope": ROPE, "pi": PI, "ntk": NTK, "yarn": YARN}
+NTK_DYNAMIC, YARN_DIMRAMP, FACTORS = 4, 5, 6
+METHODS = {"rope": ROPE, "pi": PI, "ntk": NTK, "yarn": YARN, "ntk_dynamic": NTK_DYNAMIC,
+           "yarn_dimramp": YARN_DIMRAMP, "factors": FACTORS}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "yarn_oracle.c")
@@ -60,6 +62,10 @@ def _load():
         lib.oracle_rope_theta.argtypes = [c_int, c_double, c_int, c_double, c_int,
                                           c_double, c_double, dp, dp, dp]
         lib.oracle_rope_theta.restype = c_int
+        lib.oracle_rope_theta_ext.argtypes = [c_int, c_double, c_int, c_double, c_int,
+                                              c_double, c_double, c_int, dp, c_double,
+                                              dp, dp, dp]
+        lib.oracle_rope_theta_ext.restype = c_int
         lib.oracle_rotate_rows.argtypes = [u16p, c_long, c_int, dp, dp, dp]
         lib.oracle_rotate_rows.restype = None
         lib.oracle_rotate_rows_f64.argtypes = [dp, c_long, c_int, dp, dp, dp]
@@ -94,16 +100,23 @@ def _bits(x) -> np.ndarray:
 
 
 def rope_theta(d: int, base: float, L_train: int, s: float, method, alpha: float = 1.0,
-               beta: float = 32.0):
-    """theta'_i (float64[d/2]), mscale and softmax_scale for one method."""
+               beta: float = 32.0, L_cur: int = 0, factors=None, attn_factor: float = 0.0):
+    """theta'_i (float64[d/2]), mscale and softmax_scale for one method.  L_cur is the
+    current sequence length (dynamic NTK); factors the per-dimension divisors and
+    attn_factor the temperature of the factor method."""
     lib = _load()
     m = METHODS[method] if isinstance(method, str) else int(method)
     th = np.zeros(d // 2, dtype=np.float64)
     ms = ctypes.c_double()
     ss = ctypes.c_double()
-    rc = lib.oracle_rope_theta(int(d), float(base), int(L_train), float(s), m, float(alpha),
-                               float(beta), _ptr(th, ctypes.c_double), ctypes.byref(ms),
-                               ctypes.byref(ss))
+    f = None if factors is None else np.ascontiguousarray(factors, dtype=np.float64)
+    if f is not None and f.shape != (d // 2,):
+        raise ValueError("factors must hold d/2 values")
+    rc = lib.oracle_rope_theta_ext(int(d), float(base), int(L_train), float(s), m, float(alpha),
+                                   float(beta), int(L_cur),
+                                   None if f is None else _ptr(f, ctypes.c_double),
+                                   float(attn_factor), _ptr(th, ctypes.c_double),
+                                   ctypes.byref(ms), ctypes.byref(ss))
     if rc != 0:
         raise ValueError("oracle_rope_theta: invalid arguments")
     return th, ms.value, ss.value

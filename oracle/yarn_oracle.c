@@ -34,6 +34,13 @@
  *   oracle_rope_theta   pinned (closed forms, s=1 reductions, NTK worked
  *                       number, band endpoints); the YaRN ramp INTERIOR is
  *                       a reading of the pages: parity unpinned there.
+ *   oracle_rope_theta_ext  dynamic NTK pinned (RoPE at or below L_train, equal
+ *                       to NTK at L_cur = s L_train, the page's ~82,000 base);
+ *                       dimension-ramp YaRN pinned outside its ramp and at the
+ *                       ramp's midpoint (a linear ramp's closed form), its
+ *                       edges pinned against the r-space band edges; factors
+ *                       pinned by f = 1 (RoPE), f = s (PI) and f = theta /
+ *                       theta'(YaRN) (YaRN's frequencies).
  *   oracle_rotate_rows  pinned (page's rotation matrix, complex-number
  *                       form, orthogonality, relative-position invariance).
  *   oracle_attn_rows    pinned (library SDPA special case, closed-form
@@ -50,6 +57,9 @@
 #define OR_PI 1
 #define OR_NTK 2
 #define OR_YARN 3
+#define OR_NTK_DYNAMIC 4
+#define OR_YARN_DIMRAMP 5
+#define OR_FACTORS 6
 
 static double bf16_bits_to_double(uint16_t bits)
 {
@@ -61,8 +71,8 @@ static double bf16_bits_to_double(uint16_t bits)
 }
 
 /*
- * Per-pair rotation frequencies theta'_i (i = 0 .. d/2-1), the YaRN mscale
- * and the softmax logit scale.
+ * Per-pair rotation frequencies theta'_i (i = 0 .. d/2-1), the attention
+ * temperature mscale and the softmax logit scale.
  *   RoPE  theta_i = base^(-2i/d)                       [P1] position wall; [P3] RoPE slide
  *   PI    theta'_i = theta_i / s                        [P1]; [P3] PI slide (angles of m/s); [P4] sec. 2
  *   NTK   theta'_i = (base * s^(d/(d-2)))^(-2i/d)       [P3] NTK-aware slide
@@ -71,20 +81,55 @@ static double bf16_bits_to_double(uint16_t bits)
  *         theta'_i = gamma_i * theta_i + (1 - gamma_i) * theta_i / s
  *         (short wavelengths unchanged, long wavelengths interpolated as PI,
  *          linear ramp between; alpha = 1, beta = 32 per the steps table)
- *   mscale = 0.1 ln s + 1 for YaRN, else 1             [P1] position wall; [P3] YaRN slide
+ *   Dynamic NTK  NTK with s = max(1, L_cur / L_train), the current sequence
+ *         length over the training length            [P3] NTK-aware slide, last sentence
+ *   YaRN, dimension ramp  the same band split with the ramp linear in the pair
+ *         index: i_edge(r) = d ln(L_train / (2 pi r)) / (2 ln base) is the
+ *         (fractional) index where r_i = r; low = floor(i_edge(beta)),
+ *         high = ceil(i_edge(alpha)); gamma_i = 1 - clamp((i - low) / (high - low), 0, 1)
+ *         ([P1]'s code structure: band-edge indices from a log ratio, floor
+ *          and ceil, a linear ramp over the index)
+ *   Per-dimension factors  theta'_i = theta_i / f_i for caller-supplied f_i > 0
+ *         ([P4] LongRoPE: searched non-uniform interpolation factors per
+ *          dimension; [P5] LongRoPE); mscale = the caller's attention factor,
+ *         1 when none is given
+ *   mscale = 0.1 ln s + 1 for both YaRN forms, else 1  [P1] position wall; [P3] YaRN slide
  *   softmax_scale = mscale^2 / sqrt(d)
  * Returns 0, or -1 for an invalid argument (odd or non-positive d, s < 1,
- * base <= 1, beta <= alpha for YaRN, L_train < 1 for YaRN).
+ * base <= 1, beta <= alpha or L_train < 1 for the YaRN forms and dynamic NTK,
+ * L_cur < 1 for dynamic NTK, missing or non-positive factors).
  */
-int oracle_rope_theta(int d, double base, int L_train, double s, int method,
-                      double alpha, double beta, double *theta,
-                      double *mscale, double *softmax_scale)
+int oracle_rope_theta_ext(int d, double base, int L_train, double s, int method,
+                          double alpha, double beta, int L_cur, const double *factors,
+                          double attn_factor, double *theta, double *mscale,
+                          double *softmax_scale)
 {
     if (d <= 0 || (d % 2) != 0) return -1;
     if (!(s >= 1.0) || !(base > 1.0)) return -1;
-    if (method < OR_ROPE || method > OR_YARN) return -1;
-    if (method == OR_YARN && (!(beta > alpha) || L_train < 1)) return -1;
+    if (method < OR_ROPE || method > OR_FACTORS) return -1;
+    const int yarn = method == OR_YARN || method == OR_YARN_DIMRAMP;
+    if (yarn && (!(beta > alpha) || L_train < 1)) return -1;
+    if (method == OR_NTK_DYNAMIC && (L_train < 1 || L_cur < 1)) return -1;
     const int half = d / 2;
+    if (method == OR_FACTORS) {
+        if (factors == NULL) return -1;
+        for (int i = 0; i < half; ++i)
+            if (!(factors[i] > 0.0)) return -1;
+    }
+    /* Band-edge indices of the dimension ramp. */
+    double low = 0.0, high = 1.0;
+    if (method == OR_YARN_DIMRAMP) {
+        const double i_beta = (double)d * log((double)L_train / (2.0 * M_PI * beta)) / (2.0 * log(base));
+        const double i_alpha = (double)d * log((double)L_train / (2.0 * M_PI * alpha)) / (2.0 * log(base));
+        low = floor(i_beta);
+        high = ceil(i_alpha);
+        if (low < 0.0) low = 0.0;
+        if (high > (double)(half - 1)) high = (double)(half - 1);
+        if (!(high > low)) high = low + 1.0;
+    }
+    const double s_dyn = (method == OR_NTK_DYNAMIC && (double)L_cur > (double)L_train)
+                             ? (double)L_cur / (double)L_train
+                             : 1.0;
     for (int i = 0; i < half; ++i) {
         const double expo = -2.0 * (double)i / (double)d;
         const double th = pow(base, expo);
@@ -94,19 +139,42 @@ int oracle_rope_theta(int d, double base, int L_train, double s, int method,
         } else if (method == OR_NTK) {
             const double base_ntk = base * pow(s, (double)d / (double)(d - 2));
             out = pow(base_ntk, expo);
+        } else if (method == OR_NTK_DYNAMIC) {
+            const double base_ntk = base * pow(s_dyn, (double)d / (double)(d - 2));
+            out = pow(base_ntk, expo);
         } else if (method == OR_YARN) {
             const double r = (double)L_train * th / (2.0 * M_PI);
             double g = (r - alpha) / (beta - alpha);
             if (g < 0.0) g = 0.0;
             if (g > 1.0) g = 1.0;
             out = g * th + (1.0 - g) * th / s;
+        } else if (method == OR_YARN_DIMRAMP) {
+            double ramp = ((double)i - low) / (high - low);
+            if (ramp < 0.0) ramp = 0.0;
+            if (ramp > 1.0) ramp = 1.0;
+            const double g = 1.0 - ramp;
+            out = g * th + (1.0 - g) * th / s;
+        } else if (method == OR_FACTORS) {
+            out = th / factors[i];
         }
         theta[i] = out;
     }
-    const double m = (method == OR_YARN) ? 0.1 * log(s) + 1.0 : 1.0;
+    double m = 1.0;
+    if (yarn) m = 0.1 * log(s) + 1.0;
+    if (method == OR_FACTORS && attn_factor > 0.0) m = attn_factor;
     if (mscale) *mscale = m;
     if (softmax_scale) *softmax_scale = m * m / sqrt((double)d);
     return 0;
+}
+
+/* The four fixed-table methods (RoPE, PI, NTK, YaRN). */
+int oracle_rope_theta(int d, double base, int L_train, double s, int method,
+                      double alpha, double beta, double *theta,
+                      double *mscale, double *softmax_scale)
+{
+    if (method < OR_ROPE || method > OR_YARN) return -1;
+    return oracle_rope_theta_ext(d, base, L_train, s, method, alpha, beta, 0, NULL, 0.0,
+                                 theta, mscale, softmax_scale);
 }
 
 /*

@@ -146,6 +146,78 @@ def test_invalid_table_arguments_rejected():
         oracle.rope_theta(64, 1e4, 64, 2.0, "yarn", 32.0, 1.0)
 
 
+# --------------------------------- table variants: dynamic NTK, dimension ramp, factors
+
+@pytest.mark.parametrize("L_cur", [1, 100, 4095, 4096])
+def test_dynamic_ntk_is_rope_up_to_L_train(L_cur):
+    # s = max(1, L_cur / L_train): no scaling while the sequence fits the training length
+    rope, _, _ = oracle.rope_theta(128, 10000.0, 4096, 1.0, "rope")
+    th, ms, _ = oracle.rope_theta(128, 10000.0, 4096, 1.0, "ntk_dynamic", L_cur=L_cur)
+    np.testing.assert_array_equal(th, rope)
+    assert ms == 1.0
+
+
+@pytest.mark.parametrize("k", [2, 3, 8])
+def test_dynamic_ntk_equals_static_ntk_at_the_ratio(golden, k):
+    dyn, _, _ = oracle.rope_theta(128, 10000.0, 4096, 1.0, "ntk_dynamic", L_cur=k * 4096)
+    stat, _, _ = oracle.rope_theta(128, 10000.0, 4096, float(k), "ntk")
+    np.testing.assert_allclose(dyn, stat, rtol=1e-15)
+    if k == 8:  # the page's worked number: base ~ 10000 * 8^(128/126) ~ 82,000
+        g = golden("pages_worked_numbers.json")["ntk_base"]
+        assert dyn[1] ** (-64) == pytest.approx(g["printed_base"], rel=g["rel_tol"])
+
+
+@pytest.mark.parametrize("d,base,L,s,low,high", [
+    (128, 10000.0, 4096, 4.0, 20, 46),    # 16K workload: r-space bands 0-20 | 21-45 | 46-63
+    (128, 500000.0, 8192, 16.0, 18, 35),  # 128K workload: r-space bands 0-18 | 19-34 | 35-63
+])
+def test_yarn_dimension_ramp_edges_and_midpoint(golden, d, base, L, s, low, high):
+    g = golden("pages_worked_numbers.json")["yarn_defaults"]
+    rope, _, _ = oracle.rope_theta(d, base, L, 1.0, "rope")
+    th, ms, ss = oracle.rope_theta(d, base, L, s, "yarn_dimramp", g["alpha"], g["beta"])
+    # outside the ramp: the same bands as the wavelength split (pinned above)
+    hi, _, lo = _bands(d, base, L, g["alpha"], g["beta"])
+    assert hi.max() == low and lo.min() == high
+    np.testing.assert_array_equal(th[: low + 1], rope[: low + 1])
+    np.testing.assert_allclose(th[high:], rope[high:] / s, rtol=1e-15)
+    # inside: linear in the index, so kept fractions of mirrored indices add up to one
+    frac = (th - rope / s) / (rope - rope / s)
+    for i in range(low, high + 1):
+        assert frac[i] == pytest.approx((high - i) / (high - low), abs=1e-12)
+        assert frac[i] + frac[low + high - i] == pytest.approx(1.0, abs=1e-12)
+    # the same temperature as YaRN
+    assert ms == pytest.approx(0.1 * math.log(s) + 1.0, rel=1e-15)
+    assert ss == pytest.approx(ms * ms / math.sqrt(d), rel=1e-15)
+
+
+def test_factor_table_reductions():
+    d, base, L, s = 128, 10000.0, 4096, 8.0
+    rope, _, _ = oracle.rope_theta(d, base, L, 1.0, "rope")
+    pi, _, _ = oracle.rope_theta(d, base, L, s, "pi")
+    yarn, _, _ = oracle.rope_theta(d, base, L, s, "yarn")
+    th, ms, ss = oracle.rope_theta(d, base, L, 1.0, "factors", factors=np.ones(d // 2))
+    np.testing.assert_array_equal(th, rope)
+    assert ms == 1.0 and ss == pytest.approx(1 / math.sqrt(d), rel=1e-15)
+    th, _, _ = oracle.rope_theta(d, base, L, 1.0, "factors", factors=np.full(d // 2, s))
+    np.testing.assert_allclose(th, pi, rtol=1e-15)
+    th, ms, ss = oracle.rope_theta(d, base, L, 1.0, "factors", factors=rope / yarn,
+                                   attn_factor=1.2)
+    np.testing.assert_allclose(th, yarn, rtol=1e-14)
+    assert ms == 1.2 and ss == pytest.approx(1.44 / math.sqrt(d), rel=1e-15)
+
+
+def test_table_variant_arguments_rejected():
+    with pytest.raises(ValueError):
+        oracle.rope_theta(64, 1e4, 64, 1.0, "ntk_dynamic", L_cur=0)
+    with pytest.raises(ValueError):
+        oracle.rope_theta(64, 1e4, 64, 1.0, "factors")
+    for bad in (np.zeros(32), np.full(32, -1.0)):
+        with pytest.raises(ValueError):
+            oracle.rope_theta(64, 1e4, 64, 1.0, "factors", factors=bad)
+    with pytest.raises(ValueError):
+        oracle.rope_theta(64, 1e4, 64, 2.0, "yarn_dimramp", 32.0, 1.0)
+
+
 # -------------------------------------------------------------- the rotation
 
 def test_rotation_matrix_from_the_page(golden):
