@@ -78,6 +78,10 @@ def _load():
                                       c_int, c_int, c_int, c_int, dp, c_double, c_int, c_int,
                                       dp, dp, dp, dp]
         lib.oracle_decode.restype = c_int
+        lib.oracle_prefill_chunk.argtypes = [u16p, u16p, u16p, u16p, u16p, c_int, c_int,
+                                             c_int, c_int, c_int, c_int, c_int, dp, c_double,
+                                             c_int, c_int, dp, dp, dp]
+        lib.oracle_prefill_chunk.restype = c_int
         lib.oracle_kv_cache_bytes.argtypes = [c_double] * 6
         lib.oracle_kv_cache_bytes.restype = c_double
         _lib = lib
@@ -216,6 +220,32 @@ def decode(q_new, k_new, v_new, k_cache, v_cache, cache_len, theta, softmax_scal
     if rc != 0:
         raise ValueError(f"oracle_decode failed ({rc})")
     return o, lse, kr, qr
+
+
+def prefill_chunk(q, k_new, v_new, k_cache, v_cache, P0, theta, softmax_scale, window=0,
+                  n_sink=0):
+    """A chunk of Tq tokens at positions P0.. against a rotated cache prefix (slots < P0).
+    q bf16 [B,Hq,Tq,d]; k_new, v_new bf16 [B,Hkv,Tq,d]; caches bf16 [B,Hkv,T_max,d].
+    Returns (o [B,Hq,Tq,d], lse [B,Hq,Tq], k_rot_new [B,Hkv,Tq,d]) in float64."""
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k_new), _bits(v_new)
+    kc, vc = _bits(k_cache), _bits(v_cache)
+    B, Hq, Tq, d = qb.shape
+    Hkv = kb.shape[1]
+    T_max = kc.shape[2]
+    o = np.zeros((B, Hq, Tq, d), dtype=np.float64)
+    lse = np.zeros((B, Hq, Tq), dtype=np.float64)
+    kr = np.zeros((B, Hkv, Tq, d), dtype=np.float64)
+    th = np.ascontiguousarray(theta, dtype=np.float64)
+    rc = lib.oracle_prefill_chunk(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16),
+                                  _ptr(vb, ctypes.c_uint16), _ptr(kc, ctypes.c_uint16),
+                                  _ptr(vc, ctypes.c_uint16), int(T_max), int(P0), B, Hq, Hkv,
+                                  Tq, d, _ptr(th, ctypes.c_double), float(softmax_scale),
+                                  int(window), int(n_sink), _ptr(o, ctypes.c_double),
+                                  _ptr(lse, ctypes.c_double), _ptr(kr, ctypes.c_double))
+    if rc != 0:
+        raise ValueError(f"oracle_prefill_chunk failed ({rc})")
+    return o, lse, kr
 
 
 def kv_cache_bytes(n_layers, n_kv_heads, head_dim, seq_len, batch=1, dtype_bytes=2) -> float:

@@ -46,6 +46,8 @@
  *   oracle_attn_rows    pinned (library SDPA special case, closed-form
  *                       means, page's "4 + last 4096" sink count, T=1).
  *   oracle_decode       pinned (equals the prefill row at the same position).
+ *   oracle_prefill_chunk pinned (Tq = 1 is decode; P0 = 0 is the full
+ *                       prefill; torch float64 SDPA on the assembled keys).
  *   oracle_kv_cache_bytes pinned (the pages' ~69 GB / ~17 GB / 40 GiB).
  */
 #include <math.h>
@@ -421,6 +423,105 @@ int oracle_decode(const uint16_t *q_new, const uint16_t *k_new, const uint16_t *
         }
         free(x); free(qr); free(kn); free(acc); free(sc);
     }
+    return bad ? -2 : 0;
+}
+
+/*
+ * Prefill of a chunk against a rotated cache prefix: the Tq new tokens of each
+ * sequence sit at positions P0 .. P0+Tq-1 ([P1] deployment notes: cache
+ * prefix KV pairs; [P4] sec. 6 prefix caching and its exercise on chunked
+ * prefill).  Cache slots 0 .. P0-1 hold keys that were rotated when they were
+ * written, and their values (bf16, used as given, as decode reads them); the
+ * chunk's keys are rotated at their positions.  Query i (position P0 + i) sees
+ * key n iff n <= P0 + i and (window == 0 or P0 + i - n < window or n < n_sink).
+ *   q      bf16 [B][Hq][Tq][d]        k_new, v_new  bf16 [B][Hkv][Tq][d]
+ *   cache  bf16 [B][Hkv][T_max][d]    (P0 + Tq <= T_max)
+ *   o      [B][Hq][Tq][d], lse [B][Hq][Tq] (natural log), k_rot_new [B][Hkv][Tq][d]
+ * Returns 0, -1 for invalid arguments, -2 when out of memory.
+ */
+int oracle_prefill_chunk(const uint16_t *q, const uint16_t *k_new, const uint16_t *v_new,
+                         const uint16_t *k_cache, const uint16_t *v_cache, int T_max, int P0,
+                         int B, int Hq, int Hkv, int Tq, int d,
+                         const double *theta, double softmax_scale, int window, int n_sink,
+                         double *o, double *lse, double *k_rot_new)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || Tq < 1 || d < 2 || (d % 2) || (Hq % Hkv)) return -1;
+    if (P0 < 0 || (long)P0 + Tq > (long)T_max) return -1;
+    const int group = Hq / Hkv;
+    const long n_kv = (long)B * Hkv;
+    /* The chunk's rotated keys, k~_{P0+i} = R_{P0+i} k_i. */
+    double *krot = (double *)malloc(sizeof(double) * (size_t)n_kv * Tq * d);
+    if (!krot) return -2;
+#pragma omp parallel
+    {
+        double *tmp = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for collapse(2) schedule(static)
+        for (long kv = 0; kv < n_kv; ++kv) {
+            for (long i = 0; i < Tq; ++i) {
+                const uint16_t *src = k_new + (kv * Tq + i) * d;
+                for (int j = 0; j < d; ++j) tmp[j] = bf16_bits_to_double(src[j]);
+                rotate_vec(tmp, (double)(P0 + i), theta, d, krot + (kv * Tq + i) * d);
+            }
+        }
+        free(tmp);
+    }
+    if (k_rot_new) memcpy(k_rot_new, krot, sizeof(double) * (size_t)n_kv * Tq * d);
+    const long Tk = (long)P0 + Tq;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *x = (double *)malloc(sizeof(double) * (size_t)d);
+        double *qr = (double *)malloc(sizeof(double) * (size_t)d);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)d);
+        double *sc = (double *)malloc(sizeof(double) * (size_t)Tk);
+        if (!x || !qr || !acc || !sc) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for collapse(3) schedule(dynamic, 4)
+        for (int b = 0; b < B; ++b) {
+            for (int h = 0; h < Hq; ++h) {
+                for (long i = 0; i < Tq; ++i) {
+                    if (bad) continue;
+                    const long m = (long)P0 + i;
+                    const long kv = (long)b * Hkv + h / group;
+                    const long qi = ((long)b * Hq + h) * Tq + i;
+                    for (int j = 0; j < d; ++j) x[j] = bf16_bits_to_double(q[qi * d + j]);
+                    rotate_vec(x, (double)m, theta, d, qr);
+                    const uint16_t *kc = k_cache + kv * (long)T_max * d;
+                    const uint16_t *vc = v_cache + kv * (long)T_max * d;
+                    const double *kn = krot + kv * (long)Tq * d;
+                    const uint16_t *vn = v_new + kv * (long)Tq * d;
+                    double mx = -INFINITY;
+                    for (long n = 0; n <= m; ++n) {
+                        if (!visible(m, n, 1, window, n_sink)) { sc[n] = -INFINITY; continue; }
+                        double dot = 0.0;
+                        if (n < P0)
+                            for (int j = 0; j < d; ++j) dot += qr[j] * bf16_bits_to_double(kc[n * d + j]);
+                        else
+                            for (int j = 0; j < d; ++j) dot += qr[j] * kn[(n - P0) * d + j];
+                        sc[n] = softmax_scale * dot;
+                        if (sc[n] > mx) mx = sc[n];
+                    }
+                    double z = 0.0;
+                    for (int j = 0; j < d; ++j) acc[j] = 0.0;
+                    for (long n = 0; n <= m; ++n) {
+                        if (sc[n] == -INFINITY) continue;
+                        const double p = exp(sc[n] - mx);
+                        z += p;
+                        if (n < P0)
+                            for (int j = 0; j < d; ++j) acc[j] += p * bf16_bits_to_double(vc[n * d + j]);
+                        else
+                            for (int j = 0; j < d; ++j) acc[j] += p * bf16_bits_to_double(vn[(n - P0) * d + j]);
+                    }
+                    for (int j = 0; j < d; ++j) o[qi * d + j] = acc[j] / z;
+                    if (lse) lse[qi] = mx + log(z);
+                }
+            }
+        }
+        free(x); free(qr); free(acc); free(sc);
+    }
+    free(krot);
     return bad ? -2 : 0;
 }
 

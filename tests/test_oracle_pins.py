@@ -435,6 +435,75 @@ def test_decode_brute_force(window, n_sink):
             np.testing.assert_allclose(lse[b, h], scipy.special.logsumexp(sc), atol=1e-12)
 
 
+# ------------------------------------------------- chunked prefill on a cache prefix
+
+def _chunk_inputs(B, Hq, Hkv, Tq, d, T_max):
+    q = bf16_bits(RNG.standard_normal((B, Hq, Tq, d)))
+    kn = bf16_bits(RNG.standard_normal((B, Hkv, Tq, d)))
+    vn = bf16_bits(RNG.standard_normal((B, Hkv, Tq, d)))
+    kc = bf16_bits(RNG.standard_normal((B, Hkv, T_max, d)))
+    vc = bf16_bits(RNG.standard_normal((B, Hkv, T_max, d)))
+    return q, kn, vn, kc, vc
+
+
+@pytest.mark.parametrize("window,n_sink", [(0, 0), (7, 0), (7, 3)])
+def test_chunk_brute_force_against_library_softmax(window, n_sink):
+    B, Hq, Hkv, Tq, d, P0, T_max = 2, 4, 2, 9, 16, 11, 24
+    th, _, ss = oracle.rope_theta(d, 10000.0, 8, 4.0, "yarn")
+    q, kn, vn, kc, vc = _chunk_inputs(B, Hq, Hkv, Tq, d, T_max)
+    o, lse, kr = oracle.prefill_chunk(q, kn, vn, kc, vc, P0, th, ss, window, n_sink)
+    g = Hq // Hkv
+    for b in range(B):
+        for j in range(Hkv):
+            krot = complex_rotate(bits_to_f64(kn[b, j]), np.arange(P0, P0 + Tq, dtype=float), th)
+            np.testing.assert_allclose(kr[b, j], krot, atol=1e-12)
+            keys = torch.from_numpy(np.vstack([bits_to_f64(kc[b, j, :P0]), krot]))
+            vals = torch.from_numpy(np.vstack([bits_to_f64(vc[b, j, :P0]), bits_to_f64(vn[b, j])]))
+            for h in range(j * g, (j + 1) * g):
+                qrot = complex_rotate(bits_to_f64(q[b, h]), np.arange(P0, P0 + Tq, dtype=float), th)
+                m = np.arange(P0, P0 + Tq)[:, None]
+                n = np.arange(P0 + Tq)[None, :]
+                vis = n <= m
+                if window:
+                    vis = vis & (((m - n) < window) | (n < n_sink))
+                ref = torch.nn.functional.scaled_dot_product_attention(
+                    torch.from_numpy(qrot)[None], keys[None], vals[None],
+                    attn_mask=torch.from_numpy(vis)[None], scale=ss)[0].numpy()
+                np.testing.assert_allclose(o[b, h], ref, atol=1e-12)
+                sc = np.where(vis, ss * qrot @ keys.numpy().T, -np.inf)
+                np.testing.assert_allclose(lse[b, h], scipy.special.logsumexp(sc, axis=1), atol=1e-12)
+
+
+def test_chunk_of_one_token_is_decode():
+    B, Hq, Hkv, d, T_max, P0 = 2, 8, 2, 32, 40, 17
+    th, _, ss = oracle.rope_theta(d, 500000.0, 16, 16.0, "yarn")
+    q, kn, vn, kc, vc = _chunk_inputs(B, Hq, Hkv, 1, d, T_max)
+    o, lse, kr = oracle.prefill_chunk(q, kn, vn, kc, vc, P0, th, ss, 9, 2)
+    od, lsed, krd, _ = oracle.decode(q[:, :, 0], kn[:, :, 0], vn[:, :, 0], kc, vc,
+                                     np.full(B, P0, np.int32), th, ss, 9, 2)
+    np.testing.assert_allclose(o[:, :, 0], od, rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(lse[:, :, 0], lsed, rtol=1e-14)
+    np.testing.assert_allclose(kr[:, :, 0], krd, rtol=1e-14, atol=1e-15)
+
+
+@pytest.mark.parametrize("window,n_sink", [(0, 0), (5, 2)])
+def test_chunk_at_position_zero_is_full_prefill(window, n_sink):
+    B, Hq, Hkv, Tq, d = 1, 4, 1, 21, 16
+    th, _, ss = oracle.rope_theta(d, 10000.0, 16, 2.0, "ntk")
+    q, kn, vn, kc, vc = _chunk_inputs(B, Hq, Hkv, Tq, d, Tq)
+    o, lse, _ = oracle.prefill_chunk(q, kn, vn, kc, vc, 0, th, ss, window, n_sink)
+    ro, rl, _ = oracle.attn_rows(q, kn, vn, th, ss, True, window, n_sink)
+    np.testing.assert_allclose(o.reshape(ro.shape), ro, rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(lse.reshape(-1), rl, rtol=1e-14)
+
+
+def test_chunk_rejects_overflowing_cache():
+    th, _, ss = oracle.rope_theta(8, 10000.0, 8, 1.0, "rope")
+    q, kn, vn, kc, vc = _chunk_inputs(1, 1, 1, 4, 8, 10)
+    with pytest.raises(ValueError):
+        oracle.prefill_chunk(q, kn, vn, kc, vc, 7, th, ss)
+
+
 def test_decode_rejects_full_cache():
     d = 8
     th, _, ss = oracle.rope_theta(d, 10000.0, 8, 2.0, "yarn")
