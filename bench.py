@@ -353,6 +353,40 @@ def workload_prefill(w, steps, stream, dist, peak_t):
             "frac_of_peak": attn / peak_t}
 
 
+def chunk_bench(w, steps, stream, dist, peak_t):
+    """Chunked prefill after a cached prefix: the whole yr_attn_prefill_chunk call (prefix
+    and chunk laid out as fp16, chunk keys rotated and appended, attention) as causal
+    TFLOP/s."""
+    from yarn_position_scaling_b200 import api
+    q, kn, vn, kc, vc = synth.chunk_inputs(w, "cuda")
+    tab = api.rope_freq_table(w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta)
+    ws = torch.empty(api.attn_prefill_workspace_bytes(w.B, w.Hkv, w.P0 + w.Tq, w.d),
+                     dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(q)
+
+    def step(_):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(stream)
+        api.attn_prefill_chunk(q, kn, vn, kc, vc, w.P0, tab, out=o, workspace=ws, stream=stream)
+        e[1].record(stream)
+        return [(e[0], e[1])]
+
+    for i in range(2):
+        step(i)
+    api.device_status(stream)
+    dist.barrier()
+    total_ms, (call_ms,) = time_events(step, steps, stream)
+    dist.barrier()
+    api.device_status(stream)
+    call_ms = dist.max(call_ms)
+    flops = metrics.chunk_flops(w.B, w.Hq, w.d, w.P0, w.Tq)
+    tf = flops / (call_ms / steps * 1e-3) / 1e12
+    return {"P0": w.P0, "Tq": w.Tq, "Hq": w.Hq, "Hkv": w.Hkv, "T_max": w.T, "method": w.method,
+            "flops_per_step": flops, "steps": steps, "call_ms": call_ms / steps,
+            "call_tflops": tf, "frac_of_peak": tf / peak_t,
+            "timed_over": "the whole call (prefix/chunk layout + attention launches)"}
+
+
 def e2e_prefill(w, steps, warmup, stream):
     """Through the public API with host buffers: pinned H2D of q, k, v, the call, D2H of o."""
     from yarn_position_scaling_b200 import api
@@ -451,6 +485,8 @@ def main():
         for w in [synth.LLAMA3_128K] + synth.SWEEP:
             others[w.name] = workload_prefill(w, args.other_steps, stream, dist, peak_t)
             torch.cuda.empty_cache()
+        others[synth.CHUNK.name] = chunk_bench(synth.CHUNK, args.other_steps, stream, dist, peak_t)
+        torch.cuda.empty_cache()
 
     # ---------------- end to end through the API with host buffers
     estep, h2d, d2h = e2e_prefill(wp, esteps, 2, stream)

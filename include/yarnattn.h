@@ -47,6 +47,11 @@ extern "C" {
 #define YR_PI 1    /* theta_i / s: positions compressed by the extension factor s */
 #define YR_NTK 2   /* (base * s^(d/(d-2)))^(-2i/d) */
 #define YR_YARN 3  /* per-band ramp between theta_i and theta_i / s, plus temperature */
+/* Table variants ("Arch_03_Long_Context" NTK-aware slide, last sentence: dynamic NTK;
+ * "Long context (engineering 100k+ tokens)" and "long-context-models": LongRoPE). */
+#define YR_NTK_DYNAMIC 4  /* NTK-aware with s = max(1, L_cur / L_train) */
+#define YR_YARN_DIMRAMP 5 /* YaRN with the ramp linear in the pair index (floor/ceil band edges) */
+#define YR_FACTORS 6      /* theta_i / f_i with caller-supplied per-dimension factors */
 
 #define YR_MAX_HEAD_DIM 128
 
@@ -60,6 +65,9 @@ typedef struct yr_rope_params {
     int method;     /* YR_ROPE, YR_PI, YR_NTK or YR_YARN */
     double alpha;   /* YaRN ramp start, in rotations per L_train (pages: 1) */
     double beta;    /* YaRN ramp end (pages: 32); must exceed alpha */
+    int L_cur;      /* YR_NTK_DYNAMIC: current sequence length (>= 1); else unused */
+    const double *factors; /* YR_FACTORS: d/2 host doubles f_i > 0, read during the call */
+    double attn_factor;    /* YR_FACTORS: mscale (attention temperature); <= 0 means 1 */
 } yr_rope_params;
 
 /* Frequency and temperature table, built on the host in double precision and
@@ -69,7 +77,8 @@ typedef struct yr_rope_table {
     int method;
     double inv_freq[YR_MAX_HEAD_DIM / 2]; /* theta'_i, radians per position */
     double turns[YR_MAX_HEAD_DIM / 2];    /* theta'_i / (2 pi): rotations per position */
-    double mscale;                        /* 0.1 ln s + 1 for YaRN, else 1 */
+    double mscale;                        /* 0.1 ln s + 1 for both YaRN forms, the caller's
+                                             factor for YR_FACTORS, else 1 */
     double softmax_scale;                 /* mscale^2 / sqrt(d): the logit multiplier */
     uint64_t digest;                      /* FNV-1a of the parameters (position-config identity) */
 } yr_rope_table;
@@ -82,10 +91,19 @@ typedef struct yr_rope_table {
  *   (2 pi), gamma_i = clamp((r_i - alpha)/(beta - alpha), 0, 1), theta'_i =
  *   gamma_i theta_i + (1 - gamma_i) theta_i / s, and mscale = 0.1 ln s + 1
  *   (YaRN slide and steps table).  softmax_scale = mscale^2 / sqrt(d).
+ *   Dynamic NTK: NTK with s = max(1, L_cur / L_train) ("Arch_03_Long_Context",
+ *   NTK-aware slide).  YaRN dimension ramp: i_edge(r) = d ln(L_train / (2 pi
+ *   r)) / (2 ln base), low = floor(i_edge(beta)), high = ceil(i_edge(alpha)),
+ *   gamma_i = 1 - clamp((i - low)/(high - low), 0, 1) ("LLM context window
+ *   mechanics", the structure of its YaRN code).  Factors: theta'_i = theta_i /
+ *   f_i and mscale = attn_factor (LongRoPE's per-dimension interpolation factors,
+ *   "Long context (engineering 100k+ tokens)" and "long-context-models").
  *   The digest hashes the parameters, so a server can fold the position policy
  *   into its engine identity ("long-context-models", operational failure modes).
  * Errors: YR_EINVAL for NULL pointers, odd/out-of-range head_dim, base <= 1,
- *   scale < 1, unknown method, and for YaRN L_train < 1 or beta <= alpha.
+ *   scale < 1, unknown method, for either YaRN form L_train < 1 or beta <=
+ *   alpha, for dynamic NTK L_train < 1 or L_cur < 1, and for YR_FACTORS a NULL
+ *   factors pointer or a factor that is not a positive finite number.
  */
 int yr_rope_freq_table(const yr_rope_params *p, yr_rope_table *out);
 
@@ -167,6 +185,32 @@ int yr_prefill_attend(const void *q, void *o, float *lse, float *q_rot_dbg,
                       const int64_t *q_strides, const int64_t *o_strides,
                       const yr_rope_table *tab, int causal, int window, int n_sink,
                       const void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * attn_prefill_chunk -- prefill of a chunk of Tq new tokens per sequence after a
+ * cached prefix ("LLM context window mechanics", deployment notes: cache prefix KV
+ * pairs; "Long context (engineering 100k+ tokens)", sec. 6 prefix caching and its
+ * exercise on chunked prefill).  The tokens sit at positions P0 .. P0+Tq-1: the
+ * call rotates q and k_new at those positions, writes the rotated keys (bf16) and
+ * v_new into cache slots P0 .. P0+Tq-1, and returns causal attention of each new
+ * query over keys 0 .. its position, with the window/sink rule of yr_attn_prefill.
+ * Slots 0 .. P0-1 are taken as already rotated.  With P0 = 0 it is a causal
+ * yr_attn_prefill that also fills the cache; with Tq = 1 it is one decode step.
+ * Arguments (device pointers, contiguous):
+ *   q, o bf16 [B, Hq, Tq, d]; k_new, v_new bf16 [B, Hkv, Tq, d]
+ *   k_cache, v_cache bf16 [B, Hkv, T_max, d], 0 <= P0 and P0 + Tq <= T_max
+ *   lse fp32 [B, Hq, Tq] (nullable)
+ *   workspace: >= yr_attn_prefill_workspace_bytes(B, Hkv, P0 + Tq, d) bytes,
+ *     256-byte aligned; it receives fp16 copies of all P0 + Tq keys and values.
+ * Errors: YR_EINVAL for NULL or misaligned pointers, sizes out of range, Hq not a
+ *   multiple of Hkv, a window/sink combination yr_attn_prefill rejects, or a
+ *   small workspace; YR_EUNSUPPORTED for d not 64/128 or a non-sm_100 device.
+ */
+int yr_attn_prefill_chunk(const void *q, const void *k_new, const void *v_new,
+                          void *k_cache, void *v_cache, void *o, float *lse,
+                          int B, int Hq, int Hkv, int Tq, int d, int P0, int T_max,
+                          const yr_rope_table *tab, int window, int n_sink,
+                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * attn_decode_workspace_bytes -- bytes of device workspace yr_attn_decode needs

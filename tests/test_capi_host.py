@@ -45,6 +45,43 @@ def test_table_matches_oracle(lib, method, d, base, L, s):
     assert t.head_dim == d and t.method == api.METHODS[method]
 
 
+@pytest.mark.parametrize("method,kw", [
+    ("ntk_dynamic", {"L_cur": 1}), ("ntk_dynamic", {"L_cur": 4096}), ("ntk_dynamic", {"L_cur": 131072}),
+    ("yarn_dimramp", {}),
+    ("factors", {"factors": np.geomspace(1.0, 16.0, 64)}),
+    ("factors", {"factors": np.linspace(1.0, 4.0, 64), "attn_factor": 1.3}),
+])
+@pytest.mark.parametrize("base,L,s", [(10000.0, 4096, 4.0), (500000.0, 8192, 16.0)])
+def test_table_variants_match_oracle(lib, method, kw, base, L, s):
+    t = api.rope_freq_table(128, base, L, s, method, **kw)
+    th, ms, ss = oracle.rope_theta(128, base, L, s, method, **kw)
+    np.testing.assert_allclose(np.array(t.inv_freq[:64]), th, rtol=4e-15, atol=0)
+    np.testing.assert_allclose(np.array(t.turns[:64]), th / (2 * math.pi), rtol=4e-15)
+    assert t.mscale == pytest.approx(ms, rel=1e-15)
+    assert t.softmax_scale == pytest.approx(ss, rel=1e-15)
+    assert t.method == api.METHODS[method]
+
+
+def test_table_variant_digests(lib):
+    dyn = [api.rope_freq_table(128, 1e4, 4096, 1.0, "ntk_dynamic", L_cur=L).digest
+           for L in (4096, 8192, 8192)]
+    assert dyn[1] == dyn[2] and dyn[0] != dyn[1]
+    f = np.linspace(1.0, 4.0, 64)
+    a = api.rope_freq_table(128, 1e4, 4096, 1.0, "factors", factors=f).digest
+    b = api.rope_freq_table(128, 1e4, 4096, 1.0, "factors", factors=f * 1.0001).digest
+    c = api.rope_freq_table(128, 1e4, 4096, 1.0, "factors", factors=f, attn_factor=1.2).digest
+    assert len({a, b, c}) == 3
+
+
+@pytest.mark.parametrize("method,kw", [
+    ("ntk_dynamic", {"L_cur": 0}), ("factors", {}), ("factors", {"factors": np.zeros(64)}),
+    ("factors", {"factors": np.full(64, np.inf)}), ("yarn_dimramp", {"alpha": 32.0, "beta": 1.0}),
+])
+def test_table_variant_arguments_rejected(lib, method, kw):
+    with pytest.raises(RuntimeError):
+        api.rope_freq_table(128, 1e4, 4096, 2.0, method, **kw)
+
+
 def test_table_digest_identifies_the_position_policy(lib):
     a = api.rope_freq_table(128, 10000.0, 4096, 4.0, "yarn")
     b = api.rope_freq_table(128, 10000.0, 4096, 4.0, "yarn")

@@ -24,18 +24,21 @@ def _lib():
     api.load()
 
 
-def run_decode(w, lens, T_max, window=0, n_sink=0):
+def run_decode(w, lens, T_max, window=0, n_sink=0, table_kw=None):
     B = len(lens)
     qn, kn, vn, kc, vc, _ = synth.decode_inputs(w, "cuda", T_max=T_max, B=B)
     cl = torch.tensor(lens, dtype=torch.int32)
     kc0, vc0 = to_bits(kc), to_bits(vc)
-    tab = api.rope_freq_table(w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta)
+    table_kw = table_kw or {}
+    tab = api.rope_freq_table(w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta,
+                              **table_kw)
     lse = torch.empty(qn.shape[:2], device="cuda")
     qd = torch.empty(qn.shape, device="cuda")
     o = api.attn_decode(qn, kn, vn, kc, vc, cl.cuda(), tab, window, n_sink, lse=lse,
                         q_rot_dbg=qd)
     api.device_status()
-    th, _, ss = oracle.rope_theta(w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta)
+    th, _, ss = oracle.rope_theta(w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta,
+                                  **table_kw)
     ro, rl, rk, rq = oracle.decode(to_bits(qn), to_bits(kn), to_bits(vn), kc0, vc0, cl.numpy(),
                                    th, ss, window, n_sink)
     emax, emean = err_stats(to_f64(o), ro)
@@ -110,3 +113,13 @@ def test_decode_at_L_equals_prefill_row_L(L):
     assert err_stats(to_f64(pre[0, :, L]), ro)[0] <= O_MAX_ABS
     assert err_stats(to_f64(dec[0]), ro)[0] <= O_MAX_ABS
     assert err_stats(to_f64(dec[0]), to_f64(pre[0, :, L]))[0] <= 2 * O_MAX_ABS
+
+
+@pytest.mark.parametrize("method,kw", [
+    ("ntk_dynamic", {"L_cur": 9001}),  # one table per call: the longest sequence's length
+    ("yarn_dimramp", {}),
+    ("factors", {"factors": np.geomspace(1.0, 16.0, 64), "attn_factor": 1.2}),
+])
+def test_decode_table_variants(method, kw):
+    w = dataclasses.replace(synth.DECODE, method=method, B=2)
+    run_decode(w, [4000, 9000], 9001, table_kw=kw)

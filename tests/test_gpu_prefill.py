@@ -26,25 +26,29 @@ def _lib():
     assert torch.cuda.is_available()
 
 
-def _table(w, d=None):
-    return api.rope_freq_table(d or w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta)
+def _table(w, d=None, **kw):
+    return api.rope_freq_table(d or w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta,
+                               **kw)
 
 
-def _oracle_table(w, d=None):
-    return oracle.rope_theta(d or w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta)
+def _oracle_table(w, d=None, **kw):
+    return oracle.rope_theta(d or w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta,
+                             **kw)
 
 
-def run_full(w, T, B=1, causal=True, window=0, n_sink=0, d=None, Hq=None, Hkv=None):
+def run_full(w, T, B=1, causal=True, window=0, n_sink=0, d=None, Hq=None, Hkv=None,
+             table_kw=None):
     w = dataclasses.replace(w, d=d or w.d, Hq=Hq or w.Hq, Hkv=Hkv or w.Hkv)
+    table_kw = table_kw or {}
     q, k, v = synth.prefill_inputs(w, "cuda", T=T, B=B)
-    tab = _table(w)
+    tab = _table(w, **table_kw)
     lse = torch.empty(q.shape[:3], device="cuda")
     qd = torch.empty(q.shape, device="cuda")
     kd = torch.empty(k.shape, device="cuda")
     o = api.attn_prefill(q, k, v, tab, causal, window, n_sink, lse=lse, q_rot_dbg=qd,
                          k_rot_dbg=kd)
     api.device_status()
-    th, _, ss = _oracle_table(w)
+    th, _, ss = _oracle_table(w, **table_kw)
     ro, rl, rq = oracle.attn_rows(to_bits(q), to_bits(k), to_bits(v), th, ss, causal, window,
                                   n_sink, want_qrot=True)
     emax, emean = err_stats(to_f64(o).reshape(ro.shape), ro)
@@ -89,6 +93,21 @@ def test_non_causal(T, d):
 @pytest.mark.parametrize("method", ["rope", "pi", "ntk", "yarn"])
 def test_position_methods(method):
     run_full(synth.sweep(method, False), 600)
+
+
+# Table variants (dynamic NTK, dimension-ramp YaRN, per-dimension factors): the kernels
+# consume the table as given, so one small shape per variant checks that it arrives.
+TABLE_VARIANTS = [
+    ("ntk_dynamic", {"L_cur": 3000}),     # below L_train: plain RoPE
+    ("ntk_dynamic", {"L_cur": 40000}),    # s = 40000 / 4096
+    ("yarn_dimramp", {}),
+    ("factors", {"factors": np.geomspace(1.0, 16.0, 64), "attn_factor": 1.2}),
+]
+
+
+@pytest.mark.parametrize("method,kw", TABLE_VARIANTS)
+def test_table_variants(method, kw):
+    run_full(dataclasses.replace(synth.sweep("yarn", False), method=method), 600, table_kw=kw)
 
 
 def test_strided_inputs_and_outputs_match_contiguous():

@@ -79,3 +79,26 @@ def test_synthetic_inputs_are_seeded_and_shaped():
     assert lens.dtype == torch.int32 and lens.shape == (8,)
     assert int(lens.min()) >= 32768 and int(lens.max()) <= 131072
     assert torch.equal(lens, synth.cache_lengths(synth.DECODE))
+
+
+@pytest.mark.parametrize("window,n_sink", [(0, 0), (64, 4)])
+def test_chunk_flops_reduce_to_prefill_and_decode(window, n_sink):
+    # a chunk at position 0 is a causal prefill; a one-token chunk is a decode step
+    assert metrics.chunk_flops(2, 8, 128, 0, 300, window, n_sink) == \
+        metrics.prefill_flops(2, 8, 300, 128, True, window, n_sink)
+    assert metrics.chunk_flops(1, 8, 128, 5000, 1, window, n_sink) == \
+        metrics.decode_flops([5000], 8, 128, window, n_sink)
+    # splitting a prompt into prefix + chunk splits its FLOPs
+    assert metrics.chunk_flops(1, 4, 64, 0, 700, window, n_sink) == \
+        metrics.chunk_flops(1, 4, 64, 0, 300, window, n_sink) + \
+        metrics.chunk_flops(1, 4, 64, 300, 400, window, n_sink)
+
+
+def test_chunk_inputs_are_seeded_and_shaped():
+    w = synth.CHUNK
+    a = synth.chunk_inputs(w, "cpu", P0=10, Tq=5, T_max=20)
+    b = synth.chunk_inputs(w, "cpu", P0=10, Tq=5, T_max=20)
+    assert [t.shape for t in a] == [(1, 32, 5, 128), (1, 8, 5, 128), (1, 8, 5, 128),
+                                    (1, 8, 20, 128), (1, 8, 20, 128)]
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
+    assert all(t.dtype == torch.bfloat16 for t in a)

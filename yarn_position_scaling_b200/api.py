@@ -16,10 +16,12 @@ from .build import LIB
 
 YR_OK, YR_EINVAL, YR_EUNSUPPORTED, YR_ECUDA, YR_ETIMEOUT = 0, -1, -2, -3, -4
 ROPE, PI, NTK, YARN = 0, 1, 2, 3
-METHODS = {"rope": ROPE, "pi": PI, "ntk": NTK, "yarn": YARN}
+NTK_DYNAMIC, YARN_DIMRAMP, FACTORS = 4, 5, 6
+METHODS = {"rope": ROPE, "pi": PI, "ntk": NTK, "yarn": YARN, "ntk_dynamic": NTK_DYNAMIC,
+           "yarn_dimramp": YARN_DIMRAMP, "factors": FACTORS}
 SYMBOLS = ("yr_rope_freq_table", "yr_attn_prefill_workspace_bytes", "yr_attn_prefill",
-           "yr_prefill_prepare_kv", "yr_prefill_attend", "yr_attn_decode_workspace_bytes",
-           "yr_attn_decode", "yr_attn_decode_noalloc", "yr_device_status", "yr_last_error",
+           "yr_prefill_prepare_kv", "yr_prefill_attend", "yr_attn_prefill_chunk",
+           "yr_attn_decode_workspace_bytes", "yr_attn_decode", "yr_attn_decode_noalloc", "yr_device_status", "yr_last_error",
            "yr_version")
 
 
@@ -32,7 +34,8 @@ class YarnAttnError(RuntimeError):
 class RopeParams(ctypes.Structure):
     _fields_ = [("head_dim", ctypes.c_int), ("base", ctypes.c_double), ("L_train", ctypes.c_int),
                 ("scale", ctypes.c_double), ("method", ctypes.c_int), ("alpha", ctypes.c_double),
-                ("beta", ctypes.c_double)]
+                ("beta", ctypes.c_double), ("L_cur", ctypes.c_int),
+                ("factors", ctypes.POINTER(ctypes.c_double)), ("attn_factor", ctypes.c_double)]
 
 
 class RopeTable(ctypes.Structure):
@@ -70,6 +73,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.yr_prefill_attend.argtypes = ([vp] * 4 + [ci] * 5 + [i64p] * 2 +
                                       [ctypes.POINTER(RopeTable), ci, ci, ci, vp, cs, vp])
     lib.yr_prefill_attend.restype = ci
+    lib.yr_attn_prefill_chunk.argtypes = ([vp] * 7 + [ci] * 7 +
+                                          [ctypes.POINTER(RopeTable), ci, ci, vp, cs, vp])
+    lib.yr_attn_prefill_chunk.restype = ci
     lib.yr_attn_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
     lib.yr_attn_decode_workspace_bytes.restype = cs
     lib.yr_attn_decode.argtypes = ([vp] * 9 + [ci] * 5 +
@@ -111,11 +117,19 @@ def _strides(t: torch.Tensor):
 
 
 def rope_freq_table(head_dim: int, base: float, L_train: int, scale: float, method,
-                    alpha: float = 1.0, beta: float = 32.0) -> RopeTable:
-    """Frequency/temperature table for one position method (host only)."""
+                    alpha: float = 1.0, beta: float = 32.0, L_cur: int = 0, factors=None,
+                    attn_factor: float = 0.0) -> RopeTable:
+    """Frequency/temperature table for one position method (host only).  L_cur is the
+    current sequence length (dynamic NTK); factors the d/2 per-dimension divisors and
+    attn_factor the temperature of the factor method."""
     m = METHODS[method] if isinstance(method, str) else int(method)
+    fac = None
+    if factors is not None:
+        fac = (ctypes.c_double * len(factors))(*[float(x) for x in factors])
     p = RopeParams(int(head_dim), float(base), int(L_train), float(scale), m, float(alpha),
-                   float(beta))
+                   float(beta), int(L_cur),
+                   ctypes.cast(fac, ctypes.POINTER(ctypes.c_double)) if fac is not None else None,
+                   float(attn_factor))
     out = RopeTable()
     _check(load().yr_rope_freq_table(ctypes.byref(p), ctypes.byref(out)))
     return out
@@ -174,6 +188,30 @@ def prefill_attend(q, Hkv: int, table: RopeTable, workspace, causal: bool = True
     rc = load().yr_prefill_attend(
         _ptr(q), _ptr(out), _ptr(lse), _ptr(q_rot_dbg), B, Hq, Hkv, T, d, _strides(q),
         _strides(out), ctypes.byref(table), int(bool(causal)), int(window), int(n_sink),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc)
+    return out
+
+
+def attn_prefill_chunk(q, k_new, v_new, k_cache, v_cache, P0: int, table: RopeTable,
+                       window: int = 0, n_sink: int = 0, out=None, lse=None, workspace=None,
+                       stream=None):
+    """Chunked prefill after a cached prefix: q [B,Hq,Tq,d], k_new/v_new [B,Hkv,Tq,d] at
+    positions P0.., caches [B,Hkv,T_max,d] (contiguous bf16; slots < P0 already rotated).
+    Writes slots P0..P0+Tq-1 of the caches; returns the output [B,Hq,Tq,d] bf16."""
+    B, Hq, Tq, d = q.shape
+    Hkv, T_max = k_cache.shape[1], k_cache.shape[2]
+    for t in (q, k_new, v_new, k_cache, v_cache):
+        if not t.is_contiguous():
+            raise ValueError("attn_prefill_chunk expects contiguous tensors")
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.empty(attn_prefill_workspace_bytes(B, Hkv, P0 + Tq, d),
+                                dtype=torch.uint8, device=q.device)
+    rc = load().yr_attn_prefill_chunk(
+        _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
+        B, Hq, Hkv, Tq, d, int(P0), T_max, ctypes.byref(table), int(window), int(n_sink),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc)
     return out

@@ -62,7 +62,8 @@ struct alignas(64) PrefillParams {
     long long osb, osh, ost;
     float *lse;
     float *q_dbg;
-    int B, Hq, Hkv, T, group;
+    int B, Hq, Hkv, T, group;  // T: query rows
+    int Tk, q_off;             // keys, and the position of query row 0 (a chunk after a prefix)
     int causal, window, n_sink;
     int n_qblocks;
     int kv_major;  // CTA order: 1 = by KV head first (grouped heads), 0 = by query block
@@ -92,9 +93,10 @@ struct TilePlan {
     int sink_end, lo, n;
 };
 
+// q0 and last_row are query positions.
 __device__ __forceinline__ TilePlan plan_tiles(const PrefillParams &p, int q0, int last_row) {
     TilePlan tp;
-    const int hi = p.causal ? last_row / kBlockN : (p.T - 1) / kBlockN;
+    const int hi = p.causal ? last_row / kBlockN : (p.Tk - 1) / kBlockN;
     if (p.window > 0) {
         const int first_key = max(0, q0 - p.window + 1);
         tp.lo = first_key / kBlockN;
@@ -115,8 +117,8 @@ __device__ __forceinline__ int tile_at(const TilePlan &tp, int idx) {
 __device__ __forceinline__ bool tile_visible(const PrefillParams &p, int r_lo, int r_hi, int j) {
     if (r_lo > r_hi) return false;
     const int k_lo = j * kBlockN;
-    const int k_hi = min(k_lo + kBlockN - 1, p.T - 1);
-    if (k_lo > p.T - 1) return false;
+    const int k_hi = min(k_lo + kBlockN - 1, p.Tk - 1);
+    if (k_lo > p.Tk - 1) return false;
     if (!p.causal) return true;
     if (k_lo > r_hi) return false;
     if (p.window > 0) {
@@ -129,7 +131,7 @@ __device__ __forceinline__ bool tile_visible(const PrefillParams &p, int r_lo, i
 __device__ __forceinline__ bool tile_full(const PrefillParams &p, int r_lo, int r_hi, int j) {
     const int k_lo = j * kBlockN;
     const int k_hi = k_lo + kBlockN - 1;
-    if (k_hi > p.T - 1) return false;
+    if (k_hi > p.Tk - 1) return false;
     if (p.causal && k_hi > r_lo) return false;
     if (p.window > 0 && !(r_hi - k_lo < p.window || k_hi < p.n_sink)) return false;
     return true;
@@ -188,14 +190,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         h = rem % p.Hq;
     }
     const int kvh = h / p.group;
-    const int q0 = qb * (kQTiles * kBlockM);
-    const int last_row = min(q0 + kQTiles * kBlockM - 1, p.T - 1);
-    const TilePlan tp = plan_tiles(p, q0, last_row);
+    // Query tiles by position: row r of the query tensor sits at position q_off + r.
+    const int q0 = p.q_off + qb * (kQTiles * kBlockM);
+    const int last_pos = min(q0 + kQTiles * kBlockM - 1, p.q_off + p.T - 1);
+    const TilePlan tp = plan_tiles(p, q0, last_pos);
     int r_lo[kQTiles], r_hi[kQTiles];
 #pragma unroll
     for (int t = 0; t < kQTiles; ++t) {
         r_lo[t] = q0 + t * kBlockM;
-        r_hi[t] = min(r_lo[t] + kBlockM - 1, p.T - 1);
+        r_hi[t] = min(r_lo[t] + kBlockM - 1, last_pos);
     }
 
     if (threadIdx.x == 0) {
@@ -246,7 +249,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 if (r_lo[t] > r_hi[t]) continue;
                 mbar_arrive_expect_tx(&sm->q_full[t], kSub * kSubTileBytes);
                 for (int s = 0; s < kSub; ++s)
-                    tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64, r_lo[t], h, b, pol_q);
+                    tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64, r_lo[t] - p.q_off, h,
+                                b, pol_q);
             }
             const int kv_plane = b * p.Hkv + kvh;
             int issued_k[kKStages] = {}, issued_v[kVStages] = {};
@@ -391,7 +395,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const int my_hi = t == 0 ? r_hi[0] : r_hi[1];
         const int lane_base = (warp & 3) * 32;
         const int r = lane_base + lane;  // row within the tile = TMEM lane
-        const int row = my_lo + r;
+        const int pos = my_lo + r;       // position of this thread's query row
+        const int row = pos - p.q_off;   // its index in the query tensor
         const uint32_t tm_lane = static_cast<uint32_t>(lane_base) << 16;
         const uint32_t tm_s = tmem + tm_lane + t * kBlockN;
         const uint32_t tm_o = tmem + tm_lane + 2 * kBlockN + t * HD;
@@ -420,7 +425,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         for (int pp = 0; pp < 4; ++pp) {
                             const float a = __uint_as_float(w[pp] << 16);
                             const float bb = __uint_as_float(w[pp] & 0xFFFF0000u);
-                            const double turns = static_cast<double>(row) * p.turns[s * 32 + c * 4 + pp];
+                            const double turns = static_cast<double>(pos) * p.turns[s * 32 + c * 4 + pp];
                             const double frac = turns - rint(turns);
                             float sn, cs;
                             __sincosf(static_cast<float>(frac * 6.283185307179586), &sn, &cs);
@@ -471,9 +476,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
                 for (int c = 0; c < kBlockN; ++c) {
                     const int n = k0 + c;
-                    bool v = n < p.T;
-                    if (p.causal) v = v && (n <= row);
-                    if (p.window > 0) v = v && ((row - n) < p.window || n < p.n_sink);
+                    bool v = n < p.Tk;
+                    if (p.causal) v = v && (n <= pos);
+                    if (p.window > 0) v = v && ((pos - n) < p.window || n < p.n_sink);
                     if (!v) s[c] = -INFINITY;
                 }
             }

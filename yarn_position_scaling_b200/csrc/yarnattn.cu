@@ -286,15 +286,17 @@ int prefill_regs_ok() {
     return g_dev[dev].prefill_regs_ok ? 1 : 0;
 }
 
+// T query rows at positions q_off .. q_off+T-1 against Tk keys laid out in the
+// workspace as fp16 [B*Hkv][Tk][d] rotated keys, then the same for values.
 int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, int Hq, int Hkv,
                   int T, int d, const long long qs[3], const long long os[3],
                   const yr_rope_table *tab, int causal, int window, int n_sink,
-                  const void *workspace, cudaStream_t st) {
+                  const void *workspace, cudaStream_t st, int Tk, int q_off) {
     if (!prefill_regs_ok())
         return fail(YR_EUNSUPPORTED, "prefill kernel was built with too few registers per thread "
                                      "for its warpgroup register split");
     const __half *k16 = static_cast<const __half *>(workspace);
-    const __half *v16 = k16 + static_cast<size_t>(B) * Hkv * T * d;
+    const __half *v16 = k16 + static_cast<size_t>(B) * Hkv * Tk * d;
     yr::PrefillParams pp;
     std::memset(&pp, 0, sizeof pp);
     int rc;
@@ -309,10 +311,10 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
         if (rc != YR_OK) return rc;
     }
     {
-        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T),
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(Tk),
                                     static_cast<cuuint64_t>(B) * Hkv};
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                                       static_cast<cuuint64_t>(T) * d * 2};
+                                       static_cast<cuuint64_t>(Tk) * d * 2};
         const cuuint32_t box[3] = {64, 128, 1};
         rc = encode(&pp.tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, k16, dims, strides, box,
                     "rotated k");
@@ -325,6 +327,7 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     pp.lse = lse;
     pp.q_dbg = q_rot_dbg;
     pp.B = B; pp.Hq = Hq; pp.Hkv = Hkv; pp.T = T; pp.group = Hq / Hkv;
+    pp.Tk = Tk; pp.q_off = q_off;
     pp.causal = causal; pp.window = window; pp.n_sink = n_sink;
     pp.n_qblocks = (T + 255) / 256;
     // Grouped query heads read each K/V tile several times: order the CTAs by KV head
@@ -379,7 +382,7 @@ extern "C" int yr_prefill_attend(const void *q, void *o, float *lse, float *q_ro
     rc = prepare_device(nullptr);
     if (rc != YR_OK) return rc;
     return launch_attend(q, o, lse, q_rot_dbg, B, Hq, Hkv, T, d, qs, os, tab, causal, window,
-                         n_sink, workspace, static_cast<cudaStream_t>(stream));
+                         n_sink, workspace, static_cast<cudaStream_t>(stream), T, 0);
 }
 
 extern "C" int yr_attn_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
@@ -406,7 +409,54 @@ extern "C" int yr_attn_prefill(const void *q, const void *k, const void *v, void
                         sm_count, st);
     if (rc != YR_OK) return rc;
     return launch_attend(q, o, lse, q_rot_dbg, B, Hq, Hkv, T, d, qs, os, tab, causal, window,
-                         n_sink, workspace, st);
+                         n_sink, workspace, st, T, 0);
+}
+
+extern "C" int yr_attn_prefill_chunk(const void *q, const void *k_new, const void *v_new,
+                                     void *k_cache, void *v_cache, void *o, float *lse, int B,
+                                     int Hq, int Hkv, int Tq, int d, int P0, int T_max,
+                                     const yr_rope_table *tab, int window, int n_sink,
+                                     void *workspace, size_t workspace_bytes, void *stream) {
+    set_error("");
+    const std::string f("yr_attn_prefill_chunk");
+    if (!q || !k_new || !v_new || !k_cache || !v_cache || !o)
+        return fail(YR_EINVAL, f + ": NULL pointer argument");
+    if (B < 1 || Hq < 1 || Hkv < 1 || Tq < 1) return fail(YR_EINVAL, f + ": B, Hq, Hkv and Tq must be >= 1");
+    if (P0 < 0 || T_max < 1 || static_cast<long long>(P0) + Tq > T_max)
+        return fail(YR_EINVAL, f + ": need 0 <= P0 and P0 + Tq <= T_max");
+    const int Tk = P0 + Tq;
+    long long qs[3], os[3];
+    int rc = check_attend(q, o, lse, nullptr, B, Hq, Hkv, Tq, d, nullptr, nullptr, tab, 1, window,
+                          n_sink, workspace, workspace_bytes, "yr_attn_prefill_chunk", qs, os);
+    if (rc != YR_OK) return rc;
+    rc = check_common("yr_attn_prefill_chunk", B, Hkv, Tk, d, tab, workspace, workspace_bytes);
+    if (rc != YR_OK) return rc;
+    for (const void *ptr : {k_new, v_new, static_cast<const void *>(k_cache),
+                            static_cast<const void *>(v_cache)})
+        if (!aligned(ptr, 16)) return fail(YR_EINVAL, f + ": pointers must be 16-byte aligned");
+    int sm_count = 0;
+    rc = prepare_device(&sm_count);
+    if (rc != YR_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    yr::ChunkPrepParams cp;
+    std::memset(&cp, 0, sizeof cp);
+    cp.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+    cp.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+    cp.kc = static_cast<__nv_bfloat16 *>(k_cache);
+    cp.vc = static_cast<__nv_bfloat16 *>(v_cache);
+    cp.k16 = static_cast<__half *>(workspace);
+    cp.v16 = cp.k16 + static_cast<size_t>(B) * Hkv * Tk * d;
+    cp.Tq = Tq; cp.P0 = P0; cp.Tk = Tk; cp.T_max = T_max; cp.d = d;
+    cp.n_items = static_cast<long long>(B) * Hkv * Tk * (d / 8);
+    for (int i = 0; i < d / 2; ++i) cp.turns[i] = tab->turns[i];
+    long long blocks = (cp.n_items + 255) / 256;
+    const long long cap = static_cast<long long>(sm_count) * 16;
+    if (blocks > cap) blocks = cap;
+    yr::chunk_prep_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(cp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("chunk_prep_kernel launch", e);
+    return launch_attend(q, o, lse, nullptr, B, Hq, Hkv, Tq, d, qs, os, tab, 1, window, n_sink,
+                         workspace, st, Tk, P0);
 }
 
 extern "C" int yr_attn_decode(const void *q_new, const void *k_new, const void *v_new,

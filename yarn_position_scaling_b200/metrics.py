@@ -43,6 +43,14 @@ def decode_visible_keys(L: int, window: int = 0, n_sink: int = 0) -> int:
     return min(L + 1, window) + min(n_sink, max(0, L - window + 1))
 
 
+def chunk_flops(B: int, Hq: int, d: int, P0: int, Tq: int, window: int = 0,
+                n_sink: int = 0) -> float:
+    """Causal FLOPs of a chunk of Tq queries at positions P0.. over the cached prefix and the
+    chunk itself: 4 d per visible (query, key) pair per head."""
+    keys = sum(decode_visible_keys(P0 + i, window, n_sink) for i in range(Tq))
+    return 4.0 * d * Hq * B * keys
+
+
 def decode_kv_bytes(cache_len, Hkv: int, d: int, window: int = 0, n_sink: int = 0,
                     elem_bytes: int = 2) -> float:
     keys = sum(decode_visible_keys(int(L), window, n_sink) for L in cache_len)

@@ -22,7 +22,7 @@ import torch
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str            # "prefill" or "decode"
+    kind: str            # "prefill", "decode" or "chunk"
     seed: int
     B: int
     Hq: int
@@ -40,6 +40,8 @@ class Workload:
     n_sink: int = 0
     len_lo: int = 0      # decode: cache-length range (inclusive)
     len_hi: int = 0
+    P0: int = 0          # chunk: position of the chunk's first token (cached prefix length)
+    Tq: int = 0          # chunk: tokens in the chunk (T is the cache capacity T_max)
 
     def describe(self) -> dict:
         return dataclasses.asdict(self)
@@ -52,6 +54,9 @@ LLAMA3_128K = Workload("llama3_8b_128k_gqa_prefill", "prefill", 2, 1, 32, 8, 128
                        500000.0, 8192, 16.0)
 DECODE = Workload("decode_b8_gqa_128k", "decode", 3, 8, 32, 8, 128, 131073, "yarn", 500000.0,
                   8192, 16.0, len_lo=32768, len_hi=131072)
+# The last 4096 tokens of a 128K Llama-3-8B-shaped prompt, after a cached 124K prefix.
+CHUNK = Workload("chunk_llama3_8b_124k_plus_4k", "chunk", 5, 1, 32, 8, 128, 131072, "yarn",
+                 500000.0, 8192, 16.0, P0=126976, Tq=4096)
 
 
 def sweep(method: str, windowed: bool) -> Workload:
@@ -62,7 +67,7 @@ def sweep(method: str, windowed: bool) -> Workload:
 
 
 SWEEP = [sweep(m, w) for m in ("rope", "pi", "ntk", "yarn") for w in (False, True)]
-ALL = {w.name: w for w in [TINY, LLAMA2_16K, LLAMA3_128K, DECODE] + SWEEP}
+ALL = {w.name: w for w in [TINY, LLAMA2_16K, LLAMA3_128K, DECODE, CHUNK] + SWEEP}
 
 
 def _gen(seed: int, device) -> torch.Generator:
@@ -107,3 +112,19 @@ def decode_inputs(w: Workload, device="cpu", T_max: int | None = None, B: int | 
     k_cache = randn_bf16((B, w.Hkv, T_max, w.d), w.seed, device, 6)
     v_cache = randn_bf16((B, w.Hkv, T_max, w.d), w.seed, device, 7)
     return q_new, k_new, v_new, k_cache, v_cache, cache_lengths(w, B)
+
+
+def chunk_inputs(w: Workload, device="cpu", P0: int | None = None, Tq: int | None = None,
+                 T_max: int | None = None, B: int | None = None):
+    """q [B,Hq,Tq,d]; k_new, v_new [B,Hkv,Tq,d]; caches [B,Hkv,T_max,d] whose slots before P0
+    stand for already rotated keys (N(0,1) like the rest)."""
+    P0 = w.P0 if P0 is None else P0
+    Tq = w.Tq if Tq is None else Tq
+    T_max = w.T if T_max is None else T_max
+    B = w.B if B is None else B
+    q = randn_bf16((B, w.Hq, Tq, w.d), w.seed, device, 10)
+    k_new = randn_bf16((B, w.Hkv, Tq, w.d), w.seed, device, 11)
+    v_new = randn_bf16((B, w.Hkv, Tq, w.d), w.seed, device, 12)
+    k_cache = randn_bf16((B, w.Hkv, T_max, w.d), w.seed, device, 13)
+    v_cache = randn_bf16((B, w.Hkv, T_max, w.d), w.seed, device, 14)
+    return q, k_new, v_new, k_cache, v_cache
