@@ -72,16 +72,18 @@ def _load():
         lib.oracle_rotate_rows_f64.restype = None
         lib.oracle_attn_rows.argtypes = [u16p, u16p, u16p, c_int, c_int, c_int, c_int, c_int,
                                          dp, c_double, c_int, c_int, c_int, i64p, c_long,
-                                         dp, dp, dp]
+                                         dp, dp, dp, dp]
         lib.oracle_attn_rows.restype = c_int
         lib.oracle_decode.argtypes = [u16p, u16p, u16p, u16p, u16p, c_int, i32p,
                                       c_int, c_int, c_int, c_int, dp, c_double, c_int, c_int,
-                                      dp, dp, dp, dp]
+                                      dp, dp, dp, dp, dp]
         lib.oracle_decode.restype = c_int
         lib.oracle_prefill_chunk.argtypes = [u16p, u16p, u16p, u16p, u16p, c_int, c_int,
                                              c_int, c_int, c_int, c_int, c_int, dp, c_double,
-                                             c_int, c_int, dp, dp, dp]
+                                             c_int, c_int, dp, dp, dp, dp]
         lib.oracle_prefill_chunk.restype = c_int
+        lib.oracle_alibi_slopes.argtypes = [c_int, dp]
+        lib.oracle_alibi_slopes.restype = None
         lib.oracle_kv_cache_bytes.argtypes = [c_double] * 6
         lib.oracle_kv_cache_bytes.restype = c_double
         _lib = lib
@@ -158,12 +160,30 @@ def rotate_f64(x, pos, theta) -> np.ndarray:
     return out.reshape(x.shape)
 
 
+def _slopes(slopes, Hq):
+    if slopes is None:
+        return ctypes.POINTER(ctypes.c_double)(), None
+    a = np.ascontiguousarray(slopes, dtype=np.float64)
+    if a.shape != (Hq,):
+        raise ValueError("slopes must hold one value per query head")
+    return _ptr(a, ctypes.c_double), a
+
+
+def alibi_slopes(H: int) -> np.ndarray:
+    """ALiBi slope of each of H heads (geometric series 2^(-8/H), 2^(-16/H), ...)."""
+    out = np.zeros(H, dtype=np.float64)
+    _load().oracle_alibi_slopes(int(H), _ptr(out, ctypes.c_double))
+    return out
+
+
 def attn_rows(q_bits, k_bits, v_bits, theta, softmax_scale, causal=True, window=0, n_sink=0,
-              rows=None, want_qrot=False):
+              rows=None, want_qrot=False, slopes=None):
     """Exact attention for selected rows.
 
     q [B,Hq,T,d], k/v [B,Hkv,T,d] as bf16 bits.  rows: flat indices
-    (b*Hq+h)*T+m (None = all).  Returns (o [n,d], lse [n], q_rot [n,d] or None).
+    (b*Hq+h)*T+m (None = all).  slopes: per query head, subtracted times (m - n) from
+    the scaled logits (ALiBi); None = no bias.  Returns (o [n,d], lse [n], q_rot [n,d]
+    or None).
     """
     lib = _load()
     q, k, v = _bits(q_bits), _bits(k_bits), _bits(v_bits)
@@ -182,20 +202,21 @@ def attn_rows(q_bits, k_bits, v_bits, theta, softmax_scale, causal=True, window=
     o = np.empty((n, d), dtype=np.float64)
     lse = np.empty(n, dtype=np.float64)
     qr = np.empty((n, d), dtype=np.float64) if want_qrot else None
+    sp, _keep = _slopes(slopes, Hq)
     rc = lib.oracle_attn_rows(_ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16),
                               _ptr(v, ctypes.c_uint16), B, Hq, Hkv, T, d,
                               _ptr(th, ctypes.c_double), float(softmax_scale), int(bool(causal)),
                               int(window), int(n_sink), rp, n, _ptr(o, ctypes.c_double),
                               _ptr(lse, ctypes.c_double),
                               _ptr(qr, ctypes.c_double) if qr is not None
-                              else ctypes.POINTER(ctypes.c_double)())
+                              else ctypes.POINTER(ctypes.c_double)(), sp)
     if rc != 0:
         raise ValueError(f"oracle_attn_rows failed ({rc})")
     return o, lse, qr
 
 
 def decode(q_new, k_new, v_new, k_cache, v_cache, cache_len, theta, softmax_scale,
-           window=0, n_sink=0):
+           window=0, n_sink=0, slopes=None):
     """Exact single-token decode.  Returns (o [B,Hq,d], lse [B,Hq], k_rot_new [B,Hkv,d],
     q_rot_new [B,Hq,d])."""
     lib = _load()
@@ -210,20 +231,21 @@ def decode(q_new, k_new, v_new, k_cache, v_cache, cache_len, theta, softmax_scal
     lse = np.empty((B, Hq), dtype=np.float64)
     kr = np.empty((B, Hkv, d), dtype=np.float64)
     qr = np.empty((B, Hq, d), dtype=np.float64)
+    sp, _keep = _slopes(slopes, Hq)
     rc = lib.oracle_decode(_ptr(qn, ctypes.c_uint16), _ptr(kn, ctypes.c_uint16),
                            _ptr(vn, ctypes.c_uint16), _ptr(kc, ctypes.c_uint16),
                            _ptr(vc, ctypes.c_uint16), T_max, _ptr(cl, ctypes.c_int32),
                            B, Hq, Hkv, d, _ptr(th, ctypes.c_double), float(softmax_scale),
                            int(window), int(n_sink), _ptr(o, ctypes.c_double),
                            _ptr(lse, ctypes.c_double), _ptr(kr, ctypes.c_double),
-                           _ptr(qr, ctypes.c_double))
+                           _ptr(qr, ctypes.c_double), sp)
     if rc != 0:
         raise ValueError(f"oracle_decode failed ({rc})")
     return o, lse, kr, qr
 
 
 def prefill_chunk(q, k_new, v_new, k_cache, v_cache, P0, theta, softmax_scale, window=0,
-                  n_sink=0):
+                  n_sink=0, slopes=None):
     """A chunk of Tq tokens at positions P0.. against a rotated cache prefix (slots < P0).
     q bf16 [B,Hq,Tq,d]; k_new, v_new bf16 [B,Hkv,Tq,d]; caches bf16 [B,Hkv,T_max,d].
     Returns (o [B,Hq,Tq,d], lse [B,Hq,Tq], k_rot_new [B,Hkv,Tq,d]) in float64."""
@@ -237,12 +259,13 @@ def prefill_chunk(q, k_new, v_new, k_cache, v_cache, P0, theta, softmax_scale, w
     lse = np.zeros((B, Hq, Tq), dtype=np.float64)
     kr = np.zeros((B, Hkv, Tq, d), dtype=np.float64)
     th = np.ascontiguousarray(theta, dtype=np.float64)
+    sp, _keep = _slopes(slopes, Hq)
     rc = lib.oracle_prefill_chunk(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16),
                                   _ptr(vb, ctypes.c_uint16), _ptr(kc, ctypes.c_uint16),
                                   _ptr(vc, ctypes.c_uint16), int(T_max), int(P0), B, Hq, Hkv,
                                   Tq, d, _ptr(th, ctypes.c_double), float(softmax_scale),
                                   int(window), int(n_sink), _ptr(o, ctypes.c_double),
-                                  _ptr(lse, ctypes.c_double), _ptr(kr, ctypes.c_double))
+                                  _ptr(lse, ctypes.c_double), _ptr(kr, ctypes.c_double), sp)
     if rc != 0:
         raise ValueError(f"oracle_prefill_chunk failed ({rc})")
     return o, lse, kr

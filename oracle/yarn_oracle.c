@@ -48,6 +48,10 @@
  *   oracle_decode       pinned (equals the prefill row at the same position).
  *   oracle_prefill_chunk pinned (Tq = 1 is decode; P0 = 0 is the full
  *                       prefill; torch float64 SDPA on the assembled keys).
+ *   ALiBi (slopes argument of the three attention functions, and
+ *   oracle_alibi_slopes) pinned: the page's geometric series, torch float64
+ *   SDPA with the additive bias, zero slopes give plain attention, and the
+ *   output is invariant to a common shift of all positions.
  *   oracle_kv_cache_bytes pinned (the pages' ~69 GB / ~17 GB / 40 GiB).
  */
 #include <math.h>
@@ -227,6 +231,18 @@ void oracle_rotate_rows_f64(const double *x, long n, int d, const double *pos,
  *   ([P3] sliding-window and StreamingLLM slides; [P4] sec. 5
  *    "always keep the first K tokens and the last W")
  */
+/*
+ * ALiBi slopes for H heads: one slope per head, falling geometrically from
+ * 2^(-8/H) by a factor 2^(-8/H) per head ([P3] ALiBi slide), i.e.
+ * m_h = 2^(-8 (h+1) / H).  ALiBi adds
+ * -m_h * (i - j) to the scaled logit of query position i and key position j
+ * and rotates nothing.
+ */
+void oracle_alibi_slopes(int H, double *m)
+{
+    for (int h = 0; h < H; ++h) m[h] = pow(2.0, -8.0 * (double)(h + 1) / (double)H);
+}
+
 static int visible(long m, long n, int causal, int window, int n_sink)
 {
     if (causal && n > m) return 0;
@@ -250,7 +266,7 @@ int oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      const double *theta, double softmax_scale,
                      int causal, int window, int n_sink,
                      const int64_t *rows, long n_rows,
-                     double *o, double *lse, double *q_rot)
+                     double *o, double *lse, double *q_rot, const double *slopes)
 {
     if (B < 1 || Hq < 1 || Hkv < 1 || T < 1 || d < 2 || (d % 2) || (Hq % Hkv)) return -1;
     const int group = Hq / Hkv;
@@ -326,6 +342,7 @@ int oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                 double dot = 0.0;
                 for (int j = 0; j < d; ++j) dot += qr[j] * kr[n * d + j];
                 sc[n] = softmax_scale * dot;
+                if (slopes) sc[n] -= slopes[h] * (double)(m - n);
                 if (sc[n] > mx) mx = sc[n];
             }
             double z = 0.0;
@@ -362,7 +379,8 @@ int oracle_decode(const uint16_t *q_new, const uint16_t *k_new, const uint16_t *
                   const uint16_t *k_cache, const uint16_t *v_cache, int T_max,
                   const int32_t *cache_len, int B, int Hq, int Hkv, int d,
                   const double *theta, double softmax_scale, int window, int n_sink,
-                  double *o, double *lse, double *k_rot_new, double *q_rot_new)
+                  double *o, double *lse, double *k_rot_new, double *q_rot_new,
+                  const double *slopes)
 {
     if (B < 1 || Hq < 1 || Hkv < 1 || d < 2 || (d % 2) || (Hq % Hkv) || T_max < 1) return -1;
     for (int b = 0; b < B; ++b)
@@ -404,6 +422,7 @@ int oracle_decode(const uint16_t *q_new, const uint16_t *k_new, const uint16_t *
                     else
                         for (int j = 0; j < d; ++j) dot += qr[j] * kn[j];
                     sc[n] = softmax_scale * dot;
+                    if (slopes) sc[n] -= slopes[h] * (double)(L - n);
                     if (sc[n] > mx) mx = sc[n];
                 }
                 double z = 0.0;
@@ -443,7 +462,7 @@ int oracle_prefill_chunk(const uint16_t *q, const uint16_t *k_new, const uint16_
                          const uint16_t *k_cache, const uint16_t *v_cache, int T_max, int P0,
                          int B, int Hq, int Hkv, int Tq, int d,
                          const double *theta, double softmax_scale, int window, int n_sink,
-                         double *o, double *lse, double *k_rot_new)
+                         double *o, double *lse, double *k_rot_new, const double *slopes)
 {
     if (B < 1 || Hq < 1 || Hkv < 1 || Tq < 1 || d < 2 || (d % 2) || (Hq % Hkv)) return -1;
     if (P0 < 0 || (long)P0 + Tq > (long)T_max) return -1;
@@ -501,6 +520,7 @@ int oracle_prefill_chunk(const uint16_t *q, const uint16_t *k_new, const uint16_
                         else
                             for (int j = 0; j < d; ++j) dot += qr[j] * kn[(n - P0) * d + j];
                         sc[n] = softmax_scale * dot;
+                        if (slopes) sc[n] -= slopes[h] * (double)(m - n);
                         if (sc[n] > mx) mx = sc[n];
                     }
                     double z = 0.0;

@@ -405,6 +405,72 @@ def test_sampled_rows_equal_full_rows():
     np.testing.assert_allclose(qr, oracle.rotate(q.reshape(-1, 16)[rows], pos, th), atol=0)
 
 
+# ------------------------------------------------------------------------- ALiBi
+
+@pytest.mark.parametrize("H", [1, 4, 8, 12, 32])
+def test_alibi_slopes_geometric_series(H):
+    # the page's series: 2^(-8/H), 2^(-16/H), ... one term per head
+    m = oracle.alibi_slopes(H)
+    assert m[0] == pytest.approx(2.0 ** (-8.0 / H), rel=1e-15)
+    np.testing.assert_allclose(m[1:] / m[:-1], 2.0 ** (-8.0 / H), rtol=1e-14)
+    assert m[-1] == pytest.approx(2.0 ** -8, rel=1e-15)
+
+
+@pytest.mark.parametrize("window,n_sink", [(0, 0), (6, 2)])
+def test_alibi_against_library_sdpa_with_bias(window, n_sink):
+    B, Hq, Hkv, T, d = 1, 4, 2, 19, 16
+    ss = 1.0 / math.sqrt(d)
+    theta = np.zeros(d // 2)  # ALiBi rotates nothing
+    q = bf16_bits(RNG.standard_normal((B, Hq, T, d)))
+    k = bf16_bits(RNG.standard_normal((B, Hkv, T, d)))
+    v = bf16_bits(RNG.standard_normal((B, Hkv, T, d)))
+    slopes = oracle.alibi_slopes(Hq)
+    o, lse, _ = oracle.attn_rows(q, k, v, theta, ss, True, window, n_sink, slopes=slopes)
+    o = o.reshape(B, Hq, T, d)
+    mpos = np.arange(T)[:, None]
+    npos = np.arange(T)[None, :]
+    vis = npos <= mpos
+    if window:
+        vis = vis & (((mpos - npos) < window) | (npos < n_sink))
+    for h in range(Hq):
+        bias = np.where(vis, -slopes[h] * (mpos - npos), -np.inf)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(bits_to_f64(q[0, h]))[None],
+            torch.from_numpy(bits_to_f64(k[0, h // 2]))[None],
+            torch.from_numpy(bits_to_f64(v[0, h // 2]))[None],
+            attn_mask=torch.from_numpy(bias)[None], scale=ss)[0].numpy()
+        np.testing.assert_allclose(o[0, h], ref, atol=1e-12)
+
+
+def test_alibi_zero_slopes_and_cross_function_identities():
+    B, Hq, Hkv, T, d = 1, 2, 1, 12, 8
+    ss = 1.0 / math.sqrt(d)
+    theta = np.zeros(d // 2)
+    q = bf16_bits(RNG.standard_normal((B, Hq, T, d)))
+    k = bf16_bits(RNG.standard_normal((B, Hkv, T, d)))
+    v = bf16_bits(RNG.standard_normal((B, Hkv, T, d)))
+    plain, _, _ = oracle.attn_rows(q, k, v, theta, ss)
+    zero, _, _ = oracle.attn_rows(q, k, v, theta, ss, slopes=np.zeros(Hq))
+    np.testing.assert_array_equal(plain, zero)
+    # with no rotation the cache holds the raw keys: the last rows of a prefill equal a
+    # chunk over the same keys at the same positions, and its last row equals decode
+    slopes = oracle.alibi_slopes(Hq)
+    full, fl, _ = oracle.attn_rows(q, k, v, theta, ss, slopes=slopes)
+    P0 = 5
+    kc = np.zeros((B, Hkv, T, d), np.uint16)
+    vc = np.zeros((B, Hkv, T, d), np.uint16)
+    kc[:, :, :P0], vc[:, :, :P0] = k[:, :, :P0], v[:, :, :P0]
+    ch, cl, _ = oracle.prefill_chunk(q[:, :, P0:], k[:, :, P0:], v[:, :, P0:], kc, vc, P0, theta,
+                                     ss, slopes=slopes)
+    np.testing.assert_allclose(ch, full.reshape(B, Hq, T, d)[:, :, P0:], rtol=1e-13, atol=1e-15)
+    # and decode of the last token equals the last prefill row
+    od, ld, _, _ = oracle.decode(q[:, :, T - 1], k[:, :, T - 1], v[:, :, T - 1], kc * 0 + k,
+                                 vc * 0 + v, np.array([T - 1], np.int32), theta, ss,
+                                 slopes=slopes)
+    np.testing.assert_allclose(od, full.reshape(B, Hq, T, d)[:, :, T - 1], rtol=1e-13,
+                               atol=1e-15)
+
+
 # ----------------------------------------------------------------- the decode
 
 @pytest.mark.parametrize("window,n_sink", [(0, 0), (6, 0), (6, 2)])
