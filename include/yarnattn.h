@@ -52,6 +52,10 @@ extern "C" {
 #define YR_NTK_DYNAMIC 4  /* NTK-aware with s = max(1, L_cur / L_train) */
 #define YR_YARN_DIMRAMP 5 /* YaRN with the ramp linear in the pair index (floor/ceil band edges) */
 #define YR_FACTORS 6      /* theta_i / f_i with caller-supplied per-dimension factors */
+/* ALiBi ("Arch_03_Long_Context", ALiBi slide; "long-context-models"): no rotation; the
+ * kernels subtract m_h (i - j) from the scaled logit of query position i and key j,
+ * with m_h = 2^(-8 (h+1) / Hq) for query head h. */
+#define YR_ALIBI 7
 
 #define YR_MAX_HEAD_DIM 128
 
@@ -98,6 +102,8 @@ typedef struct yr_rope_table {
  *   mechanics", the structure of its YaRN code).  Factors: theta'_i = theta_i /
  *   f_i and mscale = attn_factor (LongRoPE's per-dimension interpolation factors,
  *   "Long context (engineering 100k+ tokens)" and "long-context-models").
+ *   ALiBi: every theta'_i = 0 (no rotation), mscale = 1; the attention entry
+ *   points add the per-head linear bias when they see this method.
  *   The digest hashes the parameters, so a server can fold the position policy
  *   into its engine identity ("long-context-models", operational failure modes).
  * Errors: YR_EINVAL for NULL pointers, odd/out-of-range head_dim, base <= 1,

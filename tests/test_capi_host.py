@@ -62,6 +62,13 @@ def test_table_variants_match_oracle(lib, method, kw, base, L, s):
     assert t.method == api.METHODS[method]
 
 
+def test_alibi_table_rotates_nothing(lib):
+    t = api.rope_freq_table(128, 1e4, 4096, 1.0, "alibi")
+    assert all(x == 0.0 for x in t.inv_freq[:64]) and all(x == 0.0 for x in t.turns[:64])
+    assert t.mscale == 1.0 and t.softmax_scale == pytest.approx(1 / math.sqrt(128), rel=1e-15)
+    assert t.method == api.ALIBI
+
+
 def test_table_variant_digests(lib):
     dyn = [api.rope_freq_table(128, 1e4, 4096, 1.0, "ntk_dynamic", L_cur=L).digest
            for L in (4096, 8192, 8192)]

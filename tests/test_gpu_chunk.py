@@ -111,3 +111,20 @@ def test_chunk_rejects_bad_arguments():
         api.attn_prefill_chunk(q, kn, vn, kc, vc, 10, tab)  # P0 + Tq > T_max
     with pytest.raises(api.YarnAttnError):
         api.attn_prefill_chunk(q, kn, vn, kc, vc, 0, tab, 0, 4)  # sinks without a window
+
+
+def test_chunk_alibi():
+    w = dataclasses.replace(SMALL, method="alibi")
+    P0, Tq, T_max = 700, 300, 1000
+    q, kn, vn, kc, vc = synth.chunk_inputs(w, "cuda", P0=P0, Tq=Tq, T_max=T_max)
+    kc0, vc0 = to_bits(kc), to_bits(vc)
+    tab = api.rope_freq_table(w.d, w.base, w.L_train, w.scale, "alibi")
+    o = api.attn_prefill_chunk(q, kn, vn, kc, vc, P0, tab)
+    api.device_status()
+    ro, _, _ = oracle.prefill_chunk(to_bits(q), to_bits(kn), to_bits(vn), kc0, vc0, P0,
+                                    np.zeros(w.d // 2), 1.0 / np.sqrt(w.d),
+                                    slopes=oracle.alibi_slopes(w.Hq))
+    emax, emean = err_stats(to_f64(o), ro)
+    assert emax <= O_MAX_ABS and emean <= O_MEAN_ABS, (emax, emean)
+    # no rotation: the appended keys are the new keys as given
+    assert torch.equal(kc[:, :, P0:P0 + Tq], kn)

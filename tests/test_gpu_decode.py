@@ -123,3 +123,22 @@ def test_decode_at_L_equals_prefill_row_L(L):
 def test_decode_table_variants(method, kw):
     w = dataclasses.replace(synth.DECODE, method=method, B=2)
     run_decode(w, [4000, 9000], 9001, table_kw=kw)
+
+
+@pytest.mark.parametrize("Hq,Hkv,window,n_sink", [(32, 8, 0, 0), (8, 2, 3000, 4)])
+def test_decode_alibi(Hq, Hkv, window, n_sink):
+    w = dataclasses.replace(synth.DECODE, Hq=Hq, Hkv=Hkv, B=2, method="alibi")
+    lens = [4000, 9000]
+    qn, kn, vn, kc, vc, _ = synth.decode_inputs(w, "cuda", T_max=9001, B=2)
+    cl = torch.tensor(lens, dtype=torch.int32)
+    kc0, vc0 = to_bits(kc), to_bits(vc)
+    tab = api.rope_freq_table(w.d, w.base, w.L_train, w.scale, "alibi")
+    lse = torch.empty(qn.shape[:2], device="cuda")
+    o = api.attn_decode(qn, kn, vn, kc, vc, cl.cuda(), tab, window, n_sink, lse=lse)
+    api.device_status()
+    ro, rl, _, _ = oracle.decode(to_bits(qn), to_bits(kn), to_bits(vn), kc0, vc0, cl.numpy(),
+                                 np.zeros(w.d // 2), 1.0 / np.sqrt(w.d), window, n_sink,
+                                 slopes=oracle.alibi_slopes(Hq))
+    emax, emean = err_stats(to_f64(o), ro)
+    assert emax <= O_MAX_ABS and emean <= O_MEAN_ABS, (emax, emean)
+    assert err_stats(to_f64(lse), rl)[0] <= LSE_ABS

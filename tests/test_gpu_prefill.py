@@ -110,6 +110,24 @@ def test_table_variants(method, kw):
     run_full(dataclasses.replace(synth.sweep("yarn", False), method=method), 600, table_kw=kw)
 
 
+@pytest.mark.parametrize("Hq,Hkv,T,window,n_sink", [(8, 2, 600, 0, 0), (8, 2, 700, 256, 4),
+                                                    (32, 8, 1000, 0, 0), (4, 4, 300, 0, 0)])
+def test_alibi(Hq, Hkv, T, window, n_sink):
+    # ALiBi: no rotation, the bias -m_h (i - j) on the logits (slopes 2^(-8(h+1)/Hq))
+    w = dataclasses.replace(synth.LLAMA3_128K, Hq=Hq, Hkv=Hkv, method="alibi")
+    q, k, v = synth.prefill_inputs(w, "cuda", T=T)
+    tab = api.rope_freq_table(w.d, w.base, w.L_train, w.scale, "alibi")
+    lse = torch.empty(q.shape[:3], device="cuda")
+    o = api.attn_prefill(q, k, v, tab, True, window, n_sink, lse=lse)
+    api.device_status()
+    ro, rl, _ = oracle.attn_rows(to_bits(q), to_bits(k), to_bits(v), np.zeros(w.d // 2),
+                                 1.0 / np.sqrt(w.d), True, window, n_sink,
+                                 slopes=oracle.alibi_slopes(Hq))
+    emax, emean = err_stats(to_f64(o).reshape(ro.shape), ro)
+    assert emax <= O_MAX_ABS and emean <= O_MEAN_ABS, (emax, emean)
+    assert err_stats(to_f64(lse).reshape(-1), rl)[0] <= LSE_ABS
+
+
 def test_strided_inputs_and_outputs_match_contiguous():
     w = synth.LLAMA3_128K
     T = 333

@@ -16,9 +16,9 @@ from .build import LIB
 
 YR_OK, YR_EINVAL, YR_EUNSUPPORTED, YR_ECUDA, YR_ETIMEOUT = 0, -1, -2, -3, -4
 ROPE, PI, NTK, YARN = 0, 1, 2, 3
-NTK_DYNAMIC, YARN_DIMRAMP, FACTORS = 4, 5, 6
+NTK_DYNAMIC, YARN_DIMRAMP, FACTORS, ALIBI = 4, 5, 6, 7
 METHODS = {"rope": ROPE, "pi": PI, "ntk": NTK, "yarn": YARN, "ntk_dynamic": NTK_DYNAMIC,
-           "yarn_dimramp": YARN_DIMRAMP, "factors": FACTORS}
+           "yarn_dimramp": YARN_DIMRAMP, "factors": FACTORS, "alibi": ALIBI}
 SYMBOLS = ("yr_rope_freq_table", "yr_attn_prefill_workspace_bytes", "yr_attn_prefill",
            "yr_prefill_prepare_kv", "yr_prefill_attend", "yr_attn_prefill_chunk",
            "yr_attn_decode_workspace_bytes", "yr_attn_decode", "yr_attn_decode_noalloc", "yr_device_status", "yr_last_error",

@@ -45,6 +45,7 @@ struct DecodeParams {
     int B, Hq, Hkv, T_max, group, n_chunks;
     int window, n_sink;
     float sl2;
+    int alibi;  // 1: add the ALiBi bias -m_h (L - n) to the logits
     double turns[64];
 };
 
@@ -250,10 +251,20 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 #pragma unroll
             for (int e = 0; e < 4; ++e) o[mt][nt][e] = 0.f;
     float m_run[NT][2], l_run[NT][2];
+    // ALiBi slope (log2 units) of this thread's two head columns per n-tile; 0 without ALiBi.
+    float slope2[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
         m_run[nt][0] = m_run[nt][1] = -INFINITY;
         l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+            const int col = nt * 8 + 2 * (lane & 3) + jj;
+            slope2[nt][jj] = (p.alibi && col < g)
+                                 ? exp2f(-8.0f * static_cast<float>(kvh * g + col + 1) /
+                                         static_cast<float>(p.Hq)) * 1.4426950408889634f
+                                 : 0.0f;
+        }
     }
 
     for (int i = 0; i < n_tiles; ++i) {
@@ -293,14 +304,15 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         const int n_b = n_a + 8;
         const bool vis_a = n_a < n_end && dec_key_visible(n_a, L, p.window, p.n_sink);
         const bool vis_b = n_b < n_end && dec_key_visible(n_b, L, p.window, p.n_sink);
+        const float dist_a = static_cast<float>(L - n_a), dist_b = static_cast<float>(L - n_b);
         uint32_t pb[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             float x[4];
-            x[0] = vis_a ? sc[nt][0] * p.sl2 : -INFINITY;
-            x[1] = vis_a ? sc[nt][1] * p.sl2 : -INFINITY;
-            x[2] = vis_b ? sc[nt][2] * p.sl2 : -INFINITY;
-            x[3] = vis_b ? sc[nt][3] * p.sl2 : -INFINITY;
+            x[0] = vis_a ? fmaf(sc[nt][0], p.sl2, -slope2[nt][0] * dist_a) : -INFINITY;
+            x[1] = vis_a ? fmaf(sc[nt][1], p.sl2, -slope2[nt][1] * dist_a) : -INFINITY;
+            x[2] = vis_b ? fmaf(sc[nt][2], p.sl2, -slope2[nt][0] * dist_b) : -INFINITY;
+            x[3] = vis_b ? fmaf(sc[nt][3], p.sl2, -slope2[nt][1] * dist_b) : -INFINITY;
             float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) {

@@ -67,8 +67,12 @@ struct alignas(64) PrefillParams {
     int causal, window, n_sink;
     int n_qblocks;
     int kv_major;  // CTA order: 1 = by KV head first (grouped heads), 0 = by query block
+    int alibi;     // 1: add the ALiBi bias -m_h (i - j) to the logits
     float sl2;  // softmax_scale * log2(e)
     unsigned long long timeout_ns;
+    // Failure-detection test hook: CTA 0's producer issues no copy for this key tile
+    // index (-1: off), so a wait that nothing will complete runs out of time.
+    int fault_drop_tile;
     double turns[64];
 };
 
@@ -257,6 +261,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             for (int idx = 0; idx < tp.n && ok; ++idx) {
                 const int j = tile_at(tp, idx);
                 const int ks = idx % kKStages, vs = idx % kVStages;
+                if (idx == p.fault_drop_tile && blockIdx.x == 0) continue;
                 ok = mbar_wait(&sm->k_empty[ks], ((idx / kKStages) & 1) ^ 1, abort, p.timeout_ns);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&sm->k_full[ks], kSub * kSubTileBytes);
@@ -447,6 +452,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
         }
 
+        // ALiBi slope of this head, m_h = 2^(-8 (h+1) / Hq), over the softmax scale.
+        const float alibi_coef =
+            p.alibi ? exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(p.Hq)) *
+                          1.4426950408889634f / p.sl2
+                    : 0.0f;
         float m_run = -INFINITY;  // reference max of this row, log2 units (score * sl2)
         float l_run = 0.0f;       // sum of exp2(score * sl2 - m_run) so far
         int it = 0;
@@ -470,6 +480,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[c][e]);
                 }
+            }
+            if (p.alibi) {
+                // ALiBi: logit - m_h (pos - n), folded into the raw score as
+                // s + (m_h / softmax_scale) (n - pos).  Far keys get a large negative
+                // score whose rounding does not matter: their weight is ~0.
+                const float b0 = alibi_coef * static_cast<float>(j * kBlockN - pos);
+#pragma unroll
+                for (int c = 0; c < kBlockN; ++c) s[c] += fmaf(alibi_coef, static_cast<float>(c), b0);
             }
             if (!tile_full(p, my_lo, my_hi, j)) {
                 const int k0 = j * kBlockN;

@@ -19,6 +19,8 @@
 //          code finds band-edge indices from a log ratio with floor and ceil)
 //   Factors  theta_i / f_i with caller-supplied f_i, mscale = attn_factor
 //          (LongRoPE: searched per-dimension interpolation factors)
+//   ALiBi  no rotation (theta' = 0); the kernels add the per-head linear bias
+//          (ALiBi slide)
 //   softmax_scale = mscale^2 / sqrt(d): the temperature on both rotated q and k.
 // The table also carries theta'_i / (2 pi) (rotations per position), which the
 // kernels multiply by the position in fp64 to reduce the angle exactly.
@@ -65,7 +67,7 @@ extern "C" int yr_rope_freq_table(const yr_rope_params *p, yr_rope_table *out) {
         yr_host::set_error("yr_rope_freq_table: scale must be a finite number >= 1");
         return YR_EINVAL;
     }
-    if (p->method < YR_ROPE || p->method > YR_FACTORS) {
+    if (p->method < YR_ROPE || p->method > YR_ALIBI) {
         yr_host::set_error("yr_rope_freq_table: unknown method");
         return YR_EINVAL;
     }
@@ -142,6 +144,9 @@ extern "C" int yr_rope_freq_table(const yr_rope_params *p, yr_rope_table *out) {
             }
             case YR_FACTORS:
                 th = theta / p->factors[i];
+                break;
+            case YR_ALIBI:
+                th = 0.0;  // position enters as a bias on the logits, not a rotation
                 break;
             default:
                 break;

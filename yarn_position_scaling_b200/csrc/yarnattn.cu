@@ -333,8 +333,12 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     // Grouped query heads read each K/V tile several times: order the CTAs by KV head
     // so that re-reads hit L2 (measured: +2.7% at the 128K GQA workload, neutral for MHA).
     pp.kv_major = pp.group > 1 ? 1 : 0;
+    pp.alibi = tab->method == YR_ALIBI ? 1 : 0;
     pp.sl2 = static_cast<float>(tab->softmax_scale * 1.4426950408889634);
     pp.timeout_ns = wait_timeout_ns();
+    // Test hook for the failure path (read on every launch; unset in normal use).
+    const char *drop = std::getenv("YR_FAULT_DROP_KV_TILE");
+    pp.fault_drop_tile = drop ? static_cast<int>(std::strtol(drop, nullptr, 10)) : -1;
     for (int i = 0; i < d / 2; ++i) pp.turns[i] = tab->turns[i];
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * Hq * pp.n_qblocks);
     if (d == 128)
@@ -505,6 +509,7 @@ extern "C" int yr_attn_decode(const void *q_new, const void *k_new, const void *
     dp.B = B; dp.Hq = Hq; dp.Hkv = Hkv; dp.T_max = T_max; dp.group = g; dp.n_chunks = nc;
     dp.window = window; dp.n_sink = n_sink;
     dp.sl2 = static_cast<float>(tab->softmax_scale * 1.4426950408889634);
+    dp.alibi = tab->method == YR_ALIBI ? 1 : 0;
     for (int i = 0; i < d / 2; ++i) dp.turns[i] = tab->turns[i];
     const dim3 grid(nc, Hkv, B);
     if (d == 128) {
