@@ -43,12 +43,13 @@ constexpr int kKStages = YR_PREFILL_KSTAGES;  // 2 or 3 (3 fits 227 KB only at d
 constexpr int kVStages = 2;
 constexpr int kPrefillThreads = 384;  // 3 warpgroups: softmax Q0, softmax Q1, load/MMA
 // Register split (setmaxnreg): the softmax warpgroups grow, the load/MMA one
-// shrinks.  256 * 200 + 128 * 96 = 63488 <= 384 * 168 registers at launch; the
+// shrinks.  256 * 192 + 128 * 112 = 63488 <= 384 * 168 registers at launch; the
 // host checks the launched count before the first launch.
-constexpr int kRegsSoftmax = 200;
-constexpr int kRegsOther = 96;
+constexpr int kRegsSoftmax = 192;
+constexpr int kRegsOther = 112;
 constexpr int kMinLaunchRegs = (256 * kRegsSoftmax + 128 * kRegsOther + 383) / 384;
 constexpr uint32_t kTmemCols = 512;
+constexpr int kMaxPairs = 64;
 constexpr int kSubTileBytes = 128 * 128;  // 128 rows x 64 16-bit columns, 128-byte swizzle
 // Upper bound on a row's probabilities within one tile before its reference max
 // must move: P is stored as fp16 (max 65504), so 2^15 leaves a factor of two.
@@ -86,6 +87,9 @@ struct PrefillSmem {
     uint64_t k_full[kKStages], k_empty[kKStages];
     uint64_t v_full[kVStages], v_empty[kVStages];
     uint64_t s_full[kQTiles], p_full[kQTiles], o_done[kQTiles];
+    // Q rotation: per softmax warp, the angle (turns, reduced) of each pair at the
+    // warp's first row, and the pair's rotations per position in fp32.
+    float q_base[8][kMaxPairs], q_turn[8][kMaxPairs];
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort;
@@ -139,6 +143,13 @@ __device__ __forceinline__ bool tile_full(const PrefillParams &p, int r_lo, int 
     if (p.causal && k_hi > r_lo) return false;
     if (p.window > 0 && !(r_hi - k_lo < p.window || k_hi < p.n_sink)) return false;
     return true;
+}
+
+// Bits 0..min(c, 31) set (0 for c < 0): columns at or below c of a 32-column word.
+__device__ __forceinline__ uint32_t cols_upto(int c) {
+    if (c < 0) return 0u;
+    if (c >= 31) return 0xFFFFFFFFu;
+    return (2u << c) - 1u;
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -416,9 +427,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 float *dbg = (p.q_dbg != nullptr && row < p.T)
                                  ? p.q_dbg + ((static_cast<long long>(b) * p.Hq + h) * p.T + row) * HD
                                  : nullptr;
-#pragma unroll
+                // Angle of pair i at this row, in turns: the warp's first row reduced in
+                // fp64 (turns minus the nearest integer) plus lane * turns_i in fp32
+                // (lane <= 31, so the sum stays below 6 turns: ~3e-7 turns of rounding).
+                float *qb = sm->q_base[warp], *qt = sm->q_turn[warp];
+                const int pos0 = pos - lane;
+                for (int i = lane; i < HD / 2; i += 32) {
+                    const double tr = static_cast<double>(pos0) * p.turns[i];
+                    qb[i] = static_cast<float>(tr - rint(tr));
+                    qt[i] = static_cast<float>(p.turns[i]);
+                }
+                __syncwarp();
+                const float lanef = static_cast<float>(lane);
+#pragma unroll 1
                 for (int s = 0; s < kSub; ++s) {
-#pragma unroll
+#pragma unroll 1
                     for (int c = 0; c < 8; ++c) {
                         uint4 *ptr = reinterpret_cast<uint4 *>(sm->q[t][s] + r * 128 +
                                                                ((c ^ (r & 7)) << 4));
@@ -430,10 +453,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         for (int pp = 0; pp < 4; ++pp) {
                             const float a = __uint_as_float(w[pp] << 16);
                             const float bb = __uint_as_float(w[pp] & 0xFFFF0000u);
-                            const double turns = static_cast<double>(pos) * p.turns[s * 32 + c * 4 + pp];
-                            const double frac = turns - rint(turns);
+                            const int i = s * 32 + c * 4 + pp;
+                            const float turns = fmaf(lanef, qt[i], qb[i]);
+                            // nearest integer by the 1.5 * 2^23 rounding trick (|turns| < 6)
+                            const float near = (turns + 12582912.0f) - 12582912.0f;
                             float sn, cs;
-                            __sincosf(static_cast<float>(frac * 6.283185307179586), &sn, &cs);
+                            __sincosf((turns - near) * 6.2831853071795865f, &sn, &cs);
                             y[2 * pp] = a * cs - bb * sn;
                             y[2 * pp + 1] = a * sn + bb * cs;
                             out[pp] = pack_half2(y[2 * pp], y[2 * pp + 1]);
@@ -490,14 +515,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 for (int c = 0; c < kBlockN; ++c) s[c] += fmaf(alibi_coef, static_cast<float>(c), b0);
             }
             if (!tile_full(p, my_lo, my_hi, j)) {
+                // Visible columns of this row as a bit mask: c <= c_hi (causal, in range)
+                // and (c >= c_lo or c < c_sink) (window, sinks); one select per score.
                 const int k0 = j * kBlockN;
+                int c_hi = p.Tk - 1 - k0;
+                if (p.causal) c_hi = min(c_hi, pos - k0);
+                const int c_lo = p.window > 0 ? pos - p.window + 1 - k0 : -(1 << 30);
+                const int c_sink = p.window > 0 ? p.n_sink - k0 : -(1 << 30);
 #pragma unroll
-                for (int c = 0; c < kBlockN; ++c) {
-                    const int n = k0 + c;
-                    bool v = n < p.Tk;
-                    if (p.causal) v = v && (n <= pos);
-                    if (p.window > 0) v = v && ((pos - n) < p.window || n < p.n_sink);
-                    if (!v) s[c] = -INFINITY;
+                for (int w32 = 0; w32 < kBlockN / 32; ++w32) {
+                    const uint32_t vis = cols_upto(c_hi - 32 * w32) &
+                                         (~cols_upto(c_lo - 1 - 32 * w32) | cols_upto(c_sink - 1 - 32 * w32));
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (!((vis >> e) & 1u)) s[w32 * 32 + e] = -INFINITY;
                 }
             }
             auto exps_to_tmem = [&](float m_ref_in) -> float {
@@ -524,17 +555,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             };
             // A row with a reference max takes its exponentials against it without
             // looking at this tile's max: P only has to fit fp16, and since every
-            // p <= l_tile, l_tile <= kPBound proves it does.  Rows with no reference
-            // yet, and warps where some row fails the test, take the tile max, move
-            // the reference of those rows to it and redo P (rare after a row's first
-            // tile: the running max of a row grows slowly).
-            const bool have_ref = __all_sync(0xffffffffu, m_run != -INFINITY);
-            float l_tile = 0.0f;
-            bool over = true;
-            if (have_ref) {
-                l_tile = exps_to_tmem(m_run);
-                over = !(l_tile <= kPBound);
-            }
+            // p <= l_tile, l_tile <= kPBound proves it does.  A row with no reference
+            // yet tries 0 (log2 units) and keeps it when kBlockN <= l_tile <= kPBound:
+            // then its largest p is at least 1, as with the exact max, so the small p
+            // keep the precision they would have had.
+            // Rows that fail, in warps where any row fails, take the tile max, move
+            // their reference to it and redo P (rare: a row's running max grows
+            // slowly, and typical scores pass the first test).
+            const bool fresh = m_run == -INFINITY;
+            float l_tile = exps_to_tmem(m_run);  // reference 0 for a fresh row
+            bool over = fresh ? !(l_tile >= static_cast<float>(kBlockN) && l_tile <= kPBound)
+                              : !(l_tile <= kPBound);
+            if (fresh && !over) m_run = 0.0f;
             if (__any_sync(0xffffffffu, over)) {
                 // Tile max in four independent chains of three-input max.
                 float m4[4] = {s[0], s[1], s[2], s[3]};
@@ -547,7 +579,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 }
                 const float m_tile = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * sl2;
                 const bool first = m_run == -INFINITY;
-                const bool move = first || (have_ref && over && m_tile > m_run);
+                const bool move = first || (over && m_tile > m_run);
                 const float m_new = move ? fmaxf(m_run, m_tile) : m_run;
                 const bool rescale = !first && m_new > m_run;
                 const float alpha = rescale ? ex2(m_run - m_new) : 1.0f;
