@@ -20,10 +20,16 @@
 // moves when its probabilities against the current reference would not fit
 // fp16 (some p > 2^15), so O is rescaled rarely and most tiles need no row max.
 //
+// A row with no reference yet tries 0 and keeps it when its tile sum lies in
+// [128, 2^15] (then its largest p is at least 1).  Masked tiles apply a per-row
+// bit mask built from the causal, window and sink bounds.
+//
 // Rotation ("Arch_03_Long_Context", RoPE slide): pair (2i, 2i+1) of the query
-// at position m turns by m * theta'_i.  The angle is reduced in fp64 as
-// turns = m * theta'_i / (2 pi) minus its nearest integer, then sin/cos run
-// in fp32 on an argument in [-pi, pi].
+// at position m turns by m * theta'_i.  Each softmax warp reduces the angle of
+// every pair at its first row in fp64 (turns minus the nearest integer); a row
+// adds lane * theta'_i / (2 pi) in fp32 and takes fp32 sin/cos.  Rarely run
+// paths are kept small (rolled loops, compact masks): their instructions are
+// fetched cold.
 //
 // Every wait is bounded (wall clock + a CTA abort flag + the device status
 // word); a CTA that gives up drains its own copies and MMAs, frees TMEM and
@@ -36,10 +42,7 @@ namespace yr {
 constexpr int kBlockM = 128;
 constexpr int kBlockN = 128;
 constexpr int kQTiles = 2;
-#ifndef YR_PREFILL_KSTAGES
-#define YR_PREFILL_KSTAGES 2
-#endif
-constexpr int kKStages = YR_PREFILL_KSTAGES;  // 2 or 3 (3 fits 227 KB only at d=128 with 2 V stages)
+constexpr int kKStages = 2;
 constexpr int kVStages = 2;
 constexpr int kPrefillThreads = 384;  // 3 warpgroups: softmax Q0, softmax Q1, load/MMA
 // Register split (setmaxnreg): the softmax warpgroups grow, the load/MMA one
