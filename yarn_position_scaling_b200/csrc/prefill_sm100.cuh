@@ -361,38 +361,48 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             return true;
         };
 
-        bool prev_vis1 = false;
-        for (int idx = 0; idx < tp.n && ok; ++idx) {
-            const int j = tile_at(tp, idx);
-            const int ks = idx % kKStages, vs = idx % kVStages;
+        // Tensor-pipe order: S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) ...
+        // S_t(i+1) overwrites the P that PV_t(i) reads; tcgen05 MMAs from one thread
+        // run in issue order, so it is issued right behind PV_t(i), with nothing in
+        // between: the next tile's bookkeeping and its K and V waits are done while
+        // this tile's softmax runs, before the wait for P.
+        if (tp.n > 0) {
+            const int j = tile_at(tp, 0);
             for (int t = 0; t < kQTiles; ++t) vis[t] = tile_visible(p, r_lo[t], r_hi[t], j);
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(&sm->k_full[ks], (idx / kKStages) & 1, abort, p.timeout_ns));
-            if (!ok) break;
-            tc_fence_after();
-            if (vis[0]) issue_s(0, ks);
-            if (idx > 0 && prev_vis1) {
-                ok = issue_pv(1, (idx - 1) % kVStages);
-                if (!ok) break;
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm->k_full[0], 0, abort, p.timeout_ns));
+            if (ok) {
+                tc_fence_after();
+                if (vis[0]) issue_s(0, 0);
+                if (vis[1]) issue_s(1, 0);
+                if (leader) mma_commit(&sm->k_empty[0]);
+                __syncwarp();
             }
-            if (vis[1]) issue_s(1, ks);
-            if (leader) {
-                mma_commit(&sm->k_empty[ks]);
-                if (idx > 0) mma_commit(&sm->v_empty[(idx - 1) % kVStages]);
+        }
+        for (int idx = 0; idx < tp.n && ok; ++idx) {
+            const int vs = idx % kVStages;
+            const int ks1 = (idx + 1) % kKStages;
+            const bool has_next = idx + 1 < tp.n;
+            bool vis1[kQTiles] = {false, false};
+            if (has_next) {
+                const int j1 = tile_at(tp, idx + 1);
+                for (int t = 0; t < kQTiles; ++t) vis1[t] = tile_visible(p, r_lo[t], r_hi[t], j1);
             }
-            __syncwarp();
             ok = __all_sync(0xffffffffu,
                             mbar_wait(&sm->v_full[vs], (idx / kVStages) & 1, abort, p.timeout_ns));
+            if (ok && has_next)
+                ok = __all_sync(0xffffffffu, mbar_wait(&sm->k_full[ks1], ((idx + 1) / kKStages) & 1,
+                                                       abort, p.timeout_ns));
             if (!ok) break;
             tc_fence_after();
-            if (vis[0]) ok = issue_pv(0, vs);
-            prev_vis1 = vis[1];
-        }
-        if (ok && tp.n > 0) {
-            const int vs = (tp.n - 1) % kVStages;
-            if (prev_vis1) ok = issue_pv(1, vs);
-            if (ok && leader) mma_commit(&sm->v_empty[vs]);
+            if (vis[0] && !(ok = issue_pv(0, vs))) break;
+            if (vis1[0]) issue_s(0, ks1);
+            if (vis[1] && !(ok = issue_pv(1, vs))) break;
+            if (leader) mma_commit(&sm->v_empty[vs]);
+            if (vis1[1]) issue_s(1, ks1);
+            if (leader && has_next) mma_commit(&sm->k_empty[ks1]);
             __syncwarp();
+            vis[0] = vis1[0];
+            vis[1] = vis1[1];
         }
         if (!ok) {
             if (leader) {
