@@ -161,6 +161,16 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// (a0, a1) += (b0, b1) as one packed f32x2 add: same per-lane rounding as two
+// scalar adds, half the instructions in the row-sum chains.
+__device__ __forceinline__ void add_f32x2(float &a0, float &a1, float b0, float b1) {
+    uint64_t a = (static_cast<uint64_t>(__float_as_uint(a1)) << 32) | __float_as_uint(a0);
+    const uint64_t b = (static_cast<uint64_t>(__float_as_uint(b1)) << 32) | __float_as_uint(b0);
+    asm("add.rn.f32x2 %0, %0, %1;" : "+l"(a) : "l"(b));
+    a0 = __uint_as_float(static_cast<uint32_t>(a));
+    a1 = __uint_as_float(static_cast<uint32_t>(a >> 32));
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -545,9 +555,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 }
             }
             auto exps_to_tmem = [&](float m_ref_in) -> float {
-                // Scalar FMA and adds throughout: measured on sm_100a, a packed f32x2
-                // FMA feeding the scalar ex2 costs about twice as many cycles per
-                // element as two scalar FMAs.
+                // Scalar FMAs feed the scalar ex2 (measured on sm_100a, a packed f32x2
+                // FMA there costs about twice as many cycles per element); the row
+                // sums take packed adds.
                 const float m_ref = (m_ref_in == -INFINITY) ? 0.0f : m_ref_in;
                 const float neg_m = -m_ref;
                 float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -558,8 +568,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     for (int e = 0; e < 16; ++e) {
                         const float p0 = ex2(fmaf(s[c * 32 + 2 * e], sl2, neg_m));
                         const float p1 = ex2(fmaf(s[c * 32 + 2 * e + 1], sl2, neg_m));
-                        acc[(2 * e) & 7] += p0;
-                        acc[(2 * e + 1) & 7] += p1;
+                        add_f32x2(acc[(2 * e) & 7], acc[(2 * e + 1) & 7], p0, p1);
                         pk[e] = pack_half2(p0, p1);
                     }
                     tmem_st16(tm_s + c * 16, pk);
