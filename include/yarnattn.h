@@ -219,6 +219,67 @@ int yr_attn_prefill_chunk(const void *q, const void *k_new, const void *v_new,
                           void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * prefill_prepare_kv_at -- yr_prefill_prepare_kv for a block of keys that starts at
+ * absolute position k_pos0 (key t is rotated at k_pos0 + t): the step a worker of
+ * ring attention / context parallelism ("long-context-models", section "Context
+ * parallelism distributes exact attention"; "Long context (engineering 100k+
+ * tokens)", sec. 3) runs once on its own slice of the sequence before the blocks
+ * circulate.  With k_pos0 = 0 it is yr_prefill_prepare_kv.  Arguments, layout and
+ * errors as there; YR_EINVAL also for k_pos0 < 0 or k_pos0 + T > 2^30.
+ */
+int yr_prefill_prepare_kv_at(const void *k, const void *v, void *k_cache, float *k_rot_dbg,
+                             int B, int Hkv, int T, int d,
+                             const int64_t *k_strides, const int64_t *v_strides,
+                             const int64_t *kc_strides, const yr_rope_table *tab, int k_pos0,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * prefill_attend_block -- attention of T query rows at absolute positions
+ * q_pos0 .. q_pos0+T-1 to the Tk keys and values of one block, at positions
+ * k_pos0 .. k_pos0+Tk-1, that yr_prefill_prepare_kv_at(.., T = Tk, k_pos0, ..) left
+ * in `workspace` (only read).  The queries are rotated at their absolute positions;
+ * the causal, window and sink rules of yr_attn_prefill apply to absolute positions
+ * (sinks are the first n_sink positions of the whole sequence).  o is the block's
+ * own softmax-normalised output, kept in fp32 so that merging adds no rounding, and
+ * lse (natural log, nullable) its log-sum-exp; a row with no visible key in the
+ * block gets o = 0, lse = -inf.  yr_attn_merge folds such partials into the result.
+ * Arguments: q bf16 [B, Hq, T, d] with optional strides as in yr_attn_prefill;
+ *   o fp32 [B, Hq, T, d] contiguous; lse fp32 [B, Hq, T];
+ *   workspace >= yr_attn_prefill_workspace_bytes(B, Hkv, Tk, d).
+ * Errors: as yr_attn_prefill; YR_EINVAL also for Tk < 1, negative positions or
+ *   positions past 2^30, and causal blocks with q_pos0 < k_pos0 (a block wholly
+ *   in the future has no visible key: the caller skips it).
+ */
+int yr_prefill_attend_block(const void *q, float *o, float *lse,
+                            int B, int Hq, int Hkv, int T, int Tk, int d,
+                            const int64_t *q_strides,
+                            const yr_rope_table *tab, int causal, int window, int n_sink,
+                            int q_pos0, int k_pos0,
+                            const void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * attn_merge -- fold one block's partial attention (o_part, lse_part) into a
+ * running result (o_acc, lse_acc) by their log-sum-exp weights, the online-softmax
+ * combination of ring attention (sections above):
+ *   L = log(e^lse_acc + e^lse_part),
+ *   o_acc = e^(lse_acc - L) o_acc + e^(lse_part - L) o_part,  lse_acc = L,
+ * row by row; rows where both lse are -inf are left alone, and a side whose lse is
+ * -inf is not read.  init != 0 takes the
+ * accumulator as empty without reading it (the first block: o_acc, lse_acc are
+ * then just written); otherwise a row with lse_acc = -inf is empty and its o_acc
+ * is not read.  If o_out is non-NULL it also receives the merged rows as bf16
+ * (round to nearest even), e.g. on the last block.
+ * Arguments (device pointers, contiguous, rows = B * Hq * T of the block call):
+ *   o_part fp32 [rows, d]; lse_part fp32 [rows]; o_acc fp32 [rows, d];
+ *   lse_acc fp32 [rows]; o_out bf16 [rows, d] (nullable).
+ *   o pointers 16-byte aligned, lse pointers 4-byte aligned.
+ * Errors: YR_EINVAL for NULL or misaligned pointers or rows < 1; YR_EUNSUPPORTED
+ *   for d not 64/128 or a non-sm_100 device.
+ */
+int yr_attn_merge(const float *o_part, const float *lse_part, float *o_acc, float *lse_acc,
+                  void *o_out, long long rows, int d, int init, void *stream);
+
+/*
  * attn_decode_workspace_bytes -- bytes of device workspace yr_attn_decode needs
  * for its split-KV partial results with a cache of T_max slots.  0 if invalid.
  */

@@ -21,8 +21,9 @@ METHODS = {"rope": ROPE, "pi": PI, "ntk": NTK, "yarn": YARN, "ntk_dynamic": NTK_
            "yarn_dimramp": YARN_DIMRAMP, "factors": FACTORS, "alibi": ALIBI}
 SYMBOLS = ("yr_rope_freq_table", "yr_attn_prefill_workspace_bytes", "yr_attn_prefill",
            "yr_prefill_prepare_kv", "yr_prefill_attend", "yr_attn_prefill_chunk",
-           "yr_attn_decode_workspace_bytes", "yr_attn_decode", "yr_attn_decode_noalloc", "yr_device_status", "yr_last_error",
-           "yr_version")
+           "yr_prefill_prepare_kv_at", "yr_prefill_attend_block", "yr_attn_merge",
+           "yr_attn_decode_workspace_bytes", "yr_attn_decode", "yr_attn_decode_noalloc",
+           "yr_device_status", "yr_last_error", "yr_version")
 
 
 class YarnAttnError(RuntimeError):
@@ -76,6 +77,14 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.yr_attn_prefill_chunk.argtypes = ([vp] * 7 + [ci] * 7 +
                                           [ctypes.POINTER(RopeTable), ci, ci, vp, cs, vp])
     lib.yr_attn_prefill_chunk.restype = ci
+    lib.yr_prefill_prepare_kv_at.argtypes = ([vp] * 4 + [ci] * 4 + [i64p] * 3 +
+                                             [ctypes.POINTER(RopeTable), ci, vp, cs, vp])
+    lib.yr_prefill_prepare_kv_at.restype = ci
+    lib.yr_prefill_attend_block.argtypes = ([vp] * 3 + [ci] * 6 + [i64p] +
+                                            [ctypes.POINTER(RopeTable)] + [ci] * 5 + [vp, cs, vp])
+    lib.yr_prefill_attend_block.restype = ci
+    lib.yr_attn_merge.argtypes = [vp] * 5 + [ctypes.c_longlong, ci, ci, vp]
+    lib.yr_attn_merge.restype = ci
     lib.yr_attn_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
     lib.yr_attn_decode_workspace_bytes.restype = cs
     lib.yr_attn_decode.argtypes = ([vp] * 9 + [ci] * 5 +
@@ -191,6 +200,55 @@ def prefill_attend(q, Hkv: int, table: RopeTable, workspace, causal: bool = True
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(rc)
     return out
+
+
+def prefill_prepare_kv_at(k, v, table: RopeTable, workspace, k_pos0: int, stream=None):
+    """prefill_prepare_kv for a block of keys at absolute positions k_pos0 .. k_pos0+T-1."""
+    B, Hkv, T, d = k.shape
+    rc = load().yr_prefill_prepare_kv_at(
+        _ptr(k), _ptr(v), _ptr(None), _ptr(None), B, Hkv, T, d, _strides(k), _strides(v), None,
+        ctypes.byref(table), int(k_pos0), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc)
+    return workspace
+
+
+def prefill_attend_block(q, Hkv: int, Tk: int, table: RopeTable, workspace, q_pos0: int,
+                         k_pos0: int, causal: bool = True, window: int = 0, n_sink: int = 0,
+                         out=None, lse=None, stream=None):
+    """Attention of q [B,Hq,T,d] at positions q_pos0.. to the Tk keys at positions k_pos0..
+    that prefill_prepare_kv_at left in `workspace`.  Returns (o fp32, lse fp32 [B,Hq,T]):
+    the block's own normalised output and log-sum-exp, to be combined by attn_merge."""
+    B, Hq, T, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, T, d), dtype=torch.float32, device=q.device)
+    if out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError("prefill_attend_block writes a contiguous fp32 output")
+    if lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    rc = load().yr_prefill_attend_block(
+        _ptr(q), _ptr(out), _ptr(lse), B, Hq, Hkv, T, int(Tk), d, _strides(q),
+        ctypes.byref(table), int(bool(causal)), int(window), int(n_sink), int(q_pos0),
+        int(k_pos0), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+def attn_merge(o_part, lse_part, o_acc, lse_acc, out=None, init: bool = False, stream=None):
+    """Fold a block partial (o_part fp32 [..., d], lse_part fp32 [...]) into the running
+    (o_acc fp32, lse_acc fp32) in place by log-sum-exp weights.  init=True takes the
+    accumulator as empty (first block).  If `out` (bf16, shaped like o_part) is given it
+    receives the merged rows."""
+    d = o_part.shape[-1]
+    rows = lse_part.numel()
+    for t in (o_part, lse_part, o_acc, lse_acc) + ((out,) if out is not None else ()):
+        if not t.is_contiguous():
+            raise ValueError("attn_merge expects contiguous tensors")
+    rc = load().yr_attn_merge(_ptr(o_part), _ptr(lse_part), _ptr(o_acc), _ptr(lse_acc),
+                              _ptr(out), rows, d, int(bool(init)), _stream(stream))
+    _check(rc)
+    return o_acc, lse_acc
 
 
 def attn_prefill_chunk(q, k_new, v_new, k_cache, v_cache, P0: int, table: RopeTable,

@@ -2,9 +2,9 @@
 // once and lay keys and values out as fp16 for the tensor cores.
 //
 // Rotation ("Arch_03_Long_Context", RoPE slide): pair (2i, 2i+1) of the key at
-// position n turns by n * theta'_i; the angle is reduced in fp64 (turns minus
-// the nearest integer) before fp32 sin/cos.  Each key is rotated once here
-// instead of once per query tile that reads it.
+// position n (= pos0 + its index) turns by n * theta'_i; the angle is reduced in
+// fp64 (turns minus the nearest integer) before fp32 sin/cos.  Each key is rotated
+// once here instead of once per query tile that reads it.
 //
 // One thread handles 8 consecutive elements (16 bytes) of one key row and the
 // same 8 elements of the value row: coalesced 16-byte loads and stores, a
@@ -24,6 +24,7 @@ struct KvPrepParams {
     long long csb, csh, cst;
     float *k_dbg;  // optional [B*Hkv][T][d] fp32
     int Hkv, T, d;
+    int pos0;           // key t is rotated at position pos0 + t
     long long n_items;  // B*Hkv*T*(d/8)
     double turns[64];
 };
@@ -59,7 +60,7 @@ __global__ void __launch_bounds__(256) kv_prep_kernel(const __grid_constant__ Kv
         unpack_bf16x8(kr, x);
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp) {
-            const double tr = static_cast<double>(t) * turns[c * 4 + pp];
+            const double tr = static_cast<double>(p.pos0 + t) * turns[c * 4 + pp];
             const double frac = tr - rint(tr);
             float sn, cs;
             __sincosf(static_cast<float>(frac * 6.283185307179586), &sn, &cs);

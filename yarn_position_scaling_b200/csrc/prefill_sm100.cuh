@@ -64,10 +64,16 @@ struct alignas(64) PrefillParams {
     CUtensorMap tm_v;  // fp16 [B*Hkv][T][d] values (workspace)
     __nv_bfloat16 *o;
     long long osb, osh, ost;
+    float *o32;  // if set: O as fp32 [B][Hq][T][d] (contiguous) instead of o
     float *lse;
     float *q_dbg;
     int B, Hq, Hkv, T, group;  // T: query rows
-    int Tk, q_off;             // keys, and the position of query row 0 (a chunk after a prefix)
+    // Masks work in key-index coordinates: key n of the workspace sits at position
+    // k_pos0 + n, query row r at k_pos0 + q_off + r.  Only the rotation of Q needs the
+    // absolute position, so it adds k_pos0 back (0 unless the keys are a block of a
+    // longer sequence, as in ring attention).
+    int Tk, q_off;             // keys, and the offset of query row 0 from key 0
+    int k_pos0;
     int causal, window, n_sink;
     int n_qblocks;
     int kv_major;  // CTA order: 1 = by KV head first (grouped heads), 0 = by query block
@@ -456,7 +462,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 float *qb = sm->q_base[warp], *qt = sm->q_turn[warp];
                 const int pos0 = pos - lane;
                 for (int i = lane; i < HD / 2; i += 32) {
-                    const double tr = static_cast<double>(pos0) * p.turns[i];
+                    const double tr = static_cast<double>(pos0 + p.k_pos0) * p.turns[i];
                     qb[i] = static_cast<float>(tr - rint(tr));
                     qt[i] = static_cast<float>(p.turns[i]);
                 }
@@ -638,7 +644,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             raise_status(kStatusTimeoutSoftmax);
             sm->abort = 1;
         }
-        // Epilogue: O / l -> bf16, and the log-sum-exp in natural-log units.
+        // Epilogue: O / l -> bf16 (or fp32), and the log-sum-exp in natural-log units.
+        const long long orow_idx = (static_cast<long long>(b) * p.Hq + h) * p.T + row;
         if (ok && tile_live && it > 0) {
             ok = mbar_wait(&sm->o_done[t], (it - 1) & 1, abort, p.timeout_ns);
             ok = __all_sync(0xffffffffu, ok);
@@ -650,7 +657,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
                 for (int c = 0; c < HD / 32; ++c) {
                     tmem_ld32_sync(tm_o + c * 32, raw);
-                    if (row < p.T) {
+                    if (row < p.T && p.o32 != nullptr) {
+                        float4 *dst = reinterpret_cast<float4 *>(p.o32 + orow_idx * HD + c * 32);
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4)
+                            dst[q4] = make_float4(__uint_as_float(raw[4 * q4]) * inv_l,
+                                                  __uint_as_float(raw[4 * q4 + 1]) * inv_l,
+                                                  __uint_as_float(raw[4 * q4 + 2]) * inv_l,
+                                                  __uint_as_float(raw[4 * q4 + 3]) * inv_l);
+                    } else if (row < p.T) {
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4) {
                             uint32_t pk[4];
@@ -668,14 +683,27 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 }
                 if (p.lse != nullptr && row < p.T) {
                     const float m_ref = (m_run == -INFINITY) ? 0.0f : m_run;
-                    p.lse[(static_cast<long long>(b) * p.Hq + h) * p.T + row] =
-                        (l_run > 0.0f) ? (m_ref + __log2f(l_run)) * 0.69314718055994531f
-                                       : -INFINITY;
+                    p.lse[orow_idx] = (l_run > 0.0f) ? (m_ref + __log2f(l_run)) * 0.69314718055994531f
+                                                     : -INFINITY;
                 }
             } else {
                 raise_status(kStatusTimeoutSoftmax);
                 sm->abort = 1;
             }
+        } else if (ok && tile_live && row < p.T) {
+            // No key of this call is visible to the whole query tile (possible only when
+            // the keys are one block of a longer sequence): o = 0, lse = -inf.
+            if (p.o32 != nullptr) {
+                float4 *dst = reinterpret_cast<float4 *>(p.o32 + orow_idx * HD);
+#pragma unroll 1
+                for (int c = 0; c < HD / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+                __nv_bfloat16 *orow = p.o + b * p.osb + h * p.osh + static_cast<long long>(row) * p.ost;
+#pragma unroll 1
+                for (int c = 0; c < HD / 8; ++c)
+                    *reinterpret_cast<uint4 *>(orow + c * 8) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            if (p.lse != nullptr) p.lse[orow_idx] = -INFINITY;
         }
     }
 

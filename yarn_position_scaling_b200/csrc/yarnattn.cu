@@ -13,6 +13,7 @@
 #include "../../include/yarnattn.h"
 #include "decode_sm100.cuh"
 #include "kvprep_sm100.cuh"
+#include "merge_sm100.cuh"
 #include "prefill_sm100.cuh"
 
 namespace yr_host {
@@ -253,7 +254,7 @@ int check_attend(const void *q, const void *o, const float *lse, const float *q_
 int launch_prepare(const void *k, const void *v, void *k_cache, float *k_rot_dbg, int B, int Hkv,
                    int T, int d, const long long ks[3], const long long vs[3],
                    const long long cs[3], const yr_rope_table *tab, void *workspace,
-                   int sm_count, cudaStream_t st) {
+                   int sm_count, cudaStream_t st, int pos0 = 0) {
     __half *k16 = static_cast<__half *>(workspace);
     __half *v16 = k16 + static_cast<size_t>(B) * Hkv * T * d;
     yr::KvPrepParams kp;
@@ -268,6 +269,7 @@ int launch_prepare(const void *k, const void *v, void *k_cache, float *k_rot_dbg
     kp.csb = cs[0]; kp.csh = cs[1]; kp.cst = cs[2];
     kp.k_dbg = k_rot_dbg;
     kp.Hkv = Hkv; kp.T = T; kp.d = d;
+    kp.pos0 = pos0;
     kp.n_items = static_cast<long long>(B) * Hkv * T * (d / 8);
     for (int i = 0; i < d / 2; ++i) kp.turns[i] = tab->turns[i];
     long long blocks = (kp.n_items + 255) / 256;
@@ -286,12 +288,14 @@ int prefill_regs_ok() {
     return g_dev[dev].prefill_regs_ok ? 1 : 0;
 }
 
-// T query rows at positions q_off .. q_off+T-1 against Tk keys laid out in the
-// workspace as fp16 [B*Hkv][Tk][d] rotated keys, then the same for values.
+// T query rows against Tk keys laid out in the workspace as fp16 [B*Hkv][Tk][d]
+// rotated keys, then the same for values.  Key n sits at position k_pos0 + n and
+// query row r at k_pos0 + q_off + r; masks use the offsets relative to key 0.
 int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, int Hq, int Hkv,
                   int T, int d, const long long qs[3], const long long os[3],
                   const yr_rope_table *tab, int causal, int window, int n_sink,
-                  const void *workspace, cudaStream_t st, int Tk, int q_off) {
+                  const void *workspace, cudaStream_t st, int Tk, int q_off, int k_pos0 = 0,
+                  float *o32 = nullptr) {
     if (!prefill_regs_ok())
         return fail(YR_EUNSUPPORTED, "prefill kernel was built with too few registers per thread "
                                      "for its warpgroup register split");
@@ -324,10 +328,11 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     }
     pp.o = static_cast<__nv_bfloat16 *>(o);
     pp.osb = os[0]; pp.osh = os[1]; pp.ost = os[2];
+    pp.o32 = o32;
     pp.lse = lse;
     pp.q_dbg = q_rot_dbg;
     pp.B = B; pp.Hq = Hq; pp.Hkv = Hkv; pp.T = T; pp.group = Hq / Hkv;
-    pp.Tk = Tk; pp.q_off = q_off;
+    pp.Tk = Tk; pp.q_off = q_off; pp.k_pos0 = k_pos0;
     pp.causal = causal; pp.window = window; pp.n_sink = n_sink;
     pp.n_qblocks = (T + 255) / 256;
     // Grouped query heads read each K/V tile several times: order the CTAs by KV head
@@ -461,6 +466,95 @@ extern "C" int yr_attn_prefill_chunk(const void *q, const void *k_new, const voi
     if (e != cudaSuccess) return cuda_fail("chunk_prep_kernel launch", e);
     return launch_attend(q, o, lse, nullptr, B, Hq, Hkv, Tq, d, qs, os, tab, 1, window, n_sink,
                          workspace, st, Tk, P0);
+}
+
+extern "C" int yr_prefill_prepare_kv_at(const void *k, const void *v, void *k_cache,
+                                        float *k_rot_dbg, int B, int Hkv, int T, int d,
+                                        const int64_t *k_strides, const int64_t *v_strides,
+                                        const int64_t *kc_strides, const yr_rope_table *tab,
+                                        int k_pos0, void *workspace, size_t workspace_bytes,
+                                        void *stream) {
+    set_error("");
+    if (k_pos0 < 0 || static_cast<long long>(k_pos0) + T > (1ll << 30))
+        return fail(YR_EINVAL, "yr_prefill_prepare_kv_at: need 0 <= k_pos0 and k_pos0 + T <= 2^30");
+    long long ks[3], vs[3], cs[3];
+    int rc = check_prepare(k, v, k_cache, k_rot_dbg, B, Hkv, T, d, k_strides, v_strides,
+                           kc_strides, tab, workspace, workspace_bytes, "yr_prefill_prepare_kv_at",
+                           ks, vs, cs);
+    if (rc != YR_OK) return rc;
+    int sm_count = 0;
+    rc = prepare_device(&sm_count);
+    if (rc != YR_OK) return rc;
+    return launch_prepare(k, v, k_cache, k_rot_dbg, B, Hkv, T, d, ks, vs, cs, tab, workspace,
+                          sm_count, static_cast<cudaStream_t>(stream), k_pos0);
+}
+
+extern "C" int yr_prefill_attend_block(const void *q, float *o, float *lse, int B, int Hq,
+                                       int Hkv, int T, int Tk, int d, const int64_t *q_strides,
+                                       const yr_rope_table *tab, int causal, int window,
+                                       int n_sink, int q_pos0, int k_pos0, const void *workspace,
+                                       size_t workspace_bytes, void *stream) {
+    set_error("");
+    const std::string f("yr_prefill_attend_block");
+    if (Tk < 1) return fail(YR_EINVAL, f + ": Tk must be >= 1");
+    if (q_pos0 < 0 || k_pos0 < 0 || static_cast<long long>(q_pos0) + T > (1ll << 30) ||
+        static_cast<long long>(k_pos0) + Tk > (1ll << 30))
+        return fail(YR_EINVAL, f + ": positions must be >= 0 and end below 2^30");
+    if (causal && q_pos0 < k_pos0)
+        return fail(YR_EINVAL, f + ": causal blocks need q_pos0 >= k_pos0 (a block wholly in the "
+                                   "future has no visible key; skip it)");
+    long long qs[3], os[3];
+    // o is fp32 and contiguous here; check_attend's bf16 stride checks see it as such.
+    int rc = check_attend(q, o, lse, nullptr, B, Hq, Hkv, T, d, q_strides, nullptr, tab, causal,
+                          window, n_sink, workspace, workspace_bytes, f.c_str(), qs, os);
+    if (rc != YR_OK) return rc;
+    rc = check_common(f.c_str(), B, Hkv, Tk, d, tab, workspace, workspace_bytes);
+    if (rc != YR_OK) return rc;
+    rc = prepare_device(nullptr);
+    if (rc != YR_OK) return rc;
+    // Sinks are the first n_sink positions of the whole sequence: in this block's key
+    // coordinates they are keys [0, n_sink - k_pos0).
+    const int sinks_here = n_sink > k_pos0 ? n_sink - k_pos0 : 0;
+    return launch_attend(q, nullptr, lse, nullptr, B, Hq, Hkv, T, d, qs, os, tab, causal, window,
+                         sinks_here, workspace, static_cast<cudaStream_t>(stream), Tk,
+                         q_pos0 - k_pos0, k_pos0, o);
+}
+
+extern "C" int yr_attn_merge(const float *o_part, const float *lse_part, float *o_acc,
+                             float *lse_acc, void *o_out, long long rows, int d, int init,
+                             void *stream) {
+    set_error("");
+    const std::string f("yr_attn_merge");
+    if (!o_part || !lse_part || !o_acc || !lse_acc)
+        return fail(YR_EINVAL, f + ": o_part, lse_part, o_acc and lse_acc must be non-NULL");
+    if (rows < 1) return fail(YR_EINVAL, f + ": rows must be >= 1");
+    if (d != 64 && d != 128) return fail(YR_EUNSUPPORTED, f + ": d must be 64 or 128");
+    for (const void *ptr : {static_cast<const void *>(o_part), static_cast<const void *>(o_acc),
+                            static_cast<const void *>(o_out)})
+        if (ptr && !aligned(ptr, 16)) return fail(YR_EINVAL, f + ": o pointers must be 16-byte aligned");
+    if (!aligned(lse_part, 4) || !aligned(lse_acc, 4))
+        return fail(YR_EINVAL, f + ": lse pointers must be 4-byte aligned");
+    int sm_count = 0;
+    int rc = prepare_device(&sm_count);
+    if (rc != YR_OK) return rc;
+    yr::MergeParams mp;
+    mp.o_part = o_part;
+    mp.lse_part = lse_part;
+    mp.o_acc = o_acc;
+    mp.lse_acc = lse_acc;
+    mp.o_out = static_cast<__nv_bfloat16 *>(o_out);
+    mp.rows = rows;
+    mp.d = d;
+    mp.init = init ? 1 : 0;
+    const long long rows_per_block = 8LL * (32 / (d / 8));  // 8 warps
+    long long blocks = (rows + rows_per_block - 1) / rows_per_block;
+    const long long cap = static_cast<long long>(sm_count) * 16;
+    if (blocks > cap) blocks = cap;
+    yr::attn_merge_kernel<<<static_cast<unsigned>(blocks), 256, 0,
+                            static_cast<cudaStream_t>(stream)>>>(mp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("attn_merge_kernel launch", e);
+    return YR_OK;
 }
 
 extern "C" int yr_attn_decode(const void *q_new, const void *k_new, const void *v_new,
