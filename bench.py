@@ -387,6 +387,41 @@ def chunk_bench(w, steps, stream, dist, peak_t):
             "timed_over": "the whole call (prefix/chunk layout + attention launches)"}
 
 
+def ring_bench(w, world, steps, stream, dist, peak_t):
+    """Ring attention over `world` ranks emulated in one process on this GPU: every rank's
+    block kernels (keys prepared at their positions, one attention call per visible
+    block, fp32 partials folded by the log-sum-exp merge) run in turn, without the
+    exchange.  Causal TFLOP/s of the whole sequence over the sum of all ranks' work, i.e.
+    the single-GPU cost of the ring's compute."""
+    from yarn_position_scaling_b200 import api, ring
+    q, k, v = synth.prefill_inputs(w, "cuda")
+    tab = api.rope_freq_table(w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta)
+
+    def step(_):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        with torch.cuda.stream(stream):
+            e[0].record(stream)
+            ring.ring_prefill_emulated(q, k, v, tab, world, w.causal, w.window, w.n_sink)
+            e[1].record(stream)
+        return [(e[0], e[1])]
+
+    for i in range(2):
+        step(i)
+    api.device_status(stream)
+    dist.barrier()
+    total_ms, (call_ms,) = time_events(step, steps, stream)
+    dist.barrier()
+    api.device_status(stream)
+    call_ms = dist.max(call_ms)
+    flops = metrics.prefill_flops(w.B, w.Hq, w.T, w.d, w.causal, w.window, w.n_sink)
+    tf = flops / (call_ms / steps * 1e-3) / 1e12
+    return {"ranks_emulated": world, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "method": w.method,
+            "flops_per_step": flops, "steps": steps, "call_ms": call_ms / steps,
+            "call_tflops": tf, "frac_of_peak": tf / peak_t,
+            "timed_over": "all ranks' block preparation, block attention and merge launches, "
+                          "run in turn on one GPU (no exchange)"}
+
+
 def e2e_prefill(w, steps, warmup, stream):
     """Through the public API with host buffers: pinned H2D of q, k, v, the call, D2H of o."""
     from yarn_position_scaling_b200 import api
@@ -486,6 +521,9 @@ def main():
             others[w.name] = workload_prefill(w, args.other_steps, stream, dist, peak_t)
             torch.cuda.empty_cache()
         others[synth.CHUNK.name] = chunk_bench(synth.CHUNK, args.other_steps, stream, dist, peak_t)
+        torch.cuda.empty_cache()
+        others["ring_" + wp.name + "_4_ranks"] = ring_bench(wp, 4, args.other_steps, stream, dist,
+                                                              peak_t)
         torch.cuda.empty_cache()
 
     # ---------------- end to end through the API with host buffers
