@@ -522,7 +522,8 @@ def main():
             torch.cuda.empty_cache()
         others[synth.CHUNK.name] = chunk_bench(synth.CHUNK, args.other_steps, stream, dist, peak_t)
         torch.cuda.empty_cache()
-        others["ring_" + wp.name + "_4_ranks"] = ring_bench(wp, 4, args.other_steps, stream, dist,
+        wr = synth.LLAMA3_128K
+        others["ring_" + wr.name + "_8_ranks"] = ring_bench(wr, 8, args.other_steps, stream, dist,
                                                               peak_t)
         torch.cuda.empty_cache()
 
