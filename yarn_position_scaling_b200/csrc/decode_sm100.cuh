@@ -2,20 +2,24 @@
 // a log-sum-exp merge ("Long Context" concept page: decode is memory-bound on
 // the cache, which is read every step).
 //
-// Kernel 1 (decode_split_kernel): one block per (sequence b, KV head, chunk of
-// kDecChunk keys).  The block
+// Kernel 1 (decode_split_kernel): a balanced split.  The keys the new tokens see
+// in all (sequence b, KV head) segments are laid end to end and cut into one equal
+// share per block (at least kDecChunk keys), so every block streams the same number
+// of bytes whatever the mix of cache lengths, and all finish together.  For each
+// segment piece it holds, a block
 //   * rotates the new query of each of the g = Hq/Hkv heads of the group at
 //     position L_b (fp64 angle reduction, fp32 sin/cos) and splits it into a
 //     bf16 high part and a bf16 remainder, so the product with the bf16 cache
 //     keeps ~16 significant bits of the rotated query;
-//   * if its chunk holds position L_b, rotates the new key and writes it, with
+//   * if its piece ends at position L_b, rotates the new key and writes it, with
 //     the new value, into cache slot L_b first;
 //   * streams its K and V rows with 16-byte cp.async through a 3-stage ring
-//     (rows past the end arrive as zeros), every byte read once for all g heads;
+//     (rows past the piece arrive as zeros), every byte read once for all g heads;
 //   * computes S^T = K q~^T (keys on the MMA's M side, heads on N) and
 //     O^T += V^T P^T with mma.sync.m16n8k16, online softmax per head;
 //   * leaves (max, sum, unnormalised output) per head in the workspace.
-// Kernel 2 (decode_merge_kernel): per (b, query head), the log-sum-exp merge
+// Kernel 2 (decode_merge_kernel): per (b, query head), the log-sum-exp merge of the
+// segment's pieces
 //   M = max_c m_c;  O = sum_c 2^(m_c-M) o_c / sum_c 2^(m_c-M) l_c
 // ("long-context-models", context parallelism: online softmax combines partial
 // results).
@@ -24,7 +28,7 @@
 
 namespace yr {
 
-constexpr int kDecChunk = 2048;  // keys per split (a multiple of kDecTile)
+constexpr int kDecChunk = 2048;  // least keys per block of the balanced split
 constexpr int kDecTile = 64;     // keys per pipeline stage
 constexpr int kDecStages = 3;
 constexpr int kDecWarps = 4;     // 16 keys of each stage per warp
@@ -42,20 +46,54 @@ struct DecodeParams {
     __nv_bfloat16 *o;            // [B][Hq][d]
     float *lse;                  // [B][Hq] or null
     float *q_dbg;                // [B][Hq][d] or null
-    int B, Hq, Hkv, T_max, group, n_chunks;
+    int B, Hq, Hkv, T_max, group;
+    int n_parts;      // partial-result slots per (b, KV head) in the workspace
+    int grid_blocks;  // blocks of the split launch (the partition depends on it)
     int window, n_sink;
     float sl2;
     int alibi;  // 1: add the ALiBi bias -m_h (L - n) to the logits
     double turns[64];
 };
 
-// Does chunk c (keys [c*C, min(c*C+C, L+1))) hold a key the query at L sees?
-__device__ __forceinline__ bool dec_chunk_visible(int c, int L, int window, int n_sink) {
-    const int lo = c * kDecChunk;
-    if (lo > L) return false;
-    if (window <= 0) return true;
-    const int hi = min(lo + kDecChunk, L + 1) - 1;
-    return (lo < n_sink) || (hi >= L - window + 1);
+__device__ __forceinline__ bool dec_len_ok(const DecodeParams &p, int L) {
+    return L >= 0 && L <= p.T_max - 1;
+}
+// Keys the new token at position L sees, as the ranges [0, len1) and [lo2, lo2 + len2):
+// the sinks and the window, or one range [0, L] without a window or when they meet.
+// A sequence with an out-of-range length has none.
+struct DecRanges {
+    int len1, lo2, len2;
+};
+__device__ __forceinline__ DecRanges dec_ranges(const DecodeParams &p, int L) {
+    DecRanges r{0, 0, 0};
+    if (!dec_len_ok(p, L)) return r;
+    const int s1 = min(p.n_sink, L + 1);
+    const int w0 = max(L - p.window + 1, 0);
+    if (p.window <= 0 || w0 <= s1) {
+        r.len1 = L + 1;
+        r.lo2 = L + 1;
+    } else {
+        r.len1 = s1;
+        r.lo2 = w0;
+        r.len2 = L + 1 - w0;
+    }
+    return r;
+}
+// Balanced split: the visible keys of all (b, KV head) segments, in that order, are
+// units; each block of the split launch takes U consecutive units, U at least
+// kDecChunk so that per-block work dwarfs per-block set-up.  Every block and the
+// merge derive the same partition from cache_len.
+__device__ __forceinline__ long long dec_total_units(const DecodeParams &p) {
+    long long t = 0;
+    for (int b = 0; b < p.B; ++b) {
+        const DecRanges r = dec_ranges(p, p.cache_len[b]);
+        t += static_cast<long long>(p.Hkv) * (r.len1 + r.len2);
+    }
+    return t;
+}
+__device__ __forceinline__ long long dec_units_per_block(long long total, int grid_blocks) {
+    const long long even = (total + grid_blocks - 1) / grid_blocks;
+    return even > kDecChunk ? even : kDecChunk;
 }
 __device__ __forceinline__ bool dec_key_visible(int n, int L, int window, int n_sink) {
     if (n > L) return false;
@@ -72,8 +110,6 @@ struct DecodeSmem {
     __nv_bfloat16 q_lo[16][HD];
     float red_m[kDecWarps][16];
     float red_l[kDecWarps][16];
-    int tiles[kDecChunk / kDecTile];
-    int n_tiles;
 };
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
@@ -136,17 +172,37 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     extern __shared__ uint8_t smem_raw[];
     Smem *sm = reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                         ~static_cast<uintptr_t>(127));
-    const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int L = p.cache_len[b];
-    if (L < 0 || L > p.T_max - 1) {
-        if (chunk == 0 && kvh == 0 && tid == 0) raise_status(kStatusBadCacheLen);
-        return;
-    }
-    if (!dec_chunk_visible(chunk, L, p.window, p.n_sink)) return;
     const int g = p.group;
-    const int n_begin = chunk * kDecChunk;
-    const int n_end = min(n_begin + kDecChunk, L + 1);
+    if (blockIdx.x == 0 && tid == 0)
+        for (int bb = 0; bb < p.B; ++bb)
+            if (!dec_len_ok(p, p.cache_len[bb])) raise_status(kStatusBadCacheLen);
+    // This block's units [u_lo, u_hi) of the balanced split, walked segment by segment.
+    const long long total = dec_total_units(p);
+    const long long U = dec_units_per_block(total, p.grid_blocks);
+    const long long u_lo = static_cast<long long>(blockIdx.x) * U;
+    const long long u_hi = min(u_lo + U, total);
+    long long seg0 = 0;  // first unit of segment (b, kvh)
+    for (int b = 0; b < p.B && seg0 < u_hi; ++b) {
+    const int L = p.cache_len[b];
+    const DecRanges rg = dec_ranges(p, L);
+    const long long V = rg.len1 + rg.len2;
+    for (int kvh = 0; kvh < p.Hkv && seg0 < u_hi; ++kvh, seg0 += V) {
+    if (V == 0 || seg0 + V <= u_lo) continue;
+    // Units [a, e) of this segment map to keys [a, min(e, len1)) and the window
+    // range from lo2; the key at L (the last unit) is this block's if e == V.
+    const int a = static_cast<int>(max(u_lo, seg0) - seg0);
+    const int e = static_cast<int>(min(u_hi, seg0 + V) - seg0);
+    const int part = static_cast<int>(blockIdx.x - seg0 / U);
+    const int r1_lo = a < rg.len1 ? a : 0, r1_hi = a < rg.len1 ? min(e, rg.len1) : 0;
+    const int r2_lo = e > rg.len1 ? rg.lo2 + max(a, rg.len1) - rg.len1 : 0;
+    const int r2_hi = e > rg.len1 ? rg.lo2 + e - rg.len1 : 0;
+    const int n_t1 = (r1_hi - r1_lo + kDecTile - 1) / kDecTile;
+    const int n_tiles = n_t1 + (r2_hi - r2_lo + kDecTile - 1) / kDecTile;
+    const int n_begin = r1_hi > r1_lo ? r1_lo : r2_lo;   // span of this block's keys
+    const int n_end = r2_hi > r2_lo ? r2_hi : r1_hi;
+    const bool has_L = e == V;
+    auto tile_start = [&](int i) { return i < n_t1 ? r1_lo + i * kDecTile : r2_lo + (i - n_t1) * kDecTile; };
     const long long plane = (static_cast<long long>(b) * p.Hkv + kvh) * p.T_max;
     const __nv_bfloat16 *kbase = p.k_cache + plane * HD;
     const __nv_bfloat16 *vbase = p.v_cache + plane * HD;
@@ -166,7 +222,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             __sincosf(static_cast<float>(frac * 6.283185307179586), &sn, &cs);
             y0 = a * cs - c * sn;
             y1 = a * sn + c * cs;
-            if (p.q_dbg != nullptr && chunk == L / kDecChunk) {
+            if (p.q_dbg != nullptr && has_L) {
                 float *d = p.q_dbg + (static_cast<long long>(b) * p.Hq + hq) * HD + 2 * i;
                 d[0] = y0;
                 d[1] = y1;
@@ -178,7 +234,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         *reinterpret_cast<__nv_bfloat162 *>(&sm->q_hi[hh][2 * i]) = hi;
         *reinterpret_cast<__nv_bfloat162 *>(&sm->q_lo[hh][2 * i]) = lo;
     }
-    if (L >= n_begin && L < n_begin + kDecChunk) {
+    if (has_L) {
         for (int i = tid; i < HD / 2; i += kDecThreads) {
             const long long src = (static_cast<long long>(b) * p.Hkv + kvh) * HD + 2 * i;
             const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(p.k_new + src);
@@ -195,18 +251,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                 *reinterpret_cast<const __nv_bfloat162 *>(p.v_new + src);
         }
     }
-    // Tiles of this chunk that hold a visible key.
-    int n_tiles = 0;
-    if (tid == 0) {
-        for (int t0 = n_begin; t0 < n_end; t0 += kDecTile) {
-            const int t1 = min(t0 + kDecTile, n_end) - 1;
-            bool any = p.window <= 0 || t0 < p.n_sink || t1 >= L - p.window + 1;
-            if (any) sm->tiles[n_tiles++] = t0;
-        }
-        sm->n_tiles = n_tiles;
-    }
-    __syncthreads();  // also orders the slot-L writes before the copies below
-    n_tiles = sm->n_tiles;
+    __syncthreads();  // orders the slot-L writes before the copies below
 
     // B fragments of q~^T (k = dims, n = heads), hi and lo parts, for every k-step.
     uint32_t qb_hi[HD / 16][NT][2], qb_lo[HD / 16][NT][2];
@@ -239,7 +284,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 
 #pragma unroll
     for (int s = 0; s < kDecStages - 1; ++s) {
-        if (s < n_tiles) load_tile(sm->tiles[s], s);
+        if (s < n_tiles) load_tile(tile_start(s), s);
         cp_async_commit();
     }
 
@@ -272,11 +317,14 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         __syncthreads();
         {
             const int nxt = i + kDecStages - 1;
-            if (nxt < n_tiles) load_tile(sm->tiles[nxt], nxt % kDecStages);
+            if (nxt < n_tiles) load_tile(tile_start(nxt), nxt % kDecStages);
             cp_async_commit();
         }
         const int stage = i % kDecStages;
-        const int t0 = sm->tiles[i];
+        const int t0 = tile_start(i);
+        // Keys of this tile's own range only: the last tile of the sink range can reach
+        // into the window range, whose tiles count those keys.
+        const int k_lo = i < n_t1 ? r1_lo : r2_lo, k_hi = i < n_t1 ? r1_hi : r2_hi;
         const uint32_t kst = smem_u32(sm->k[stage]), vst = smem_u32(sm->v[stage]);
         const int krow0 = warp * 16;  // this warp's 16 keys within the tile
 
@@ -302,8 +350,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         // Mask and online softmax per head (columns).
         const int n_a = t0 + krow0 + (lane >> 2);
         const int n_b = n_a + 8;
-        const bool vis_a = n_a < n_end && dec_key_visible(n_a, L, p.window, p.n_sink);
-        const bool vis_b = n_b < n_end && dec_key_visible(n_b, L, p.window, p.n_sink);
+        const bool vis_a = n_a >= k_lo && n_a < k_hi && dec_key_visible(n_a, L, p.window, p.n_sink);
+        const bool vis_b = n_b >= k_lo && n_b < k_hi && dec_key_visible(n_b, L, p.window, p.n_sink);
         const float dist_a = static_cast<float>(L - n_a), dist_b = static_cast<float>(L - n_b);
         uint32_t pb[NT][2];
 #pragma unroll
@@ -384,7 +432,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         }
     }
     __syncthreads();
-    const long long part = ((static_cast<long long>(b) * p.Hkv + kvh) * p.n_chunks + chunk) * g;
+    const long long slot = ((static_cast<long long>(b) * p.Hkv + kvh) * p.n_parts + part) * g;
     for (int e = tid; e < g * HD; e += kDecThreads) {
         const int hh = e / HD, dd = e % HD;
         float M = -INFINITY;
@@ -400,12 +448,15 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                 sum += wt * sm->red_l[w][hh];
             }
         }
-        p.ws_o[(part + hh) * HD + dd] = acc;
+        p.ws_o[(slot + hh) * HD + dd] = acc;
         if (dd == 0) {
-            p.ws_ml[(part + hh) * 2 + 0] = M;
-            p.ws_ml[(part + hh) * 2 + 1] = sum;
+            p.ws_ml[(slot + hh) * 2 + 0] = M;
+            p.ws_ml[(slot + hh) * 2 + 1] = sum;
         }
     }
+    __syncthreads();  // shared memory is reused by the next segment
+    }  // kvh
+    }  // b
 }
 
 template <int HD>
@@ -413,21 +464,29 @@ __global__ void __launch_bounds__(HD) decode_merge_kernel(const __grid_constant_
     const int hq = blockIdx.x, b = blockIdx.y, dd = threadIdx.x;
     const int L = p.cache_len[b];
     const long long oi = (static_cast<long long>(b) * p.Hq + hq);
-    if (L < 0 || L > p.T_max - 1) {
+    if (!dec_len_ok(p, L)) {
         p.o[oi * HD + dd] = __float2bfloat16(__int_as_float(0x7fc00000));
         if (p.lse != nullptr && dd == 0) p.lse[oi] = __int_as_float(0x7fc00000);
         return;
     }
     const int g = p.group, kvh = hq / g, hh = hq % g;
-    const long long base = (static_cast<long long>(b) * p.Hkv + kvh) * p.n_chunks;
-    const int nc = L / kDecChunk + 1;
+    // The split kernel's partition: this segment's units and the blocks that hold them.
+    const long long total = dec_total_units(p);
+    const long long U = dec_units_per_block(total, p.grid_blocks);
+    long long seg0 = 0;
+    for (int bb = 0; bb < b; ++bb) {
+        const DecRanges r = dec_ranges(p, p.cache_len[bb]);
+        seg0 += static_cast<long long>(p.Hkv) * (r.len1 + r.len2);
+    }
+    const DecRanges rg = dec_ranges(p, L);
+    const long long V = rg.len1 + rg.len2;
+    seg0 += kvh * V;
+    const int n_parts = static_cast<int>((seg0 + V - 1) / U - seg0 / U) + 1;
+    const long long base = (static_cast<long long>(b) * p.Hkv + kvh) * p.n_parts;
     float M = -INFINITY;
-    for (int c = 0; c < nc; ++c)
-        if (dec_chunk_visible(c, L, p.window, p.n_sink))
-            M = fmaxf(M, p.ws_ml[((base + c) * g + hh) * 2]);
+    for (int c = 0; c < n_parts; ++c) M = fmaxf(M, p.ws_ml[((base + c) * g + hh) * 2]);
     float acc = 0.f, sum = 0.f;
-    for (int c = 0; c < nc; ++c) {
-        if (!dec_chunk_visible(c, L, p.window, p.n_sink)) continue;
+    for (int c = 0; c < n_parts; ++c) {
         const long long pi = (base + c) * g + hh;
         const float mc = p.ws_ml[pi * 2];
         const float w = (mc == -INFINITY) ? 0.f : ex2f(mc - M);

@@ -164,11 +164,30 @@ size_t prefill_ws_bytes(long long B, long long Hkv, long long T, long long d) {
     return static_cast<size_t>(2 * B * Hkv * T * d * 2);
 }
 
-int decode_chunks(int T_max) { return (T_max + yr::kDecChunk - 1) / yr::kDecChunk; }
+// Partial-result slots per (b, KV head): a block of the balanced split holds at least
+// kDecChunk keys, so a segment of at most T_max keys touches at most this many blocks.
+int decode_parts(int T_max) { return (T_max + yr::kDecChunk - 1) / yr::kDecChunk + 1; }
 
 size_t decode_ws_bytes(long long B, long long Hq, long long Hkv, long long d, int T_max) {
     const long long g = Hq / Hkv;
-    return static_cast<size_t>(B * Hkv * decode_chunks(T_max) * g * (d + 2) * 4);
+    return static_cast<size_t>(B * Hkv * decode_parts(T_max) * g * (d + 2) * 4);
+}
+
+// Blocks of the split launch: one full wave (resident blocks per SM x SMs), so that the
+// equal shares of the balanced split all run at once.
+template <int HD, int NT>
+int decode_grid(int sm_count) {
+    static int per_sm = 0;  // same value on every device of this build's target
+    if (per_sm == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, yr::decode_split_kernel<HD, NT>,
+                                                          yr::kDecThreads,
+                                                          yr::decode_smem_bytes<HD>()) != cudaSuccess ||
+            n < 1)
+            n = 1;
+        per_sm = n;
+    }
+    return per_sm * sm_count;
 }
 
 }  // namespace yr_host
@@ -582,11 +601,12 @@ extern "C" int yr_attn_decode(const void *q_new, const void *k_new, const void *
         if (!aligned(ptr, 16)) return fail(YR_EINVAL, "yr_attn_decode: tensor pointers must be 16-byte aligned");
     if (!aligned(cache_len, 4) || (lse && !aligned(lse, 4)) || (q_rot_dbg && !aligned(q_rot_dbg, 4)))
         return fail(YR_EINVAL, "yr_attn_decode: cache_len/lse/q_rot_dbg must be 4-byte aligned");
-    int rc = prepare_device(nullptr);
+    int sm_count = 0;
+    int rc = prepare_device(&sm_count);
     if (rc != YR_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int g = Hq / Hkv;
-    const int nc = decode_chunks(T_max);
+    const int nc = decode_parts(T_max);
     yr::DecodeParams dp;
     std::memset(&dp, 0, sizeof dp);
     dp.q_new = static_cast<const __nv_bfloat16 *>(q_new);
@@ -600,22 +620,27 @@ extern "C" int yr_attn_decode(const void *q_new, const void *k_new, const void *
     dp.o = static_cast<__nv_bfloat16 *>(o);
     dp.lse = lse;
     dp.q_dbg = q_rot_dbg;
-    dp.B = B; dp.Hq = Hq; dp.Hkv = Hkv; dp.T_max = T_max; dp.group = g; dp.n_chunks = nc;
+    dp.B = B; dp.Hq = Hq; dp.Hkv = Hkv; dp.T_max = T_max; dp.group = g; dp.n_parts = nc;
     dp.window = window; dp.n_sink = n_sink;
     dp.sl2 = static_cast<float>(tab->softmax_scale * 1.4426950408889634);
     dp.alibi = tab->method == YR_ALIBI ? 1 : 0;
     for (int i = 0; i < d / 2; ++i) dp.turns[i] = tab->turns[i];
-    const dim3 grid(nc, Hkv, B);
     if (d == 128) {
-        if (g <= 8)
-            yr::decode_split_kernel<128, 1><<<grid, yr::kDecThreads, yr::decode_smem_bytes<128>(), st>>>(dp);
-        else
-            yr::decode_split_kernel<128, 2><<<grid, yr::kDecThreads, yr::decode_smem_bytes<128>(), st>>>(dp);
+        if (g <= 8) {
+            dp.grid_blocks = decode_grid<128, 1>(sm_count);
+            yr::decode_split_kernel<128, 1><<<dp.grid_blocks, yr::kDecThreads, yr::decode_smem_bytes<128>(), st>>>(dp);
+        } else {
+            dp.grid_blocks = decode_grid<128, 2>(sm_count);
+            yr::decode_split_kernel<128, 2><<<dp.grid_blocks, yr::kDecThreads, yr::decode_smem_bytes<128>(), st>>>(dp);
+        }
     } else {
-        if (g <= 8)
-            yr::decode_split_kernel<64, 1><<<grid, yr::kDecThreads, yr::decode_smem_bytes<64>(), st>>>(dp);
-        else
-            yr::decode_split_kernel<64, 2><<<grid, yr::kDecThreads, yr::decode_smem_bytes<64>(), st>>>(dp);
+        if (g <= 8) {
+            dp.grid_blocks = decode_grid<64, 1>(sm_count);
+            yr::decode_split_kernel<64, 1><<<dp.grid_blocks, yr::kDecThreads, yr::decode_smem_bytes<64>(), st>>>(dp);
+        } else {
+            dp.grid_blocks = decode_grid<64, 2>(sm_count);
+            yr::decode_split_kernel<64, 2><<<dp.grid_blocks, yr::kDecThreads, yr::decode_smem_bytes<64>(), st>>>(dp);
+        }
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("decode_split_kernel launch", e);
