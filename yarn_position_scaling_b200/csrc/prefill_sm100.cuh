@@ -113,17 +113,20 @@ struct TilePlan {
 // q0 and last_row are query positions.
 __device__ __forceinline__ TilePlan plan_tiles(const PrefillParams &p, int q0, int last_row) {
     TilePlan tp;
-    const int hi = p.causal ? last_row / kBlockN : (p.Tk - 1) / kBlockN;
+    // The last key any row may see: its own position (causal) or the last key, whichever
+    // comes first (the keys can end before the rows when they are one block of a longer
+    // sequence).
+    const int hi = (p.causal ? min(last_row, p.Tk - 1) : p.Tk - 1) / kBlockN;
     if (p.window > 0) {
         const int first_key = max(0, q0 - p.window + 1);
         tp.lo = first_key / kBlockN;
         const int sink_tiles = (p.n_sink + kBlockN - 1) / kBlockN;
-        tp.sink_end = min(sink_tiles, tp.lo);
+        tp.sink_end = min(min(sink_tiles, tp.lo), hi + 1);
     } else {
         tp.lo = 0;
         tp.sink_end = 0;
     }
-    tp.n = tp.sink_end + (hi - tp.lo + 1);
+    tp.n = tp.sink_end + max(0, hi - tp.lo + 1);
     return tp;
 }
 __device__ __forceinline__ int tile_at(const TilePlan &tp, int idx) {
