@@ -11,8 +11,14 @@
 //               query row (= one TMEM lane), so row max and row sum need no
 //               shuffles; P is written back over S in TMEM as fp16
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+d), O1 [256+d,256+2d).
-// The MMA issue order S0(j) | PV1(j-1) S1(j) | PV0(j) lets one softmax group
-// work while the tensor cores serve the other group ("ping-pong").
+// The MMA issue order S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ... lets one
+// softmax group work while the tensor cores serve the other ("ping-pong"); each
+// S_t(j+1) follows its PV_t(j) directly, since it overwrites the P that PV reads.
+//
+// The keys may be one block of a longer sequence (ring attention): key n sits at
+// position k_pos0 + n; masks work relative to key 0, only Q's rotation uses the
+// absolute position, and a query tile that sees none of the keys writes o = 0 and
+// lse = -inf.  The output is bf16, or fp32 for such block partials.
 //
 // Online softmax ("Long Context" concept page, key math: scores never reach
 // HBM; "long-context-models", context parallelism: running row maxima,
