@@ -170,6 +170,8 @@ def test_decode_rejects_bad_arguments_on_host(lib, kw, code):
 
 def test_workspace_sizes(lib):
     assert api.attn_prefill_workspace_bytes(1, 8, 131072, 128) == 2 * 8 * 131072 * 128 * 2
-    nc = (131073 + 2047) // 2048
-    assert api.attn_decode_workspace_bytes(8, 32, 8, 128, 131073) == 8 * 8 * nc * 4 * 130 * 4
+    # one partial slot per block of the balanced split that can hold part of a segment:
+    # blocks hold at least 2048 keys, so a segment of T_max keys touches ceil(T_max/2048)+1
+    parts = (131073 + 2047) // 2048 + 1
+    assert api.attn_decode_workspace_bytes(8, 32, 8, 128, 131073) == 8 * 8 * parts * 4 * 130 * 4
     assert api.attn_decode_workspace_bytes(8, 30, 8, 128, 100) == 0
