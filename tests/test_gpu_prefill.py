@@ -218,3 +218,19 @@ def test_llama3_128k_sampled_rows():
 @pytest.mark.parametrize("w", synth.SWEEP, ids=[w.name for w in synth.SWEEP])
 def test_sweep_sampled_rows(w):
     check_sampled(w)
+
+
+def test_host_prefill_pipeline_matches_device_call():
+    # pinned host in, pinned host out, transfers overlapped per (batch, KV-head group)
+    for w, T, B in [(synth.TINY, 700, 2), (synth.LLAMA3_128K, 1000, 1)]:
+        q, k, v = synth.prefill_inputs(w, "cpu", T=T, B=B)
+        qh, kh, vh = [t.pin_memory() for t in (q, k, v)]
+        tab = _table(w)
+        hp = api.HostPrefill(B, w.Hq, w.Hkv, T, w.d, units_per_batch=3)
+        got = hp(qh, kh, vh, tab, True, 300, 4)
+        torch.cuda.synchronize()
+        again = hp(qh, kh, vh, tab, True, 300, 4)
+        torch.cuda.synchronize()
+        ref = api.attn_prefill(q.cuda(), k.cuda(), v.cuda(), tab, True, 300, 4)
+        api.device_status()
+        assert torch.equal(got, ref.cpu()) and torch.equal(again, ref.cpu())

@@ -174,6 +174,70 @@ def attn_prefill(q, k, v, table: RopeTable, causal: bool = True, window: int = 0
     return out
 
 
+class HostPrefill:
+    """Prefill from pinned host tensors into a pinned host output with the PCIe transfers
+    hidden behind the kernels.  The work is cut into (batch, KV-head group) units; unit i
+    is copied host->device on one stream, rotated and attended on a second (the caller's
+    stream) and copied back on a third, so the copies of later and earlier units run
+    while a unit computes.  Device buffers are allocated once for a given shape and
+    reused; call it repeatedly for a stream of prompts of that shape."""
+
+    def __init__(self, B, Hq, Hkv, T, d, device="cuda", units_per_batch=None):
+        self.shape = (B, Hq, Hkv, T, d)
+        self.g = Hq // Hkv
+        n = units_per_batch or min(Hkv, 8)
+        self.kv_per_unit = -(-Hkv // n)
+        dev = torch.device(device)
+        self.qd = torch.empty((B, Hq, T, d), dtype=torch.bfloat16, device=dev)
+        self.kd = torch.empty((B, Hkv, T, d), dtype=torch.bfloat16, device=dev)
+        self.vd = torch.empty_like(self.kd)
+        self.od = torch.empty_like(self.qd)
+        self.ws = torch.empty(attn_prefill_workspace_bytes(1, self.kv_per_unit, T, d),
+                              dtype=torch.uint8, device=dev)
+        self.h2d = torch.cuda.Stream(device=dev)
+        self.d2h = torch.cuda.Stream(device=dev)
+
+    def __call__(self, q, k, v, table: RopeTable, causal: bool = True, window: int = 0,
+                 n_sink: int = 0, out=None):
+        """q [B,Hq,T,d], k/v [B,Hkv,T,d] bf16 in pinned host memory, contiguous.  Returns
+        `out` (pinned, allocated if None).  All work is ordered before the caller's
+        current stream's later work; synchronise it before reading `out`."""
+        B, Hq, Hkv, T, d = self.shape
+        if q.shape != (B, Hq, T, d) or k.shape != (B, Hkv, T, d) or v.shape != k.shape:
+            raise ValueError("HostPrefill: tensor shapes differ from the ones it was built for")
+        for t in (q, k, v):
+            if t.is_cuda or not t.is_pinned() or not t.is_contiguous():
+                raise ValueError("HostPrefill expects contiguous tensors in pinned host memory")
+        if out is None:
+            out = torch.empty((B, Hq, T, d), dtype=torch.bfloat16).pin_memory()
+        comp = torch.cuda.current_stream(self.qd.device)
+        self.h2d.wait_stream(comp)  # device buffers are free once earlier calls computed
+        units = [(b, kv0, min(kv0 + self.kv_per_unit, Hkv))
+                 for b in range(B) for kv0 in range(0, Hkv, self.kv_per_unit)]
+        g = self.g
+        for b, kv0, kv1 in units:
+            q_sl = (b, slice(kv0 * g, kv1 * g))
+            kv_sl = (b, slice(kv0, kv1))
+            with torch.cuda.stream(self.h2d):
+                self.qd[q_sl].copy_(q[q_sl], non_blocking=True)
+                self.kd[kv_sl].copy_(k[kv_sl], non_blocking=True)
+                self.vd[kv_sl].copy_(v[kv_sl], non_blocking=True)
+                arrived = torch.cuda.Event()
+                arrived.record(self.h2d)
+            comp.wait_event(arrived)
+            qu = self.qd[b:b + 1, kv0 * g:kv1 * g]
+            attn_prefill(qu, self.kd[b:b + 1, kv0:kv1], self.vd[b:b + 1, kv0:kv1], table,
+                         causal, window, n_sink, out=self.od[b:b + 1, kv0 * g:kv1 * g],
+                         workspace=self.ws, stream=comp)
+            done = torch.cuda.Event()
+            done.record(comp)
+            with torch.cuda.stream(self.d2h):
+                self.d2h.wait_event(done)
+                out[q_sl].copy_(self.od[q_sl], non_blocking=True)
+        comp.wait_stream(self.d2h)
+        return out
+
+
 def prefill_prepare_kv(k, v, table: RopeTable, workspace, k_cache=None, k_rot_dbg=None,
                        stream=None):
     """First half of attn_prefill: rotated keys and values (fp16) into `workspace`."""
