@@ -180,7 +180,9 @@ class HostPrefill:
     is copied host->device on one stream, rotated and attended on a second (the caller's
     stream) and copied back on a third, so the copies of later and earlier units run
     while a unit computes.  Device buffers are allocated once for a given shape and
-    reused; call it repeatedly for a stream of prompts of that shape."""
+    reused; call it repeatedly for a stream of prompts of that shape.  Successive calls
+    overlap too: a unit's copy-in waits only for the previous call's kernels on that unit,
+    and its kernels only for the previous call's copy-out of it."""
 
     def __init__(self, B, Hq, Hkv, T, d, device="cuda", units_per_batch=None):
         self.shape = (B, Hq, Hkv, T, d)
@@ -196,12 +198,17 @@ class HostPrefill:
                               dtype=torch.uint8, device=dev)
         self.h2d = torch.cuda.Stream(device=dev)
         self.d2h = torch.cuda.Stream(device=dev)
+        self.units = [(b, kv0, min(kv0 + self.kv_per_unit, Hkv))
+                      for b in range(B) for kv0 in range(0, Hkv, self.kv_per_unit)]
+        self.computed = [None] * len(self.units)  # per unit: its kernels of the last call
+        self.copied_out = [None] * len(self.units)  # ... and its copy-out
 
     def __call__(self, q, k, v, table: RopeTable, causal: bool = True, window: int = 0,
                  n_sink: int = 0, out=None):
         """q [B,Hq,T,d], k/v [B,Hkv,T,d] bf16 in pinned host memory, contiguous.  Returns
         `out` (pinned, allocated if None).  All work is ordered before the caller's
-        current stream's later work; synchronise it before reading `out`."""
+        current stream's later work; synchronise it before reading `out` or changing the
+        inputs."""
         B, Hq, Hkv, T, d = self.shape
         if q.shape != (B, Hq, T, d) or k.shape != (B, Hkv, T, d) or v.shape != k.shape:
             raise ValueError("HostPrefill: tensor shapes differ from the ones it was built for")
@@ -211,29 +218,34 @@ class HostPrefill:
         if out is None:
             out = torch.empty((B, Hq, T, d), dtype=torch.bfloat16).pin_memory()
         comp = torch.cuda.current_stream(self.qd.device)
-        self.h2d.wait_stream(comp)  # device buffers are free once earlier calls computed
-        units = [(b, kv0, min(kv0 + self.kv_per_unit, Hkv))
-                 for b in range(B) for kv0 in range(0, Hkv, self.kv_per_unit)]
         g = self.g
-        for b, kv0, kv1 in units:
+        for u, (b, kv0, kv1) in enumerate(self.units):
             q_sl = (b, slice(kv0 * g, kv1 * g))
             kv_sl = (b, slice(kv0, kv1))
             with torch.cuda.stream(self.h2d):
+                if self.computed[u] is not None:  # the unit's inputs were read by then
+                    self.h2d.wait_event(self.computed[u])
                 self.qd[q_sl].copy_(q[q_sl], non_blocking=True)
                 self.kd[kv_sl].copy_(k[kv_sl], non_blocking=True)
                 self.vd[kv_sl].copy_(v[kv_sl], non_blocking=True)
                 arrived = torch.cuda.Event()
                 arrived.record(self.h2d)
             comp.wait_event(arrived)
+            if self.copied_out[u] is not None:  # the unit's last output has left
+                comp.wait_event(self.copied_out[u])
             qu = self.qd[b:b + 1, kv0 * g:kv1 * g]
             attn_prefill(qu, self.kd[b:b + 1, kv0:kv1], self.vd[b:b + 1, kv0:kv1], table,
                          causal, window, n_sink, out=self.od[b:b + 1, kv0 * g:kv1 * g],
                          workspace=self.ws, stream=comp)
             done = torch.cuda.Event()
             done.record(comp)
+            self.computed[u] = done
             with torch.cuda.stream(self.d2h):
                 self.d2h.wait_event(done)
                 out[q_sl].copy_(self.od[q_sl], non_blocking=True)
+                left = torch.cuda.Event()
+                left.record(self.d2h)
+            self.copied_out[u] = left
         comp.wait_stream(self.d2h)
         return out
 
