@@ -74,6 +74,10 @@ def _load():
                                          dp, c_double, c_int, c_int, c_int, i64p, c_long,
                                          dp, dp, dp, dp]
         lib.oracle_attn_rows.restype = c_int
+        lib.oracle_attn_rotated_f64.argtypes = [dp, dp, dp, c_int, c_int, c_int, c_int, c_int,
+                                                c_double, c_int, c_int, c_int, i64p, c_long,
+                                                dp, dp, dp]
+        lib.oracle_attn_rotated_f64.restype = c_int
         lib.oracle_decode.argtypes = [u16p, u16p, u16p, u16p, u16p, c_int, i32p,
                                       c_int, c_int, c_int, c_int, dp, c_double, c_int, c_int,
                                       dp, dp, dp, dp, dp]
@@ -213,6 +217,39 @@ def attn_rows(q_bits, k_bits, v_bits, theta, softmax_scale, causal=True, window=
     if rc != 0:
         raise ValueError(f"oracle_attn_rows failed ({rc})")
     return o, lse, qr
+
+
+def attn_rotated_f64(q_rot, k_rot, v, softmax_scale, causal=True, window=0, n_sink=0,
+                     rows=None, slopes=None):
+    """Exact attention on float64 operands whose queries and keys are already rotated:
+    q_rot [B,Hq,T,d], k_rot and v [B,Hkv,T,d].  rows as in attn_rows.  Returns
+    (o [n,d], lse [n])."""
+    lib = _load()
+    q = np.ascontiguousarray(q_rot, dtype=np.float64)
+    k = np.ascontiguousarray(k_rot, dtype=np.float64)
+    vv = np.ascontiguousarray(v, dtype=np.float64)
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, T, d) or vv.shape != k.shape:
+        raise ValueError("shape mismatch")
+    if rows is None:
+        n = B * Hq * T
+        rp = ctypes.POINTER(ctypes.c_int64)()
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        n = rows.shape[0]
+        rp = _ptr(rows, ctypes.c_int64)
+    o = np.empty((n, d), dtype=np.float64)
+    lse = np.empty(n, dtype=np.float64)
+    sp, _keep = _slopes(slopes, Hq)
+    rc = lib.oracle_attn_rotated_f64(_ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double),
+                                     _ptr(vv, ctypes.c_double), B, Hq, Hkv, T, d,
+                                     float(softmax_scale), int(bool(causal)), int(window),
+                                     int(n_sink), rp, n, _ptr(o, ctypes.c_double),
+                                     _ptr(lse, ctypes.c_double), sp)
+    if rc != 0:
+        raise ValueError(f"oracle_attn_rotated_f64 failed ({rc})")
+    return o, lse
 
 
 def decode(q_new, k_new, v_new, k_cache, v_cache, cache_len, theta, softmax_scale,

@@ -45,6 +45,9 @@
  *                       form, orthogonality, relative-position invariance).
  *   oracle_attn_rows    pinned (library SDPA special case, closed-form
  *                       means, page's "4 + last 4096" sink count, T=1).
+ *   oracle_attn_rotated_f64 pinned (equals oracle_attn_rows on its own
+ *                       rotation of bf16 inputs; library SDPA on operands that
+ *                       are not bf16 values; closed-form means for q = 0).
  *   oracle_decode       pinned (equals the prefill row at the same position).
  *   oracle_prefill_chunk pinned (Tq = 1 is decode; P0 = 0 is the full
  *                       prefill; torch float64 SDPA on the assembled keys).
@@ -362,6 +365,78 @@ int oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     free(krot);
     free(need);
     return 0;
+}
+
+/*
+ * Exact attention on operands given in double precision, the queries and keys
+ * already rotated: the definition of oracle_attn_rows without its rotation step.
+ *   q_rot [B,Hq,T,d], k_rot [B,Hkv,T,d], v [B,Hkv,T,d], contiguous doubles.
+ *   For each row: s_n = softmax_scale * q_rot_m . k_rot_n (minus slopes[h] (m - n)
+ *   when slopes is given) over visible n, P = exp(s - max) / sum, O = sum_n P_n v_n,
+ *   LSE = max + ln(sum).  ([P3] "Q K^T / sqrt(d_k)" table slide; [P2] key math.)
+ * With the oracle's own rotation of bf16 inputs it is oracle_attn_rows; with
+ * operands rounded in a stated way first (a test's choice) it gives exact
+ * attention of those rounded operands.
+ *   rows: n_rows flat indices (b*Hq + h)*T + m, or NULL for every row.
+ * Returns 0, -1 on bad arguments, -2 on allocation failure.
+ */
+int oracle_attn_rotated_f64(const double *q_rot, const double *k_rot, const double *v,
+                            int B, int Hq, int Hkv, int T, int d, double softmax_scale,
+                            int causal, int window, int n_sink,
+                            const int64_t *rows, long n_rows,
+                            double *o, double *lse, const double *slopes)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || T < 1 || d < 1 || (Hq % Hkv)) return -1;
+    const int group = Hq / Hkv;
+    const long total = (long)B * Hq * T;
+    if (rows == NULL) n_rows = total;
+    for (long r = 0; r < n_rows; ++r) {
+        const long flat = rows ? (long)rows[r] : r;
+        if (flat < 0 || flat >= total) return -1;
+    }
+    int fail = 0;
+#pragma omp parallel
+    {
+        double *sc = (double *)malloc(sizeof(double) * (size_t)T);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!sc || !acc) {
+#pragma omp atomic write
+            fail = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long r = 0; r < n_rows; ++r) {
+            if (!sc || !acc) continue;
+            const long flat = rows ? (long)rows[r] : r;
+            const long m = flat % T, bh = flat / T;
+            const long b = bh / Hq, h = bh % Hq;
+            const long kv = b * Hkv + h / group;
+            const double *qr = q_rot + flat * d;
+            const double *kr = k_rot + kv * (long)T * d;
+            const double *vb = v + kv * (long)T * d;
+            double mx = -INFINITY;
+            for (long n = 0; n < T; ++n) {
+                if (!visible(m, n, causal, window, n_sink)) { sc[n] = -INFINITY; continue; }
+                double dot = 0.0;
+                for (int j = 0; j < d; ++j) dot += qr[j] * kr[n * d + j];
+                sc[n] = softmax_scale * dot;
+                if (slopes) sc[n] -= slopes[h] * (double)(m - n);
+                if (sc[n] > mx) mx = sc[n];
+            }
+            double z = 0.0;
+            for (int j = 0; j < d; ++j) acc[j] = 0.0;
+            for (long n = 0; n < T; ++n) {
+                if (sc[n] == -INFINITY) continue;
+                const double p = exp(sc[n] - mx);
+                z += p;
+                for (int j = 0; j < d; ++j) acc[j] += p * vb[n * d + j];
+            }
+            for (int j = 0; j < d; ++j) o[r * d + j] = acc[j] / z;
+            if (lse) lse[r] = mx + log(z);
+        }
+        free(sc);
+        free(acc);
+    }
+    return fail ? -2 : 0;
 }
 
 /*

@@ -313,6 +313,55 @@ def test_matches_library_sdpa_float64(causal, window, n_sink):
                                rtol=0, atol=1e-12)
 
 
+def test_rotated_f64_equals_attn_rows_on_its_own_rotation():
+    B, Hq, Hkv, T, d = 2, 6, 2, 45, 16
+    th, _, ss = oracle.rope_theta(d, 10000.0, 16, 4.0, "yarn")
+    q, k, v = _rand_qkv(B, Hq, Hkv, T, d)
+    pos = np.arange(T, dtype=np.float64)
+    qr = oracle.rotate(q, np.broadcast_to(pos, (B, Hq, T)).reshape(-1), th)
+    kr = oracle.rotate(k, np.broadcast_to(pos, (B, Hkv, T)).reshape(-1), th)
+    for causal, w, s in [(True, 0, 0), (True, 6, 2), (False, 0, 0)]:
+        o1, l1, _ = oracle.attn_rows(q, k, v, th, ss, causal, w, s)
+        o2, l2 = oracle.attn_rotated_f64(qr, kr, bits_to_f64(v), ss, causal, w, s)
+        np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(l2, l1, rtol=0, atol=1e-13)
+    rows = np.array([0, 5, 44, 45 * 7 + 3, B * Hq * T - 1])
+    o3, l3 = oracle.attn_rotated_f64(qr, kr, bits_to_f64(v), ss, rows=rows)
+    o1, l1, _ = oracle.attn_rows(q, k, v, th, ss)
+    np.testing.assert_allclose(o3, o1[rows], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l3, l1[rows], rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal,window,n_sink", [(True, 0, 0), (True, 5, 2), (False, 0, 0)])
+def test_rotated_f64_matches_library_sdpa_on_non_bf16_values(causal, window, n_sink):
+    # operands that are no bf16 (or fp16) values, large enough for a peaked softmax
+    B, Hq, Hkv, T, d = 1, 4, 1, 29, 12
+    q = RNG.standard_normal((B, Hq, T, d)) * 7.3
+    k = RNG.standard_normal((B, Hkv, T, d)) * 1.1
+    v = RNG.standard_normal((B, Hkv, T, d)) * 3e4
+    ss = 0.1442
+    o, lse = oracle.attn_rotated_f64(q, k, v, ss, causal, window, n_sink)
+    mask = torch.from_numpy(_mask(T, causal, window, n_sink))
+    kt = torch.from_numpy(k).repeat_interleave(Hq, dim=1)
+    vt = torch.from_numpy(v).repeat_interleave(Hq, dim=1)
+    ref = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(q), kt, vt,
+                                                           attn_mask=mask, scale=ss)
+    np.testing.assert_allclose(o.reshape(B, Hq, T, d), ref.numpy(), rtol=1e-12, atol=1e-8)
+    scores = np.einsum("bhmd,bhnd->bhmn", q, kt.numpy()) * ss
+    scores = np.where(mask.numpy(), scores, -np.inf)
+    np.testing.assert_allclose(lse.reshape(B, Hq, T), scipy.special.logsumexp(scores, axis=-1),
+                               rtol=0, atol=1e-10)
+
+
+def test_rotated_f64_zero_query_gives_prefix_means():
+    T, d = 120, 3
+    k = RNG.standard_normal((1, 1, T, d))
+    v = RNG.standard_normal((1, 1, T, d))
+    cs = np.vstack([np.zeros((1, d)), np.cumsum(v[0, 0], axis=0)])
+    o, _ = oracle.attn_rotated_f64(np.zeros((1, 1, T, d)), k, v, 0.3, True, 0, 0)
+    np.testing.assert_allclose(o, cs[1:] / np.arange(1, T + 1)[:, None], rtol=0, atol=1e-12)
+
+
 def test_rows_sum_to_one_through_v_ones():
     B, Hq, Hkv, T, d = 1, 4, 2, 64, 8
     th, _, ss = oracle.rope_theta(d, 10000.0, 16, 4.0, "yarn")
