@@ -41,6 +41,7 @@ extern "C" {
 #define YR_EUNSUPPORTED (-2)  /* valid but not implemented (head_dim, device) */
 #define YR_ECUDA (-3)         /* a CUDA runtime/driver call failed */
 #define YR_ETIMEOUT (-4)      /* a kernel gave up on an internal wait */
+#define YR_ERANGE (-5)        /* a prefill operand fell outside the fp16 range (see below) */
 
 /* Position methods ("Arch_03_Long_Context": RoPE, PI, NTK-aware and YaRN slides). */
 #define YR_ROPE 0  /* theta_i = base^(-2i/d) */
@@ -150,7 +151,10 @@ size_t yr_attn_prefill_workspace_bytes(int B, int Hkv, int T, int d);
  *   aligned.  It is overwritten; its contents after the call are unspecified.
  * Precision: inputs and outputs bf16; rotation angles reduced in fp64; rotated
  *   q/k, the probabilities and v enter the tensor cores as fp16; all sums fp32.
- *   |rotated q|, |rotated k| and |v| must stay below 65504 (fp16 range).
+ *   |rotated q|, |rotated k| and |v| must stay below 65520, the fp16 range: a
+ *   value outside it (or a NaN) sets the range bit of the device status word,
+ *   which yr_device_status() then reports as YR_ERANGE; the output of such a
+ *   call is unspecified.  The probabilities are kept within fp16 by the kernel.
  * Errors: YR_EINVAL (shapes, strides, alignment, flags, workspace too small),
  *   YR_EUNSUPPORTED (d not 64 or 128, device not sm_100), YR_ECUDA.
  */
@@ -332,8 +336,10 @@ int yr_attn_decode(const void *q_new, const void *k_new, const void *v_new,
  *   that needs more -- yr_attn_decode_workspace_bytes(B, Hq, Hkv, d, T_max)
  *   bytes -- returns YR_EINVAL without launching anything (e.g. 16 sequences of
  *   32768 slots with 128 query and 8 KV heads of d=128 need just over 16 MiB).
- *   The first call on each device looks up the scratch address for that device
- *   with the CUDA runtime; make that first call before any stream capture.
+ *   The scratch is per CUDA context: each device's primary context, and any
+ *   context the host application makes current, has its own copy.  The first
+ *   call in each context looks up the scratch address in that context with the
+ *   CUDA runtime; make that first call before any stream capture.
  *   Every call shares the one array, which keeps the last call's contents: calls
  *   that overlap on the GPU (other streams, other host threads) race on it, so
  *   order them.  Nothing in it needs to start at zero, because each call writes
@@ -350,8 +356,10 @@ int yr_attn_decode_noalloc(const void *q_new, const void *k_new, const void *v_n
 /*
  * device_status -- synchronise `stream`, then read and clear the device status
  * word of the current device.  Returns YR_OK, YR_ETIMEOUT (a kernel gave up on
- * a wait; yr_last_error names where) or YR_EINVAL (a decode cache length was
- * out of range), or YR_ECUDA.
+ * a wait; yr_last_error names where), YR_ERANGE (a prefill, chunk or block call
+ * met a rotated query or key, or a value, outside the fp16 range), YR_EINVAL (a
+ * decode cache length was out of range), or YR_ECUDA.  When several bits are
+ * set the first of those codes is returned and the message names them all.
  */
 int yr_device_status(void *stream);
 

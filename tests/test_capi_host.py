@@ -31,6 +31,16 @@ def test_library_exports_every_declared_symbol(lib):
     assert lib.yr_version() == 10000
 
 
+def test_error_codes_match_the_header():
+    with open(os.path.join(ROOT, "include", "yarnattn.h")) as f:
+        header = f.read()
+    codes = dict(re.findall(r"^#define (YR_E\w+|YR_OK) \(?(-?\d+)\)?", header, flags=re.M))
+    assert set(codes) == {"YR_OK", "YR_EINVAL", "YR_EUNSUPPORTED", "YR_ECUDA", "YR_ETIMEOUT",
+                          "YR_ERANGE"}
+    for name, value in codes.items():
+        assert getattr(api, name) == int(value), name
+
+
 @pytest.mark.parametrize("method", ["rope", "pi", "ntk", "yarn"])
 @pytest.mark.parametrize("d,base,L,s", [(64, 10000.0, 64, 4.0), (128, 10000.0, 4096, 4.0),
                                         (128, 500000.0, 8192, 16.0), (128, 10000.0, 4096, 1.0)])

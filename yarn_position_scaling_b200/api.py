@@ -14,7 +14,7 @@ import torch
 
 from .build import LIB
 
-YR_OK, YR_EINVAL, YR_EUNSUPPORTED, YR_ECUDA, YR_ETIMEOUT = 0, -1, -2, -3, -4
+YR_OK, YR_EINVAL, YR_EUNSUPPORTED, YR_ECUDA, YR_ETIMEOUT, YR_ERANGE = 0, -1, -2, -3, -4, -5
 ROPE, PI, NTK, YARN = 0, 1, 2, 3
 NTK_DYNAMIC, YARN_DIMRAMP, FACTORS, ALIBI = 4, 5, 6, 7
 METHODS = {"rope": ROPE, "pi": PI, "ntk": NTK, "yarn": YARN, "ntk_dynamic": NTK_DYNAMIC,
@@ -49,8 +49,9 @@ class RopeTable(ctypes.Structure):
 _lib = None
 
 
-def load(path: str | None = None) -> ctypes.CDLL:
-    """Load libyarnattn.so (once).  Raises if it is missing."""
+def load(path: str | None = None, make_default: bool = False) -> ctypes.CDLL:
+    """Load libyarnattn.so (once).  Raises if it is missing.  With `path`, load that build
+    of the library instead; make_default=True makes it the one every call below uses."""
     global _lib
     if _lib is not None and path is None:
         return _lib
@@ -99,7 +100,7 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.yr_last_error.restype = ctypes.c_char_p
     lib.yr_version.argtypes = []
     lib.yr_version.restype = ci
-    if path is None:
+    if path is None or make_default:
         _lib = lib
     return lib
 

@@ -8,7 +8,9 @@
 //
 // One thread handles 8 consecutive elements (16 bytes) of one key row and the
 // same 8 elements of the value row: coalesced 16-byte loads and stores, a
-// grid-stride loop sized to the SM count.
+// grid-stride loop sized to the SM count.  A rotated key or a value that does not
+// fit fp16 (|x| >= 65520, or not a number) sets the range bit of the device status
+// word instead of passing silently into the attention as infinity.
 #pragma once
 #include "sm100_ptx.cuh"
 
@@ -42,6 +44,7 @@ __global__ void __launch_bounds__(256) kv_prep_kernel(const __grid_constant__ Kv
     __shared__ double turns[64];
     if (threadIdx.x < p.d / 2) turns[threadIdx.x] = p.turns[threadIdx.x];
     __syncthreads();
+    bool bad = false;  // some rotated key or value of this thread does not fit fp16
     const int cpr = p.d >> 3;
     const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
     for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -73,6 +76,8 @@ __global__ void __launch_bounds__(256) kv_prep_kernel(const __grid_constant__ Kv
                        pack_half2(y[6], y[7]));
         float vf[8];
         unpack_bf16x8(vr, vf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) bad |= f16_out_of_range(y[i]) | f16_out_of_range(vf[i]);
         *reinterpret_cast<uint4 *>(p.v16 + off) =
             make_uint4(pack_half2(vf[0], vf[1]), pack_half2(vf[2], vf[3]),
                        pack_half2(vf[4], vf[5]), pack_half2(vf[6], vf[7]));
@@ -92,6 +97,7 @@ __global__ void __launch_bounds__(256) kv_prep_kernel(const __grid_constant__ Kv
             d4[1] = make_float4(y[4], y[5], y[6], y[7]);
         }
     }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) raise_status(kStatusRange);
 }
 
 // Chunked prefill: the Tq new tokens of each sequence sit at positions P0 ..
@@ -112,9 +118,12 @@ struct ChunkPrepParams {
     double turns[64];
 };
 
-__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 &raw) {
+// bf16 -> fp16, eight at a time; `bad` is set if one of them does not fit fp16.
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(const uint4 &raw, bool &bad) {
     float x[8];
     unpack_bf16x8(raw, x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) bad |= f16_out_of_range(x[i]);
     return make_uint4(pack_half2(x[0], x[1]), pack_half2(x[2], x[3]), pack_half2(x[4], x[5]),
                       pack_half2(x[6], x[7]));
 }
@@ -123,6 +132,7 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const __grid_constant__
     __shared__ double turns[64];
     if (threadIdx.x < p.d / 2) turns[threadIdx.x] = p.turns[threadIdx.x];
     __syncthreads();
+    bool bad = false;  // some key or value of this thread does not fit fp16
     const int cpr = p.d >> 3;
     const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
     for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -136,8 +146,8 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const __grid_constant__
         if (t < p.P0) {
             const uint4 kr = __ldg(reinterpret_cast<const uint4 *>(p.kc + slot));
             const uint4 vr = __ldg(reinterpret_cast<const uint4 *>(p.vc + slot));
-            *reinterpret_cast<uint4 *>(p.k16 + off) = bf16x8_to_f16x8(kr);
-            *reinterpret_cast<uint4 *>(p.v16 + off) = bf16x8_to_f16x8(vr);
+            *reinterpret_cast<uint4 *>(p.k16 + off) = bf16x8_to_f16x8(kr, bad);
+            *reinterpret_cast<uint4 *>(p.v16 + off) = bf16x8_to_f16x8(vr, bad);
             continue;
         }
         const long long src = (bh * p.Tq + (t - p.P0)) * p.d + c * 8;
@@ -164,9 +174,12 @@ __global__ void __launch_bounds__(256) chunk_prep_kernel(const __grid_constant__
             w[i] = *reinterpret_cast<uint32_t *>(&b2);
         }
         *reinterpret_cast<uint4 *>(p.kc + slot) = make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4 *>(p.v16 + off) = bf16x8_to_f16x8(vr);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) bad |= f16_out_of_range(y[i]);
+        *reinterpret_cast<uint4 *>(p.v16 + off) = bf16x8_to_f16x8(vr, bad);
         *reinterpret_cast<uint4 *>(p.vc + slot) = vr;
     }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) raise_status(kStatusRange);
 }
 
 }  // namespace yr

@@ -33,7 +33,8 @@
 // Rotation ("Arch_03_Long_Context", RoPE slide): pair (2i, 2i+1) of the query
 // at position m turns by m * theta'_i.  Each softmax warp reduces the angle of
 // every pair at its first row in fp64 (turns minus the nearest integer); a row
-// adds lane * theta'_i / (2 pi) in fp32 and takes fp32 sin/cos.  Rarely run
+// adds lane * theta'_i / (2 pi) in fp32 and takes fp32 sin/cos.  A rotated value
+// that does not fit fp16 sets the range bit of the device status word.  Rarely run
 // paths are kept small (rolled loops, compact masks): their instructions are
 // fetched cold.
 //
@@ -86,8 +87,9 @@ struct alignas(64) PrefillParams {
     int alibi;     // 1: add the ALiBi bias -m_h (i - j) to the logits
     float sl2;  // softmax_scale * log2(e)
     unsigned long long timeout_ns;
-    // Failure-detection test hook: CTA 0's producer issues no copy for this key tile
-    // index (-1: off), so a wait that nothing will complete runs out of time.
+    // Failure-detection test hook, compiled only into the test build (YR_FAULT_HOOKS):
+    // CTA 0's producer issues no copy for this key tile index (-1: off), so a wait that
+    // nothing will complete runs out of time.
     int fault_drop_tile;
     double turns[64];
 };
@@ -300,7 +302,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             for (int idx = 0; idx < tp.n && ok; ++idx) {
                 const int j = tile_at(tp, idx);
                 const int ks = idx % kKStages, vs = idx % kVStages;
+#ifdef YR_FAULT_HOOKS
                 if (idx == p.fault_drop_tile && blockIdx.x == 0) continue;
+#endif
                 ok = mbar_wait(&sm->k_empty[ks], ((idx / kKStages) & 1) ^ 1, abort, p.timeout_ns);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&sm->k_full[ks], kSub * kSubTileBytes);
@@ -477,6 +481,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 }
                 __syncwarp();
                 const float lanef = static_cast<float>(lane);
+                bool bad = false;  // a rotated value of this row does not fit fp16
 #pragma unroll 1
                 for (int s = 0; s < kSub; ++s) {
 #pragma unroll 1
@@ -499,6 +504,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                             __sincosf((turns - near) * 6.2831853071795865f, &sn, &cs);
                             y[2 * pp] = a * cs - bb * sn;
                             y[2 * pp + 1] = a * sn + bb * cs;
+                            bad |= f16_out_of_range(y[2 * pp]) | f16_out_of_range(y[2 * pp + 1]);
                             out[pp] = pack_half2(y[2 * pp], y[2 * pp + 1]);
                         }
                         *ptr = make_uint4(out[0], out[1], out[2], out[3]);
@@ -509,6 +515,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         }
                     }
                 }
+                if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(kStatusRange);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm->q_ready[t]);

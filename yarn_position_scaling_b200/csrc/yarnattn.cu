@@ -9,6 +9,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <unordered_map>
 
 #include "../../include/yarnattn.h"
 #include "decode_sm100.cuh"
@@ -59,26 +60,72 @@ uint64_t wait_timeout_ns() {
     return ns;
 }
 
-// Per-device one-time set-up: architecture check and shared-memory opt-in.
+// The context current on the calling thread.  The CUDA runtime launches into it, and
+// function attributes and the addresses of module globals belong to it, so the
+// one-time set-up below is kept per context (a host application may make a context
+// of its own current, or reset the device, between calls).
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+template <typename Fn>
+Fn driver_entry(const char *name) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        return reinterpret_cast<Fn>(ptr);
+    return nullptr;
+}
+
+int current_context(int *dev_out, unsigned long long *ctx_id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        get_current = driver_entry<CtxGetCurrentFn>("cuCtxGetCurrent");
+        get_id = driver_entry<CtxGetIdFn>("cuCtxGetId");
+    });
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if (!get_current || !get_id)
+        return fail(YR_ECUDA, "cuCtxGetCurrent/cuCtxGetId are not available from the driver");
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS)
+        return fail(YR_ECUDA, "cuCtxGetCurrent failed");
+    if (ctx == nullptr) {
+        // No context yet on this thread: the runtime would make the device's primary
+        // context current at its next call; make it current now so it can be named.
+        e = cudaSetDevice(dev);
+        if (e != cudaSuccess) return cuda_fail("cudaSetDevice", e);
+        if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+            return fail(YR_ECUDA, "no CUDA context is current");
+    }
+    if (get_id(ctx, ctx_id) != CUDA_SUCCESS) return fail(YR_ECUDA, "cuCtxGetId failed");
+    *dev_out = dev;
+    return YR_OK;
+}
+
+// Per-context one-time set-up: architecture check and shared-memory opt-in.
 struct DeviceState {
-    bool ready = false;
     bool sm100 = false;
     bool prefill_regs_ok = false;  // launched register count covers the setmaxnreg split
     int sm_count = 0;
 };
 std::mutex g_dev_mu;
-DeviceState g_dev[64];
+std::unordered_map<unsigned long long, DeviceState> g_dev;  // by context id
 
-int prepare_device(int *sm_count) {
+int prepare_device(int *sm_count, DeviceState *out = nullptr) {
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
-    if (dev < 0 || dev >= 64) return fail(YR_EUNSUPPORTED, "device index out of range");
+    unsigned long long ctx = 0;
+    int rc = current_context(&dev, &ctx);
+    if (rc != YR_OK) return rc;
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    DeviceState &st = g_dev[dev];
-    if (!st.ready) {
+    auto it = g_dev.find(ctx);
+    if (it == g_dev.end()) {
+        DeviceState st;
         cudaDeviceProp prop;
-        e = cudaGetDeviceProperties(&prop, dev);
+        cudaError_t e = cudaGetDeviceProperties(&prop, dev);
         if (e != cudaSuccess) return cuda_fail("cudaGetDeviceProperties", e);
         st.sm100 = (prop.major == 10 && prop.minor == 0);
         st.sm_count = prop.multiProcessorCount;
@@ -116,10 +163,12 @@ int prepare_device(int *sm_count) {
                 if (fa.numRegs < yr::kMinLaunchRegs) st.prefill_regs_ok = false;
             }
         }
-        st.ready = true;
+        it = g_dev.emplace(ctx, st).first;
     }
+    const DeviceState &st = it->second;
     if (!st.sm100) return fail(YR_EUNSUPPORTED, "the current device is not sm_100 (B200)");
     if (sm_count) *sm_count = st.sm_count;
+    if (out) *out = st;
     return YR_OK;
 }
 
@@ -300,13 +349,6 @@ int launch_prepare(const void *k, const void *v, void *k_cache, float *k_rot_dbg
     return YR_OK;
 }
 
-int prefill_regs_ok() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    std::lock_guard<std::mutex> lk(g_dev_mu);
-    return g_dev[dev].prefill_regs_ok ? 1 : 0;
-}
-
 // T query rows against Tk keys laid out in the workspace as fp16 [B*Hkv][Tk][d]
 // rotated keys, then the same for values.  Key n sits at position k_pos0 + n and
 // query row r at k_pos0 + q_off + r; masks use the offsets relative to key 0.
@@ -315,14 +357,16 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
                   const yr_rope_table *tab, int causal, int window, int n_sink,
                   const void *workspace, cudaStream_t st, int Tk, int q_off, int k_pos0 = 0,
                   float *o32 = nullptr) {
-    if (!prefill_regs_ok())
+    DeviceState ds;
+    int rc = prepare_device(nullptr, &ds);
+    if (rc != YR_OK) return rc;
+    if (!ds.prefill_regs_ok)
         return fail(YR_EUNSUPPORTED, "prefill kernel was built with too few registers per thread "
                                      "for its warpgroup register split");
     const __half *k16 = static_cast<const __half *>(workspace);
     const __half *v16 = k16 + static_cast<size_t>(B) * Hkv * Tk * d;
     yr::PrefillParams pp;
     std::memset(&pp, 0, sizeof pp);
-    int rc;
     {
         const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T),
                                     static_cast<cuuint64_t>(Hq), static_cast<cuuint64_t>(B)};
@@ -360,9 +404,13 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     pp.alibi = tab->method == YR_ALIBI ? 1 : 0;
     pp.sl2 = static_cast<float>(tab->softmax_scale * 1.4426950408889634);
     pp.timeout_ns = wait_timeout_ns();
-    // Test hook for the failure path (read on every launch; unset in normal use).
+#ifdef YR_FAULT_HOOKS
+    // Test build only: the failure-path hook, read on every launch.
     const char *drop = std::getenv("YR_FAULT_DROP_KV_TILE");
     pp.fault_drop_tile = drop ? static_cast<int>(std::strtol(drop, nullptr, 10)) : -1;
+#else
+    pp.fault_drop_tile = -1;
+#endif
     for (int i = 0; i < d / 2; ++i) pp.turns[i] = tab->turns[i];
     const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * Hq * pp.n_qblocks);
     if (d == 128)
@@ -658,27 +706,30 @@ extern "C" int yr_attn_decode(const void *q_new, const void *k_new, const void *
 // Decode without a caller-supplied workspace.  The split-KV partial results go to
 // this fixed array instead; every GPU that loads the library holds it until exit.
 // In host code `g_decode_noalloc_scratch` is only a stand-in for the symbol, not a
-// device address: the address is looked up per device with cudaGetSymbolAddress.
+// device address: the address is looked up per context with cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[YR_DECODE_NOALLOC_SCRATCH_BYTES];
 
 namespace yr_host {
 std::mutex g_scratch_mu;
-void *g_scratch_ptr[64] = {};
+std::unordered_map<unsigned long long, void *> g_scratch_ptr;  // by context id
 
-// Set-up, once per device, with that device current.
+// Set-up, once per context (each device's primary context, or a context the host
+// application made current), with that context current: the address of the array
+// in the context's instance of this module.
 int noalloc_scratch(void **out) {
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
-    if (dev < 0 || dev >= 64) return fail(YR_EUNSUPPORTED, "device index out of range");
+    unsigned long long ctx = 0;
+    int rc = current_context(&dev, &ctx);
+    if (rc != YR_OK) return rc;
     std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
+    auto it = g_scratch_ptr.find(ctx);
+    if (it == g_scratch_ptr.end()) {
         void *ptr = nullptr;
-        e = cudaGetSymbolAddress(&ptr, g_decode_noalloc_scratch);
+        cudaError_t e = cudaGetSymbolAddress(&ptr, g_decode_noalloc_scratch);
         if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress(decode scratch)", e);
-        g_scratch_ptr[dev] = ptr;
+        it = g_scratch_ptr.emplace(ctx, ptr).first;
     }
-    *out = g_scratch_ptr[dev];
+    *out = it->second;
     return YR_OK;
 }
 }  // namespace yr_host
@@ -728,6 +779,10 @@ extern "C" int yr_device_status(void *stream) {
     if (v & yr::kStatusTimeoutSoftmax) msg += " prefill-softmax-timeout";
     if (v & yr::kStatusTimeoutDrain) msg += " prefill-drain-timeout";
     if (v & yr::kStatusBadCacheLen) msg += " decode-cache-length-out-of-range";
+    if (v & yr::kStatusRange)
+        msg += " prefill-operand-outside-fp16-range (|rotated q|, |rotated k| or |v| >= 65520,"
+               " or not a number)";
     set_error(msg);
-    return (v & 0xFFu) ? YR_ETIMEOUT : YR_EINVAL;
+    if (v & 0xFFu) return YR_ETIMEOUT;
+    return (v & yr::kStatusRange) ? YR_ERANGE : YR_EINVAL;
 }
