@@ -3,12 +3,15 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl yarn|reference]
 
-One step is one prefill of the Llama-2-7B-shaped workload (B=1, Hq=Hkv=32,
-d=128, T=16384, causal, YaRN base 1e4, L_train 4096, s=4): the rotated-key pass
-plus the attention kernel, inputs resident in HBM.  The headline is prefill
-TFLOP/s with causal FLOPs counted (4 d Hq B sum_m |visible(m)|).  The same run
-times the single-token decode workload (B=8, Hq=32, Hkv=8, d=128, cache
-lengths U[32768,131072]) and reports it as KV-read GB/s under "decode".
+One step is one prefill of the Llama-3-8B-shaped GQA workload at 128K (B=1, Hq=32,
+Hkv=8, d=128, T=131072, causal, YaRN base 5e5, L_train 8192, s=16): the
+rotated-key pass plus the attention kernel, inputs resident in HBM.  It is the
+largest single-GPU prefill configuration; the headline is prefill TFLOP/s with
+causal FLOPs counted (4 d Hq B sum_m |visible(m)|).  The same run times the other
+workloads and puts them at the end of the line: the method/structure sweep at
+64K, the chunked prefill, ring attention over emulated ranks, the 16K MHA
+prefill, and last the single-token decode workload (B=8, Hq=32, Hkv=8, d=128,
+cache lengths U[32768,131072]) as KV-read GB/s.
 
 For N > 1 (launched with torch.distributed.run) every rank runs the same
 workload as an independent replica; NCCL carries only the barrier and the
@@ -41,15 +44,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["yarn", "reference"], default="yarn")
     ap.add_argument("--decode-steps", type=int, default=None)
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-other-workloads", action="store_true",
-                    help="skip the 128K and sweep prefill workloads")
+                    help="skip the sweep, chunk, ring and 16K prefill workloads")
+    ap.add_argument("--headline", default="llama3_8b_128k_gqa_prefill",
+                    help="prefill workload of the headline (a name from synth.ALL)")
     ap.add_argument("--other-steps", type=int, default=3)
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="sequences in the decode workload (default 8; smaller for profiling)")
@@ -255,7 +260,7 @@ def oracle_sample(w, seconds: float, seed: int = 0):
 
 
 def reference_arm(args, dist: Dist):
-    w = synth.LLAMA2_16K
+    w = synth.ALL[args.headline]
     line = {"impl": "reference"}
     if dist.rank != 0:
         return None
@@ -444,6 +449,18 @@ def e2e_prefill(w, steps, warmup, stream):
     return step, h2d, d2h
 
 
+def _r(x, nd=4):
+    """Round for the JSON line (keeps it short enough for its tail to carry the
+    per-workload results)."""
+    if isinstance(x, float):
+        return float(f"{x:.{nd}g}")
+    if isinstance(x, dict):
+        return {k: _r(v, nd) for k, v in x.items()}
+    if isinstance(x, list):
+        return [_r(v, nd) for v in x]
+    return x
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -466,13 +483,13 @@ def main():
     stream = torch.cuda.current_stream()
     peaks, peak_src = load_peaks()
     n = dist.world
-    wp, wd = synth.LLAMA2_16K, synth.DECODE
+    wp, wd = synth.ALL[args.headline], synth.DECODE
     if args.decode_batch:
         import dataclasses
         wd = dataclasses.replace(wd, B=args.decode_batch)
     steps, warm = args.steps, max(3, args.warmup)
-    dsteps = args.decode_steps or steps
-    esteps = args.e2e_steps or max(3, min(steps // 10, 30))
+    dsteps = args.decode_steps or max(steps, 20)
+    esteps = args.e2e_steps or steps
 
     # ---------------- prefill (headline)
     pstep, keep = prefill_bench(wp, steps, warm, stream)
@@ -490,9 +507,41 @@ def main():
     ms_per_step = total_ms / steps
     value = throughput(flops_step, steps, total_ms, n, 1e12)
     attn_tflops = flops_step / (attn_ms_max / steps * 1e-3) / 1e12
-    peak_t = peaks["bf16_tflops"]
+    # Each attention launch runs for a large part of a second inside a seconds-long
+    # loop: the sustained (power-capped) tensor peak is its denominator.
+    long_step = attn_ms_max / steps > 20.0
+    peak_t = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
+    peak_burst = peaks["bf16_tflops"]
     del keep, pstep
     torch.cuda.empty_cache()
+
+    # ---------------- the other prefill workloads
+    others = {}
+    if not args.no_other_workloads:
+        for w in synth.SWEEP:
+            r = workload_prefill(w, args.other_steps, stream, dist, peak_burst)
+            others[w.name.replace("sweep_", "")] = {
+                "tflops": r["attn_kernel_tflops"], "step_tflops": r["step_tflops"],
+                "frac": r["frac_of_peak"]}
+            torch.cuda.empty_cache()
+        r = chunk_bench(synth.CHUNK, args.other_steps, stream, dist, peak_burst)
+        others["chunk_124k_plus_4k"] = {"tflops": r["call_tflops"], "frac": r["frac_of_peak"],
+                                        "ms": r["call_ms"]}
+        torch.cuda.empty_cache()
+        wr = synth.LLAMA3_128K
+        r = ring_bench(wr, 8, args.other_steps, stream, dist, peak_burst)
+        others["ring_128k_8_emulated_ranks"] = {"tflops": r["call_tflops"],
+                                                "frac": r["frac_of_peak"]}
+        torch.cuda.empty_cache()
+        w16 = synth.LLAMA2_16K
+        r = workload_prefill(w16, max(args.other_steps, 20), stream, dist, peak_burst)
+        prefill_16k = {"workload": w16.name, "step_tflops": r["step_tflops"],
+                       "attn_kernel_tflops": r["attn_kernel_tflops"],
+                       "attn_kernel_ms": r["attn_kernel_ms"], "frac_of_burst": r["frac_of_peak"],
+                       "steps": r["steps"]}
+        torch.cuda.empty_cache()
+    else:
+        prefill_16k = None
 
     # ---------------- decode
     dstep, lens = decode_bench(wd, dsteps, warm, stream)
@@ -508,19 +557,6 @@ def main():
     del dstep
     torch.cuda.empty_cache()
 
-    # ---------------- the other prefill workloads (128K, method/structure sweep)
-    others = {}
-    if not args.no_other_workloads:
-        for w in [synth.LLAMA3_128K] + synth.SWEEP:
-            others[w.name] = workload_prefill(w, args.other_steps, stream, dist, peak_t)
-            torch.cuda.empty_cache()
-        others[synth.CHUNK.name] = chunk_bench(synth.CHUNK, args.other_steps, stream, dist, peak_t)
-        torch.cuda.empty_cache()
-        wr = synth.LLAMA3_128K
-        others["ring_" + wr.name + "_8_ranks"] = ring_bench(wr, 8, args.other_steps, stream, dist,
-                                                              peak_t)
-        torch.cuda.empty_cache()
-
     # ---------------- end to end through the API with host buffers
     estep, h2d, d2h = e2e_prefill(wp, esteps, 2, stream)
     dist.barrier()
@@ -528,6 +564,8 @@ def main():
     dist.barrier()
     etotal_ms = dist.max(etotal_ms)
     e2e_value = throughput(flops_step, esteps, etotal_ms, n, 1e12)
+    del estep
+    torch.cuda.empty_cache()
 
     # ---------------- CPU oracle baseline (rank 0, N=1 only)
     cpu = None
@@ -544,41 +582,41 @@ def main():
         "data": "synthetic: seeded i.i.d. N(0,1) inputs rounded to bf16",
         "config": {"workload": wp.name, "B": wp.B, "Hq": wp.Hq, "Hkv": wp.Hkv, "d": wp.d,
                    "T": wp.T, "method": wp.method, "base": wp.base, "L_train": wp.L_train,
-                   "scale": wp.scale, "causal": True, "io_dtype": "bf16",
-                   "mma_operands": "fp16", "accumulate": "fp32",
-                   "parallelism": f"replicas x{n}",
+                   "scale": wp.scale, "causal": wp.causal, "window": wp.window,
+                   "n_sink": wp.n_sink, "io_dtype": "bf16", "mma_operands": "fp16",
+                   "accumulate": "fp32", "parallelism": f"replicas x{n}",
                    "l2": "no flush: q+k+v+o = %.0f MB per step > 126 MB L2" %
-                         (4 * wp.B * wp.Hq * wp.T * wp.d * 2 / 2 ** 20),
+                         ((2 * wp.B * wp.Hq + 2 * wp.B * wp.Hkv) * wp.T * wp.d * 2 / 2 ** 20),
                    "step": "yr_prefill_prepare_kv + yr_prefill_attend (= yr_attn_prefill)"},
         "roofline": {"bound": "tensor", "kernel": "prefill_attn_kernel<128>",
                      "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
-                     "frac": attn_tflops / peak_t, "peak_source": f"{peak_src} bf16 burst "
-                     "(fp16 tensor rate equals bf16)",
-                     "peak_sustained": peaks["bf16_tflops_sustained"],
-                     "frac_of_sustained": attn_tflops / peaks["bf16_tflops_sustained"],
+                     "frac": attn_tflops / peak_t,
+                     "peak_source": f"{peak_src} bf16 "
+                                    f"{'sustained' if long_step else 'burst'} (of {peak_src}; "
+                                    "the fp16 tensor rate equals bf16)",
+                     "frac_of_burst": attn_tflops / peak_burst, "peak_burst": peak_burst,
                      "traffic": ncu_traffic("prefill_attn_kernel<128>"),
                      "algorithmic_flops_per_launch": flops_step,
                      "kernel_ms": attn_ms_max / steps,
                      "kv_prep_ms": prep_ms_max / steps},
-        "decode": {
+        "cpu_baseline": cpu,
+        "gpu_launches": 2 * steps,
+        "clocks": clk,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": esteps,
+                "path": "api.HostPrefill: pinned host q/k/v in, pinned host o out"},
+        "other_workloads": _r(others, 4),
+        "prefill_16k": _r(prefill_16k, 5),
+        "decode": _r({
             "metric": "decode KV-read GB/s", "value": d_gbs, "unit": "GB/s", "steps": dsteps,
             "ms_per_step": dtotal_ms / dsteps, "workload": wd.name,
-            "config": {"B": wd.B, "Hq": wd.Hq, "Hkv": wd.Hkv, "d": wd.d, "T_max": wd.T,
-                       "cache_len": lens, "chunk_keys": 2048,
-                       "l2": "no flush: %.2f GB of K/V read per step > 126 MB L2" % (dbytes / 1e9)},
+            "cache_len": lens,
             "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<128,1> + merge",
                          "achieved": d_call_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": d_call_gbs / peaks["hbm_gbs"],
                          "peak_source": f"{peak_src} HBM copy",
                          "traffic": ncu_traffic("decode_split_kernel<128,1>"),
-                         "algorithmic_bytes_per_launch": dbytes,
-                         "timed_over": "the whole decode call (split + merge launches)"}},
-        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": esteps},
-        "other_workloads": others,
-        "cpu_baseline": cpu,
-        "gpu_launches": 2 * steps,
-        "clocks": clk,
+                         "algorithmic_bytes_per_launch": dbytes}}, 5),
     }
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
