@@ -66,13 +66,13 @@ def _load():
                                               c_double, c_double, c_int, dp, c_double,
                                               dp, dp, dp]
         lib.oracle_rope_theta_ext.restype = c_int
-        lib.oracle_rotate_rows.argtypes = [u16p, c_long, c_int, dp, dp, dp]
+        lib.oracle_rotate_rows.argtypes = [u16p, c_long, c_int, dp, dp, c_int, dp]
         lib.oracle_rotate_rows.restype = None
-        lib.oracle_rotate_rows_f64.argtypes = [dp, c_long, c_int, dp, dp, dp]
+        lib.oracle_rotate_rows_f64.argtypes = [dp, c_long, c_int, dp, dp, c_int, dp]
         lib.oracle_rotate_rows_f64.restype = None
         lib.oracle_attn_rows.argtypes = [u16p, u16p, u16p, c_int, c_int, c_int, c_int, c_int,
                                          dp, c_double, c_int, c_int, c_int, i64p, c_long,
-                                         dp, dp, dp, dp]
+                                         dp, dp, dp, dp, c_int]
         lib.oracle_attn_rows.restype = c_int
         lib.oracle_attn_rotated_f64.argtypes = [dp, dp, dp, c_int, c_int, c_int, c_int, c_int,
                                                 c_double, c_int, c_int, c_int, i64p, c_long,
@@ -80,11 +80,11 @@ def _load():
         lib.oracle_attn_rotated_f64.restype = c_int
         lib.oracle_decode.argtypes = [u16p, u16p, u16p, u16p, u16p, c_int, i32p,
                                       c_int, c_int, c_int, c_int, dp, c_double, c_int, c_int,
-                                      dp, dp, dp, dp, dp]
+                                      dp, dp, dp, dp, dp, c_int]
         lib.oracle_decode.restype = c_int
         lib.oracle_prefill_chunk.argtypes = [u16p, u16p, u16p, u16p, u16p, c_int, c_int,
                                              c_int, c_int, c_int, c_int, c_int, dp, c_double,
-                                             c_int, c_int, dp, dp, dp, dp]
+                                             c_int, c_int, dp, dp, dp, dp, c_int]
         lib.oracle_prefill_chunk.restype = c_int
         lib.oracle_alibi_slopes.argtypes = [c_int, dp]
         lib.oracle_alibi_slopes.restype = None
@@ -132,8 +132,16 @@ def rope_theta(d: int, base: float, L_train: int, s: float, method, alpha: float
     return th, ms.value, ss.value
 
 
-def rotate(x_bits, pos, theta) -> np.ndarray:
-    """Rotate rows of bf16 bits (shape [..., d]) at positions pos (broadcast to rows)."""
+PAIRS = {"interleaved": 0, "half": 1}
+
+
+def _pairs(pairs) -> int:
+    return PAIRS[pairs] if isinstance(pairs, str) else int(pairs)
+
+
+def rotate(x_bits, pos, theta, pairs="interleaved") -> np.ndarray:
+    """Rotate rows of bf16 bits (shape [..., d]) at positions pos (broadcast to rows).
+    pairs: "interleaved" (2i, 2i+1) or "half" (i, i + d/2)."""
     lib = _load()
     x = _bits(x_bits)
     d = x.shape[-1]
@@ -143,12 +151,12 @@ def rotate(x_bits, pos, theta) -> np.ndarray:
     th = np.ascontiguousarray(theta, dtype=np.float64)
     out = np.empty(rows.shape, dtype=np.float64)
     lib.oracle_rotate_rows(_ptr(rows, ctypes.c_uint16), rows.shape[0], d,
-                           _ptr(p, ctypes.c_double), _ptr(th, ctypes.c_double),
+                           _ptr(p, ctypes.c_double), _ptr(th, ctypes.c_double), _pairs(pairs),
                            _ptr(out, ctypes.c_double))
     return out.reshape(x.shape)
 
 
-def rotate_f64(x, pos, theta) -> np.ndarray:
+def rotate_f64(x, pos, theta, pairs="interleaved") -> np.ndarray:
     """Rotate float64 rows (shape [..., d]) at positions pos."""
     lib = _load()
     x = np.ascontiguousarray(x, dtype=np.float64)
@@ -160,7 +168,7 @@ def rotate_f64(x, pos, theta) -> np.ndarray:
     out = np.empty(rows.shape, dtype=np.float64)
     lib.oracle_rotate_rows_f64(_ptr(rows, ctypes.c_double), rows.shape[0], d,
                                _ptr(p, ctypes.c_double), _ptr(th, ctypes.c_double),
-                               _ptr(out, ctypes.c_double))
+                               _pairs(pairs), _ptr(out, ctypes.c_double))
     return out.reshape(x.shape)
 
 
@@ -181,7 +189,7 @@ def alibi_slopes(H: int) -> np.ndarray:
 
 
 def attn_rows(q_bits, k_bits, v_bits, theta, softmax_scale, causal=True, window=0, n_sink=0,
-              rows=None, want_qrot=False, slopes=None):
+              rows=None, want_qrot=False, slopes=None, pairs="interleaved"):
     """Exact attention for selected rows.
 
     q [B,Hq,T,d], k/v [B,Hkv,T,d] as bf16 bits.  rows: flat indices
@@ -213,7 +221,7 @@ def attn_rows(q_bits, k_bits, v_bits, theta, softmax_scale, causal=True, window=
                               int(window), int(n_sink), rp, n, _ptr(o, ctypes.c_double),
                               _ptr(lse, ctypes.c_double),
                               _ptr(qr, ctypes.c_double) if qr is not None
-                              else ctypes.POINTER(ctypes.c_double)(), sp)
+                              else ctypes.POINTER(ctypes.c_double)(), sp, _pairs(pairs))
     if rc != 0:
         raise ValueError(f"oracle_attn_rows failed ({rc})")
     return o, lse, qr
@@ -253,7 +261,7 @@ def attn_rotated_f64(q_rot, k_rot, v, softmax_scale, causal=True, window=0, n_si
 
 
 def decode(q_new, k_new, v_new, k_cache, v_cache, cache_len, theta, softmax_scale,
-           window=0, n_sink=0, slopes=None):
+           window=0, n_sink=0, slopes=None, pairs="interleaved"):
     """Exact single-token decode.  Returns (o [B,Hq,d], lse [B,Hq], k_rot_new [B,Hkv,d],
     q_rot_new [B,Hq,d])."""
     lib = _load()
@@ -275,14 +283,14 @@ def decode(q_new, k_new, v_new, k_cache, v_cache, cache_len, theta, softmax_scal
                            B, Hq, Hkv, d, _ptr(th, ctypes.c_double), float(softmax_scale),
                            int(window), int(n_sink), _ptr(o, ctypes.c_double),
                            _ptr(lse, ctypes.c_double), _ptr(kr, ctypes.c_double),
-                           _ptr(qr, ctypes.c_double), sp)
+                           _ptr(qr, ctypes.c_double), sp, _pairs(pairs))
     if rc != 0:
         raise ValueError(f"oracle_decode failed ({rc})")
     return o, lse, kr, qr
 
 
 def prefill_chunk(q, k_new, v_new, k_cache, v_cache, P0, theta, softmax_scale, window=0,
-                  n_sink=0, slopes=None):
+                  n_sink=0, slopes=None, pairs="interleaved"):
     """A chunk of Tq tokens at positions P0.. against a rotated cache prefix (slots < P0).
     q bf16 [B,Hq,Tq,d]; k_new, v_new bf16 [B,Hkv,Tq,d]; caches bf16 [B,Hkv,T_max,d].
     Returns (o [B,Hq,Tq,d], lse [B,Hq,Tq], k_rot_new [B,Hkv,Tq,d]) in float64."""
@@ -302,7 +310,8 @@ def prefill_chunk(q, k_new, v_new, k_cache, v_cache, P0, theta, softmax_scale, w
                                   _ptr(vc, ctypes.c_uint16), int(T_max), int(P0), B, Hq, Hkv,
                                   Tq, d, _ptr(th, ctypes.c_double), float(softmax_scale),
                                   int(window), int(n_sink), _ptr(o, ctypes.c_double),
-                                  _ptr(lse, ctypes.c_double), _ptr(kr, ctypes.c_double), sp)
+                                  _ptr(lse, ctypes.c_double), _ptr(kr, ctypes.c_double), sp,
+                                  _pairs(pairs))
     if rc != 0:
         raise ValueError(f"oracle_prefill_chunk failed ({rc})")
     return o, lse, kr

@@ -25,7 +25,9 @@
  *     printed code is garbled and is not followed.
  *   - The temperature multiplies the logits by (0.1 ln s + 1)^2 / sqrt(d)
  *     (equivalently mscale on both rotated q and k).
- *   - Pairs are interleaved (2i, 2i+1) as on the [P3] RoPE slide.
+ *   - Pairs are interleaved (2i, 2i+1) as on the [P3] RoPE slide; every
+ *     rotating function also takes the half-split layout (i, i + d/2), the
+ *     common alternative the pages do not print (a `pairs` argument, 1 = half).
  *   - Window: key n is visible to query m iff n <= m (causal) and
  *     (m - n < W or n < n_sink); positions are absolute.
  *   - GQA: query head h reads KV head floor(h / (Hq/Hkv)).
@@ -42,7 +44,11 @@
  *                       pinned by f = 1 (RoPE), f = s (PI) and f = theta /
  *                       theta'(YaRN) (YaRN's frequencies).
  *   oracle_rotate_rows  pinned (page's rotation matrix, complex-number
- *                       form, orthogonality, relative-position invariance).
+ *                       form, orthogonality, relative-position invariance);
+ *                       the half-split layout pinned by its own complex form
+ *                       (z_i = x_i + i x_{i+d/2}), by equality with the
+ *                       interleaved rotation of the permuted vector, and by
+ *                       relative-position invariance.
  *   oracle_attn_rows    pinned (library SDPA special case, closed-form
  *                       means, page's "4 + last 4096" sink count, T=1).
  *   oracle_attn_rotated_f64 pinned (equals oracle_attn_rows on its own
@@ -187,26 +193,33 @@ int oracle_rope_theta(int d, double base, int L_train, double s, int method,
 }
 
 /*
- * Rotate one d-vector x at (possibly fractional) position p:
- *   [y_2i  ]   [cos(p theta_i)  -sin(p theta_i)] [x_2i  ]
- *   [y_2i+1] = [sin(p theta_i)   cos(p theta_i)] [x_2i+1]
- * [P3] RoPE slide (R_m,i on pair (2i, 2i+1)); [P5] "Position enters attention".
+ * Rotate one d-vector x at (possibly fractional) position p.  Pair i turns by
+ * the angle p theta_i:
+ *   [y_a]   [cos(p theta_i)  -sin(p theta_i)] [x_a]
+ *   [y_b] = [sin(p theta_i)   cos(p theta_i)] [x_b]
+ * with (a, b) = (2i, 2i+1) for interleaved pairs (pairs = 0, [P3] RoPE slide:
+ * R_m,i on pair (2i, 2i+1); [P5] "Position enters attention"), or
+ * (a, b) = (i, i + d/2) for the half-split layout (pairs = 1: the first half of
+ * the vector holds the first element of every pair, the second half the second
+ * element; the same rotation, another assignment of elements to pairs).
  */
-static void rotate_vec(const double *x, double p, const double *theta, int d,
+static void rotate_vec(const double *x, double p, const double *theta, int d, int pairs,
                        double *y)
 {
     for (int i = 0; i < d / 2; ++i) {
         const double phi = p * theta[i];
         const double c = cos(phi), sn = sin(phi);
-        const double a = x[2 * i], b = x[2 * i + 1];
-        y[2 * i] = a * c - b * sn;
-        y[2 * i + 1] = a * sn + b * c;
+        const int ia = pairs ? i : 2 * i;
+        const int ib = pairs ? i + d / 2 : 2 * i + 1;
+        const double a = x[ia], b = x[ib];
+        y[ia] = a * c - b * sn;
+        y[ib] = a * sn + b * c;
     }
 }
 
 /* Rotate n rows of bf16 bits (row stride d) at positions pos[r]. */
 void oracle_rotate_rows(const uint16_t *x, long n, int d, const double *pos,
-                        const double *theta, double *out)
+                        const double *theta, int pairs, double *out)
 {
 #pragma omp parallel
     {
@@ -214,7 +227,7 @@ void oracle_rotate_rows(const uint16_t *x, long n, int d, const double *pos,
 #pragma omp for schedule(static)
         for (long r = 0; r < n; ++r) {
             for (int j = 0; j < d; ++j) tmp[j] = bf16_bits_to_double(x[r * d + j]);
-            rotate_vec(tmp, pos[r], theta, d, out + r * d);
+            rotate_vec(tmp, pos[r], theta, d, pairs, out + r * d);
         }
         free(tmp);
     }
@@ -222,9 +235,9 @@ void oracle_rotate_rows(const uint16_t *x, long n, int d, const double *pos,
 
 /* Same, for rows already in double precision. */
 void oracle_rotate_rows_f64(const double *x, long n, int d, const double *pos,
-                            const double *theta, double *out)
+                            const double *theta, int pairs, double *out)
 {
-    for (long r = 0; r < n; ++r) rotate_vec(x + r * d, pos[r], theta, d, out + r * d);
+    for (long r = 0; r < n; ++r) rotate_vec(x + r * d, pos[r], theta, d, pairs, out + r * d);
 }
 
 /*
@@ -269,7 +282,7 @@ int oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      const double *theta, double softmax_scale,
                      int causal, int window, int n_sink,
                      const int64_t *rows, long n_rows,
-                     double *o, double *lse, double *q_rot, const double *slopes)
+                     double *o, double *lse, double *q_rot, const double *slopes, int pairs)
 {
     if (B < 1 || Hq < 1 || Hkv < 1 || T < 1 || d < 2 || (d % 2) || (Hq % Hkv)) return -1;
     const int group = Hq / Hkv;
@@ -314,7 +327,7 @@ int oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
 #pragma omp for schedule(static)
             for (long n = 0; n < cnt; ++n) {
                 for (int j = 0; j < d; ++j) tmp[j] = bf16_bits_to_double(kb[n * d + j]);
-                rotate_vec(tmp, (double)n, theta, d, dst + n * d);
+                rotate_vec(tmp, (double)n, theta, d, pairs, dst + n * d);
             }
             free(tmp);
         }
@@ -334,7 +347,7 @@ int oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             const long kv = b * Hkv + h / group;
             const uint16_t *qrow = q + flat * d;
             for (int j = 0; j < d; ++j) qv[j] = bf16_bits_to_double(qrow[j]);
-            rotate_vec(qv, (double)m, theta, d, qr);
+            rotate_vec(qv, (double)m, theta, d, pairs, qr);
             if (q_rot) memcpy(q_rot + r * d, qr, sizeof(double) * (size_t)d);
             const long kmax = causal ? m + 1 : T;
             const double *kr = krot[kv];
@@ -455,7 +468,7 @@ int oracle_decode(const uint16_t *q_new, const uint16_t *k_new, const uint16_t *
                   const int32_t *cache_len, int B, int Hq, int Hkv, int d,
                   const double *theta, double softmax_scale, int window, int n_sink,
                   double *o, double *lse, double *k_rot_new, double *q_rot_new,
-                  const double *slopes)
+                  const double *slopes, int pairs)
 {
     if (B < 1 || Hq < 1 || Hkv < 1 || d < 2 || (d % 2) || (Hq % Hkv) || T_max < 1) return -1;
     for (int b = 0; b < B; ++b)
@@ -481,10 +494,10 @@ int oracle_decode(const uint16_t *q_new, const uint16_t *k_new, const uint16_t *
                 const int kv = h / group;
                 const long qi = (long)b * Hq + h, ki = (long)b * Hkv + kv;
                 for (int j = 0; j < d; ++j) x[j] = bf16_bits_to_double(q_new[qi * d + j]);
-                rotate_vec(x, (double)L, theta, d, qr);
+                rotate_vec(x, (double)L, theta, d, pairs, qr);
                 if (q_rot_new) memcpy(q_rot_new + qi * d, qr, sizeof(double) * (size_t)d);
                 for (int j = 0; j < d; ++j) x[j] = bf16_bits_to_double(k_new[ki * d + j]);
-                rotate_vec(x, (double)L, theta, d, kn);
+                rotate_vec(x, (double)L, theta, d, pairs, kn);
                 if (k_rot_new && (h % group) == 0) memcpy(k_rot_new + ki * d, kn, sizeof(double) * (size_t)d);
                 const uint16_t *kc = k_cache + ki * (long)T_max * d;
                 const uint16_t *vc = v_cache + ki * (long)T_max * d;
@@ -537,7 +550,8 @@ int oracle_prefill_chunk(const uint16_t *q, const uint16_t *k_new, const uint16_
                          const uint16_t *k_cache, const uint16_t *v_cache, int T_max, int P0,
                          int B, int Hq, int Hkv, int Tq, int d,
                          const double *theta, double softmax_scale, int window, int n_sink,
-                         double *o, double *lse, double *k_rot_new, const double *slopes)
+                         double *o, double *lse, double *k_rot_new, const double *slopes,
+                         int pairs)
 {
     if (B < 1 || Hq < 1 || Hkv < 1 || Tq < 1 || d < 2 || (d % 2) || (Hq % Hkv)) return -1;
     if (P0 < 0 || (long)P0 + Tq > (long)T_max) return -1;
@@ -554,7 +568,7 @@ int oracle_prefill_chunk(const uint16_t *q, const uint16_t *k_new, const uint16_
             for (long i = 0; i < Tq; ++i) {
                 const uint16_t *src = k_new + (kv * Tq + i) * d;
                 for (int j = 0; j < d; ++j) tmp[j] = bf16_bits_to_double(src[j]);
-                rotate_vec(tmp, (double)(P0 + i), theta, d, krot + (kv * Tq + i) * d);
+                rotate_vec(tmp, (double)(P0 + i), theta, d, pairs, krot + (kv * Tq + i) * d);
             }
         }
         free(tmp);
@@ -581,7 +595,7 @@ int oracle_prefill_chunk(const uint16_t *q, const uint16_t *k_new, const uint16_
                     const long kv = (long)b * Hkv + h / group;
                     const long qi = ((long)b * Hq + h) * Tq + i;
                     for (int j = 0; j < d; ++j) x[j] = bf16_bits_to_double(q[qi * d + j]);
-                    rotate_vec(x, (double)m, theta, d, qr);
+                    rotate_vec(x, (double)m, theta, d, pairs, qr);
                     const uint16_t *kc = k_cache + kv * (long)T_max * d;
                     const uint16_t *vc = v_cache + kv * (long)T_max * d;
                     const double *kn = krot + kv * (long)Tq * d;

@@ -270,6 +270,58 @@ def test_relative_position_property(method):
     assert np.max(np.abs(a - c)) > 1e-3
 
 
+# ------------------------------------------------- the half-split pair layout
+
+def complex_rotate_half(x: np.ndarray, pos, theta) -> np.ndarray:
+    """Half-split RoPE as complex multiplication: (x_i + i x_{i+d/2}) * exp(i pos theta_i)."""
+    h = x.shape[-1] // 2
+    z = x[..., :h] + 1j * x[..., h:]
+    pos = np.asarray(pos, dtype=np.float64)[..., None]
+    w = z * np.exp(1j * pos * theta)
+    return np.concatenate([w.real, w.imag], axis=-1)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_half_layout_matches_its_complex_form(d):
+    th, _, _ = oracle.rope_theta(d, 500000.0, 8192, 16.0, "yarn")
+    x = bf16_bits(RNG.standard_normal((48, d)))
+    pos = RNG.integers(0, 131073, size=48).astype(np.float64)
+    got = oracle.rotate(x, pos, th, pairs="half")
+    np.testing.assert_allclose(got, complex_rotate_half(bits_to_f64(x), pos, th), rtol=0,
+                               atol=1e-12)
+    # not the interleaved rotation (the two layouts pair different elements)
+    assert np.abs(got - oracle.rotate(x, pos, th)).max() > 1e-2
+
+
+def test_half_layout_is_the_interleaved_rotation_of_the_permuted_vector():
+    d = 128
+    th, _, _ = oracle.rope_theta(d, 10000.0, 4096, 4.0, "yarn")
+    x = RNG.standard_normal((16, d))
+    pos = RNG.integers(0, 70000, size=16).astype(np.float64)
+    perm = np.empty(d, dtype=np.int64)           # interleaved slot -> half-split element
+    perm[0::2] = np.arange(d // 2)
+    perm[1::2] = np.arange(d // 2) + d // 2
+    inter = oracle.rotate_f64(x[:, perm], pos, th)
+    half = oracle.rotate_f64(x, pos, th, pairs="half")
+    np.testing.assert_allclose(half[:, perm], inter, rtol=0, atol=1e-13)
+
+
+def test_half_layout_relative_position_and_norm():
+    th, _, _ = oracle.rope_theta(64, 10000.0, 64, 4.0, "yarn")
+    q = bf16_bits(RNG.standard_normal((20, 64)))
+    k = bf16_bits(RNG.standard_normal((20, 64)))
+    m = RNG.integers(0, 50000, size=20).astype(np.float64)
+    n = RNG.integers(0, 50000, size=20).astype(np.float64)
+    delta = RNG.integers(1, 80000, size=20).astype(np.float64)
+    rq = oracle.rotate(q, m, th, pairs="half")
+    a = np.sum(rq * oracle.rotate(k, n, th, pairs="half"), axis=1)
+    b = np.sum(oracle.rotate(q, m + delta, th, pairs="half") *
+               oracle.rotate(k, n + delta, th, pairs="half"), axis=1)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-9)
+    np.testing.assert_allclose(np.linalg.norm(rq, axis=1), np.linalg.norm(bits_to_f64(q), axis=1),
+                               rtol=1e-14)
+
+
 # ------------------------------------------------------------- the attention
 
 def _rand_qkv(B, Hq, Hkv, T, d):
@@ -360,6 +412,58 @@ def test_rotated_f64_zero_query_gives_prefix_means():
     cs = np.vstack([np.zeros((1, d)), np.cumsum(v[0, 0], axis=0)])
     o, _ = oracle.attn_rotated_f64(np.zeros((1, 1, T, d)), k, v, 0.3, True, 0, 0)
     np.testing.assert_allclose(o, cs[1:] / np.arange(1, T + 1)[:, None], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal,window,n_sink", [(True, 0, 0), (True, 9, 3)])
+def test_half_layout_attention_matches_library_sdpa(causal, window, n_sink):
+    B, Hq, Hkv, T, d = 1, 4, 2, 41, 16
+    th, _, ss = oracle.rope_theta(d, 10000.0, 16, 4.0, "yarn")
+    q, k, v = _rand_qkv(B, Hq, Hkv, T, d)
+    o, lse, qr_o = oracle.attn_rows(q, k, v, th, ss, causal, window, n_sink, want_qrot=True,
+                                    pairs="half")
+    pos = np.arange(T, dtype=np.float64)
+    qr = torch.from_numpy(complex_rotate_half(bits_to_f64(q), pos, th))
+    kr = torch.from_numpy(complex_rotate_half(bits_to_f64(k), pos, th))
+    np.testing.assert_allclose(qr_o.reshape(B, Hq, T, d), qr.numpy(), rtol=0, atol=1e-12)
+    g = Hq // Hkv
+    mask = torch.from_numpy(_mask(T, causal, window, n_sink))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        qr, kr.repeat_interleave(g, dim=1), torch.from_numpy(bits_to_f64(v)).repeat_interleave(g, dim=1),
+        attn_mask=mask, scale=ss)
+    np.testing.assert_allclose(o.reshape(B, Hq, T, d), ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_half_layout_decode_and_chunk_equal_the_prefill_rows():
+    B, Hq, Hkv, T, d = 1, 4, 2, 50, 16
+    th, _, ss = oracle.rope_theta(d, 10000.0, 16, 4.0, "yarn")
+    q, k, v = _rand_qkv(B, Hq, Hkv, T, d)
+    o, _, _ = oracle.attn_rows(q, k, v, th, ss, pairs="half")
+    o = o.reshape(B, Hq, T, d)
+    # a cache holding the half-split rotation of keys 0..L-1, then the token at L
+    pos = np.broadcast_to(np.arange(T, dtype=np.float64), (B, Hkv, T)).reshape(-1)
+    kc = bf16_bits(oracle.rotate(k, pos, th, pairs="half").reshape(B, Hkv, T, d))
+    L = 37
+    od, _, _, _ = oracle.decode(q[:, :, L], k[:, :, L], v[:, :, L], kc, v, np.array([L]), th, ss,
+                                pairs="half")
+    # brute force: the query and the new key rotated at L in the half layout (complex form),
+    # the cached keys as given
+    g = Hq // Hkv
+    for h in range(Hq):
+        qv = complex_rotate_half(bits_to_f64(q[0, h, L]), L, th)
+        keys = np.vstack([bits_to_f64(kc[0, h // g, :L]),
+                          complex_rotate_half(bits_to_f64(k[0, h // g, L]), L, th)[None]])
+        sc = ss * keys @ qv
+        p_ = np.exp(sc - sc.max())
+        want = (p_ / p_.sum()) @ bits_to_f64(v[0, h // g, :L + 1])
+        np.testing.assert_allclose(od[0, h], want, rtol=0, atol=1e-12)
+    # and close to the exact prefill row (the cached keys went through bf16)
+    np.testing.assert_allclose(od, o[:, :, L], rtol=0, atol=5e-2)
+    oc, _, kr = oracle.prefill_chunk(q[:, :, L:], k[:, :, L:], v[:, :, L:], kc, v, L, th, ss,
+                                     pairs="half")
+    np.testing.assert_allclose(oc[:, :, 0], od, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(kr.reshape(-1, d),
+                               oracle.rotate(k[:, :, L:], pos.reshape(B, Hkv, T)[:, :, L:].reshape(-1),
+                                             th, pairs="half").reshape(-1, d), rtol=0, atol=1e-13)
 
 
 def test_rows_sum_to_one_through_v_ones():
