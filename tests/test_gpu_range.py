@@ -103,7 +103,9 @@ def test_peaked_softmax_matches_exact_attention_of_the_rounded_operands(cq, wind
     err = np.abs(got - ro)
     assert np.all(err <= O_MAX_ABS + np.abs(ro) * 2.0 ** -8), float(err.max())
     assert err.mean() <= O_MEAN_ABS + np.abs(ro).mean() * 2.0 ** -9, float(err.mean())
-    assert err_stats(lse.reshape(-1), rl)[0] <= LSE_ABS
+    # a rotated operand the kernel computes in fp32 can land one fp16 step away from the
+    # oracle's fp64 rotation rounded to fp16: a logit moves by up to 2^-11 of its size
+    assert np.all(np.abs(lse.reshape(-1) - rl) <= LSE_ABS + np.abs(rl) * 2.0 ** -11)
     # against exact attention of the unrounded inputs: the logit shifts of fp16 storage
     # are the only difference, a few hundredths at most here
     ex, _, _ = oracle.attn_rows(qb, kb, vb, th, ss, True, window, n_sink)

@@ -612,15 +612,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                               : !(l_tile <= kPBound);
             if (fresh && !over) m_run = 0.0f;
             if (__any_sync(0xffffffffu, over)) {
-                // Tile max in four independent chains of three-input max.
+                // Tile max in four independent chains of three-input max: s[0..3] start
+                // the chains, s[4..123] go eight per step, s[124..127] close them.
+                static_assert(kBlockN % 8 == 0, "tile max covers the tile in steps of 8");
                 float m4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-                for (int c = 4; c < kBlockN; c += 8) {
+                for (int c = 4; c + 8 <= kBlockN - 4; c += 8) {
                     m4[0] = fmax3(m4[0], s[c], s[c + 1]);
                     m4[1] = fmax3(m4[1], s[c + 2], s[c + 3]);
                     m4[2] = fmax3(m4[2], s[c + 4], s[c + 5]);
                     m4[3] = fmax3(m4[3], s[c + 6], s[c + 7]);
                 }
+                m4[0] = fmax3(m4[0], s[kBlockN - 4], s[kBlockN - 3]);
+                m4[1] = fmax3(m4[1], s[kBlockN - 2], s[kBlockN - 1]);
                 const float m_tile = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * sl2;
                 const bool first = m_run == -INFINITY;
                 const bool move = first || (over && m_tile > m_run);
