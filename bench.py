@@ -392,6 +392,40 @@ def chunk_bench(w, steps, stream, dist, peak_t):
             "timed_over": "the whole call (prefix/chunk layout + attention launches)"}
 
 
+def chunk_fp16cache_bench(w, Tq, steps, stream, dist, peak_t):
+    """A short chunk after a long cached prefix, the serving loop's steady state: the fp16
+    copy of the cache already holds the prefix, so a call writes only its own Tq rows,
+    cuts each query block's keys into shares (split-KV) and merges them.  The whole
+    yr_attn_prefill_chunk_fp16cache call, as causal TFLOP/s."""
+    from yarn_position_scaling_b200 import api
+    q, kn, vn, kc, vc = synth.chunk_inputs(w, "cuda", Tq=Tq, T_max=w.P0 + Tq)
+    tab = api.rope_freq_table(w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta)
+    k16, v16 = kc.to(torch.float16), vc.to(torch.float16)
+    ws = torch.empty(api.attn_prefill_chunk_split_bytes(w.B, w.Hq, Tq, w.d), dtype=torch.uint8,
+                     device="cuda")
+    o = torch.empty_like(q)
+
+    def step(_):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e[0].record(stream)
+        api.attn_prefill_chunk_fp16cache(q, kn, vn, kc, vc, k16, v16, w.P0, w.P0, tab, out=o,
+                                         workspace=ws, stream=stream)
+        e[1].record(stream)
+        return [(e[0], e[1])]
+
+    for i in range(3):
+        step(i)
+    api.device_status(stream)
+    dist.barrier()
+    total_ms, (call_ms,) = time_events(step, steps, stream)
+    dist.barrier()
+    api.device_status(stream)
+    call_ms = dist.max(call_ms)
+    flops = metrics.chunk_flops(w.B, w.Hq, w.d, w.P0, Tq)
+    tf = flops / (call_ms / steps * 1e-3) / 1e12
+    return {"tflops": tf, "frac": tf / peak_t, "ms": call_ms / steps}
+
+
 def ring_bench(w, world, steps, stream, dist, peak_t):
     """Ring attention over `world` ranks emulated in one process on this GPU: every rank's
     block kernels (keys prepared at their positions, one attention call per visible
@@ -519,7 +553,10 @@ def main():
     others = {}
     if not args.no_other_workloads:
         for w in synth.SWEEP:
-            r = workload_prefill(w, args.other_steps, stream, dist, peak_burst)
+            # at least ~0.1 s of work per variant (the windowed ones take ~4 ms a launch)
+            flops_w = metrics.prefill_flops(w.B, w.Hq, w.T, w.d, w.causal, w.window, w.n_sink)
+            r = workload_prefill(w, max(args.other_steps, int(1e14 / flops_w)), stream, dist,
+                                 peak_burst)
             others[w.name.replace("sweep_", "")] = {
                 "tflops": r["attn_kernel_tflops"], "step_tflops": r["step_tflops"],
                 "frac": r["frac_of_peak"]}
@@ -527,6 +564,9 @@ def main():
         r = chunk_bench(synth.CHUNK, args.other_steps, stream, dist, peak_burst)
         others["chunk_124k_plus_4k"] = {"tflops": r["call_tflops"], "frac": r["frac_of_peak"],
                                         "ms": r["call_ms"]}
+        torch.cuda.empty_cache()
+        others["chunk_124k_plus_256_fp16cache"] = chunk_fp16cache_bench(
+            synth.CHUNK, 256, max(args.other_steps, 10), stream, dist, peak_burst)
         torch.cuda.empty_cache()
         wr = synth.LLAMA3_128K
         r = ring_bench(wr, 8, args.other_steps, stream, dist, peak_burst)

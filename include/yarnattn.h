@@ -60,6 +60,14 @@ extern "C" {
 
 #define YR_MAX_HEAD_DIM 128
 
+/* Which elements of a head vector form the rotated pairs.  The pages print the
+ * interleaved form ("Arch_03_Long_Context", RoPE slide: pair (2i, 2i+1)); the
+ * half-split form (i, i + d/2), in which the first half of the vector holds the
+ * first element of every pair, is the common alternative layout of the same
+ * rotation.  Pair i turns by position * theta'_i in both. */
+#define YR_PAIR_INTERLEAVED 0
+#define YR_PAIR_HALF 1
+
 /* Method parameters, named after the pages' rope_scaling config (type, factor,
  * original_max_position_embeddings) and the problem statement. */
 typedef struct yr_rope_params {
@@ -73,6 +81,7 @@ typedef struct yr_rope_params {
     int L_cur;      /* YR_NTK_DYNAMIC: current sequence length (>= 1); else unused */
     const double *factors; /* YR_FACTORS: d/2 host doubles f_i > 0, read during the call */
     double attn_factor;    /* YR_FACTORS: mscale (attention temperature); <= 0 means 1 */
+    int pairs;             /* YR_PAIR_INTERLEAVED (0, default) or YR_PAIR_HALF */
 } yr_rope_params;
 
 /* Frequency and temperature table, built on the host in double precision and
@@ -86,6 +95,8 @@ typedef struct yr_rope_table {
                                              factor for YR_FACTORS, else 1 */
     double softmax_scale;                 /* mscale^2 / sqrt(d): the logit multiplier */
     uint64_t digest;                      /* FNV-1a of the parameters (position-config identity) */
+    int pairs;                            /* YR_PAIR_INTERLEAVED or YR_PAIR_HALF: every kernel
+                                             that rotates follows it */
 } yr_rope_table;
 
 /*
@@ -105,19 +116,25 @@ typedef struct yr_rope_table {
  *   "Long context (engineering 100k+ tokens)" and "long-context-models").
  *   ALiBi: every theta'_i = 0 (no rotation), mscale = 1; the attention entry
  *   points add the per-head linear bias when they see this method.
+ *   pairs: copied into the table; the kernels rotate pairs (2i, 2i+1) or
+ *   (i, i + d/2) accordingly (the q/k debug outputs and the rotated-key cache
+ *   keep the caller's element order).
  *   The digest hashes the parameters, so a server can fold the position policy
  *   into its engine identity ("long-context-models", operational failure modes).
  * Errors: YR_EINVAL for NULL pointers, odd/out-of-range head_dim, base <= 1,
  *   scale < 1, unknown method, for either YaRN form L_train < 1 or beta <=
- *   alpha, for dynamic NTK L_train < 1 or L_cur < 1, and for YR_FACTORS a NULL
- *   factors pointer or a factor that is not a positive finite number.
+ *   alpha, for dynamic NTK L_train < 1 or L_cur < 1, for YR_FACTORS a NULL
+ *   factors pointer or a factor that is not a positive finite number, and for a
+ *   pairs value other than YR_PAIR_INTERLEAVED or YR_PAIR_HALF.
  */
 int yr_rope_freq_table(const yr_rope_params *p, yr_rope_table *out);
 
 /*
  * attn_prefill_workspace_bytes -- bytes of device workspace yr_attn_prefill
- * needs: the rotated keys and the values, each [B, Hkv, T, d] in fp16.
- * Returns 0 for invalid sizes.
+ * needs: the rotated keys and the values, each [B, Hkv, T, d] in fp16, then 256
+ * bytes for the work counter of the persistent attention grid (one CTA per SM,
+ * each taking the next 256-row query block of a (batch, head) from the counter,
+ * heaviest first).  Returns 0 for invalid sizes.
  */
 size_t yr_attn_prefill_workspace_bytes(int B, int Hkv, int T, int d);
 
@@ -223,6 +240,45 @@ int yr_attn_prefill_chunk(const void *q, const void *k_new, const void *v_new,
                           void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * attn_prefill_chunk_fp16cache -- yr_attn_prefill_chunk for a serving loop that
+ * keeps, next to the bf16 cache, a second copy of it in the fp16 operand format
+ * of the attention kernel, so that a call moves only its own Tq rows instead of
+ * converting the whole cached prefix into a workspace ("Long context (engineering
+ * 100k+ tokens)", sec. 6: prefix caching, chunked prefill).
+ *   k_cache16, v_cache16: fp16 [B, Hkv, T_max, d], contiguous, 256-byte aligned,
+ *     caller-owned.  Slots 0 .. cache16_len-1 must hold fp16 copies of the keys
+ *     and values of those slots, as an earlier call of this function left them;
+ *     the call converts slots cache16_len .. P0-1 from the bf16 caches, then
+ *     writes the chunk's rotated keys and values into slots P0 .. P0+Tq-1 of both
+ *     copies.  The keys it appends are their fp32 rotation rounded once to fp16
+ *     in the copy and to bf16 in the cache (the precision yr_attn_prefill_chunk
+ *     attends them with), so later chunks read them at fp16 precision.
+ *     Afterwards slots 0 .. P0+Tq-1 of the fp16 copy are valid, so the next chunk
+ *     passes cache16_len = P0 + Tq.  Slots a decode step appended to the bf16
+ *     cache in between are picked up by passing the last valid length.
+ *   0 <= cache16_len <= P0.
+ *   workspace (nullable, 256-byte aligned): 256 bytes for the persistent grid's
+ *     work counter (without it, one CTA per query block), then room for split-KV
+ *     partials.  A short
+ *     chunk after a long prefix has few (sequence, head, 256-row query block)
+ *     items -- 32 for one 256-token chunk of a 32-head model -- too few for the
+ *     GPU's SMs; with a workspace the call cuts each item's keys into up to 16
+ *     shares run as separate CTAs, each leaving an fp32 partial output and its
+ *     log-sum-exp, and merges them (the online-softmax combination of partial
+ *     results, as in ring attention).  yr_attn_prefill_chunk_split_bytes() gives
+ *     the bytes for the most shares; a smaller workspace limits the shares, NULL
+ *     means none.  The result differs from the unsplit one only by fp32 rounding.
+ *   Other arguments, results and errors as yr_attn_prefill_chunk.
+ */
+size_t yr_attn_prefill_chunk_split_bytes(int B, int Hq, int Tq, int d);
+int yr_attn_prefill_chunk_fp16cache(const void *q, const void *k_new, const void *v_new,
+                                    void *k_cache, void *v_cache, void *k_cache16,
+                                    void *v_cache16, int cache16_len, void *o, float *lse,
+                                    int B, int Hq, int Hkv, int Tq, int d, int P0, int T_max,
+                                    const yr_rope_table *tab, int window, int n_sink,
+                                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * prefill_prepare_kv_at -- yr_prefill_prepare_kv for a block of keys that starts at
  * absolute position k_pos0 (key t is rotated at k_pos0 + t): the step a worker of
  * ring attention / context parallelism ("long-context-models", section "Context
@@ -282,6 +338,44 @@ int yr_prefill_attend_block(const void *q, float *o, float *lse,
  */
 int yr_attn_merge(const float *o_part, const float *lse_part, float *o_acc, float *lse_acc,
                   void *o_out, long long rows, int d, int init, void *stream);
+
+/*
+ * host_prefill -- prefill of prompts that live in host memory: q, k, v are read
+ * from host buffers and o is written to a host buffer, with the copies inside the
+ * call ("LLM context window mechanics", production lessons: a 128K prompt's first
+ * request pays its whole prefill).  The work is cut into units of (sequence, group
+ * of KV heads with their query heads); each unit's host-to-device copy, its
+ * yr_attn_prefill (on `stream`) and its device-to-host copy run on three streams,
+ * so the transfers of some units overlap the kernels of others, and a call's first
+ * units overlap the previous call's last ones.
+ *   A plan is made once per shape and reused:
+ *   yr_host_prefill_workspace_bytes(B, Hq, Hkv, T, d, units_per_batch) -- device
+ *     bytes the plan needs (q, k, v, o on the device plus a unit's prefill
+ *     workspace); 0 for invalid sizes.  units_per_batch <= 0 means min(Hkv, 8).
+ *   yr_host_prefill_create(&plan, B, Hq, Hkv, T, d, units_per_batch, workspace,
+ *     workspace_bytes) -- workspace: caller-owned device memory of at least that
+ *     many bytes, 256-byte aligned, kept for the plan's life.  The plan creates two
+ *     streams and three events per unit on the current device (no device memory).
+ *   yr_host_prefill_run(plan, q, k, v, o, tab, causal, window, n_sink, stream) --
+ *     q, o: host [B, Hq, T, d] bf16; k, v: host [B, Hkv, T, d] bf16; contiguous.
+ *     Page-locked (pinned) host memory lets the copies run asynchronously; with
+ *     pageable memory they still work but do not overlap.  Asynchronous: work on
+ *     `stream` after the call waits for the whole result; synchronise `stream`
+ *     before reading o or changing q, k, v.  Other arguments and errors as
+ *     yr_attn_prefill; YR_EINVAL also when called on another device than the
+ *     plan's.  One host thread at a time per plan.
+ *   yr_host_prefill_destroy(plan) -- waits for the plan's copies, frees its streams
+ *     and events (NULL is accepted).
+ */
+typedef struct yr_host_prefill yr_host_prefill;
+size_t yr_host_prefill_workspace_bytes(int B, int Hq, int Hkv, int T, int d,
+                                       int units_per_batch);
+int yr_host_prefill_create(yr_host_prefill **plan, int B, int Hq, int Hkv, int T, int d,
+                           int units_per_batch, void *workspace, size_t workspace_bytes);
+int yr_host_prefill_run(yr_host_prefill *plan, const void *q, const void *k, const void *v,
+                        void *o, const yr_rope_table *tab, int causal, int window, int n_sink,
+                        void *stream);
+int yr_host_prefill_destroy(yr_host_prefill *plan);
 
 /*
  * attn_decode_workspace_bytes -- bytes of device workspace yr_attn_decode needs

@@ -179,9 +179,46 @@ def test_decode_rejects_bad_arguments_on_host(lib, kw, code):
 
 
 def test_workspace_sizes(lib):
-    assert api.attn_prefill_workspace_bytes(1, 8, 131072, 128) == 2 * 8 * 131072 * 128 * 2
+    # rotated keys and values in fp16, then 256 bytes for the persistent grid's work counter
+    assert api.attn_prefill_workspace_bytes(1, 8, 131072, 128) == 2 * 8 * 131072 * 128 * 2 + 256
+    # the chunk's split-KV workspace: the counter, then up to 16 shares of fp32 o and lse
+    assert api.attn_prefill_chunk_split_bytes(1, 32, 256, 128) == 256 + 16 * 32 * 256 * 129 * 4
     # one partial slot per block of the balanced split that can hold part of a segment:
     # blocks hold at least 2048 keys, so a segment of T_max keys touches ceil(T_max/2048)+1
     parts = (131073 + 2047) // 2048 + 1
     assert api.attn_decode_workspace_bytes(8, 32, 8, 128, 131073) == 8 * 8 * parts * 4 * 130 * 4
     assert api.attn_decode_workspace_bytes(8, 30, 8, 128, 100) == 0
+
+
+def test_table_rejects_unknown_pair_layout(lib):
+    with pytest.raises(api.YarnAttnError):
+        api.rope_freq_table(128, 1e4, 4096, 4.0, "yarn", pairs=2)
+    t_int = api.rope_freq_table(128, 1e4, 4096, 4.0, "yarn")
+    t_half = api.rope_freq_table(128, 1e4, 4096, 4.0, "yarn", pairs="half")
+    assert t_int.digest != t_half.digest
+    assert list(t_int.inv_freq) == list(t_half.inv_freq)
+
+
+def test_host_prefill_plan_checks_arguments_before_any_cuda_call(lib):
+    # sizes: q and o [B,Hq,T,d], k and v [B,Hkv,T,d] bf16, each rounded up to 256 bytes,
+    # plus one unit's prefill workspace (rotated keys and values of its KV heads, fp16, and
+    # the work counter)
+    B, Hq, Hkv, T, d = 2, 4, 2, 16, 64
+    r = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    want = 2 * r(B * Hq * T * d * 2) + 2 * r(B * Hkv * T * d * 2) + r(4 * 1 * T * d + 256)
+    assert lib.yr_host_prefill_workspace_bytes(B, Hq, Hkv, T, d, 2) == want  # 1 KV head a unit
+    assert lib.yr_host_prefill_workspace_bytes(1, 3, 2, 16, 64, 0) == 0      # Hq % Hkv
+    assert lib.yr_host_prefill_workspace_bytes(1, 4, 2, 16, 96, 0) == 0      # head size
+    plan = ctypes.c_void_p()
+    n = want
+    assert lib.yr_host_prefill_create(ctypes.byref(plan), B, Hq, Hkv, T, d, 2, None, n) == \
+        api.YR_EINVAL
+    assert lib.yr_host_prefill_create(ctypes.byref(plan), B, Hq, Hkv, T, d, 2,
+                                      ctypes.c_void_p(4096), n - 1) == api.YR_EINVAL
+    assert "too small" in lib.yr_last_error().decode()
+    assert lib.yr_host_prefill_create(ctypes.byref(plan), B, Hq, Hkv, T, d, 2,
+                                      ctypes.c_void_p(4096 + 16), n) == api.YR_EINVAL
+    assert "aligned" in lib.yr_last_error().decode()
+    assert lib.yr_host_prefill_run(None, None, None, None, None, None, 1, 0, 0, None) == \
+        api.YR_EINVAL
+    assert lib.yr_host_prefill_destroy(None) == api.YR_OK

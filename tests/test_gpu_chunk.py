@@ -128,3 +128,124 @@ def test_chunk_alibi():
     assert emax <= O_MAX_ABS and emean <= O_MEAN_ABS, (emax, emean)
     # no rotation: the appended keys are the new keys as given
     assert torch.equal(kc[:, :, P0:P0 + Tq], kn)
+
+
+# ------------------------------------------------- chunks with a kept fp16 cache copy
+
+def test_fp16cache_matches_the_workspace_form_bit_for_bit():
+    w = SMALL
+    P0, Tq, T_max = 777, 513, 1400
+    q, kn, vn, kc, vc = synth.chunk_inputs(w, "cuda", P0=P0, Tq=Tq, T_max=T_max)
+    tab, _, _ = _tables(w)
+    kc2, vc2 = kc.clone(), vc.clone()
+    lse1 = torch.empty(q.shape[:3], device="cuda")
+    lse2 = torch.empty(q.shape[:3], device="cuda")
+    ref = api.attn_prefill_chunk(q, kn, vn, kc, vc, P0, tab, 300, 4, lse=lse1)
+    k16 = torch.full(kc.shape, float("nan"), dtype=torch.float16, device="cuda")
+    v16 = torch.full(vc.shape, float("nan"), dtype=torch.float16, device="cuda")
+    got = api.attn_prefill_chunk_fp16cache(q, kn, vn, kc2, vc2, k16, v16, 0, P0, tab, 300, 4,
+                                           lse=lse2)
+    api.device_status()
+    assert torch.equal(got, ref) and torch.equal(lse2, lse1)
+    assert torch.equal(kc2, kc) and torch.equal(vc2, vc)
+    # the converted prefix is the fp16 value of the bf16 cache; the chunk's keys are its fp32
+    # rotation rounded once to fp16 (the bf16 cache holds the same rotation rounded to bf16);
+    # values are copied; slots past the chunk are untouched
+    assert torch.equal(k16[:, :, :P0], kc[:, :, :P0].to(torch.float16))
+    _same_rotation(k16[:, :, P0:P0 + Tq], kc[:, :, P0:P0 + Tq])
+    assert torch.equal(v16[:, :, :P0 + Tq], vc[:, :, :P0 + Tq].to(torch.float16))
+    assert torch.isnan(k16[:, :, P0 + Tq:]).all() and torch.isnan(v16[:, :, P0 + Tq:]).all()
+
+
+def _same_rotation(k16, kbf16):
+    """An fp16 and a bf16 rounding of the same fp32 rotated keys: within one bf16 rounding."""
+    a, b = k16.float(), kbf16.float()
+    assert torch.all((a - b).abs() <= b.abs() * 2.0 ** -8 + 1e-6)
+
+
+def test_fp16cache_chunk_sequence_against_the_oracle():
+    # a prompt fed in chunks of 300, 257, 1 and 700 tokens; each call converts only what
+    # the copy lacks (nothing after the first), and two decode-appended slots are picked
+    # up by passing the last valid length
+    w = SMALL
+    T_max = 1400
+    tab, th, ss = _tables(w)
+    _, _, _, kc, vc = synth.chunk_inputs(w, "cuda", P0=0, Tq=1, T_max=T_max)
+    k16 = torch.zeros(kc.shape, dtype=torch.float16, device="cuda")
+    v16 = torch.zeros(vc.shape, dtype=torch.float16, device="cuda")
+    P0, valid = 0, 0
+    for i, Tq in enumerate([300, 257, 1, 700]):
+        if i == 3:
+            P0 += 2      # two slots appended to the bf16 cache by someone else
+        qq, kn, vn, _, _ = synth.chunk_inputs(dataclasses.replace(w, seed=w.seed + 10 + i),
+                                              "cuda", P0=P0, Tq=Tq, T_max=T_max)
+        kc0, vc0 = to_bits(kc), to_bits(vc)
+        o = api.attn_prefill_chunk_fp16cache(qq, kn, vn, kc, vc, k16, v16, valid, P0, tab,
+                                             256, 4)
+        api.device_status()
+        ro, _, _ = oracle.prefill_chunk(to_bits(qq), to_bits(kn), to_bits(vn), kc0, vc0, P0, th,
+                                        ss, 256, 4)
+        emax, emean = err_stats(to_f64(o), ro)
+        assert emax <= O_MAX_ABS and emean <= O_MEAN_ABS, (i, emax, emean)
+        _same_rotation(k16[:, :, P0:P0 + Tq], kc[:, :, P0:P0 + Tq])
+        P0 += Tq
+        valid = P0
+        assert torch.equal(v16[:, :, :P0], vc[:, :, :P0].to(torch.float16))
+
+
+def test_fp16cache_small_chunk_after_a_long_prefix():
+    # 256 new tokens after a 124K prefix that is already in the fp16 copy: only the
+    # chunk's rows are written; sampled rows against the oracle
+    w = dataclasses.replace(synth.CHUNK, Hq=8, Hkv=2)
+    P0, Tq = w.P0, 256
+    q, kn, vn, kc, vc = synth.chunk_inputs(w, "cuda", P0=P0, Tq=Tq, T_max=P0 + Tq)
+    kc0, vc0 = to_bits(kc), to_bits(vc)
+    k16, v16 = kc.to(torch.float16), vc.to(torch.float16)
+    tab, th, ss = _tables(w)
+    o = api.attn_prefill_chunk_fp16cache(q, kn, vn, kc, vc, k16, v16, P0, P0, tab)
+    api.device_status()
+    ro, _, _ = oracle.prefill_chunk(to_bits(q), to_bits(kn), to_bits(vn), kc0, vc0, P0, th, ss)
+    emax, emean = err_stats(to_f64(o), ro)
+    assert emax <= O_MAX_ABS and emean <= O_MEAN_ABS, (emax, emean)
+
+
+def test_fp16cache_rejects_bad_arguments():
+    w = SMALL
+    q, kn, vn, kc, vc = synth.chunk_inputs(w, "cuda", P0=10, Tq=20, T_max=40)
+    tab, _, _ = _tables(w)
+    k16 = torch.zeros(kc.shape, dtype=torch.float16, device="cuda")
+    v16 = torch.zeros(vc.shape, dtype=torch.float16, device="cuda")
+    with pytest.raises(api.YarnAttnError) as ei:
+        api.attn_prefill_chunk_fp16cache(q, kn, vn, kc, vc, k16, v16, 11, 10, tab)
+    assert ei.value.code == api.YR_EINVAL and "cache16_len" in str(ei.value)
+    with pytest.raises(api.YarnAttnError):
+        api.attn_prefill_chunk_fp16cache(q, kn, vn, kc, vc, k16, v16, 0, 25, tab)  # > T_max
+    api.device_status()
+
+
+@pytest.mark.parametrize("P0,Tq,window,n_sink", [(5000, 100, 0, 0), (3000, 64, 1000, 4),
+                                                 (2000, 300, 0, 0)])
+def test_fp16cache_split_kv_against_the_oracle_and_unsplit(P0, Tq, window, n_sink):
+    # few query blocks against a long prefix: the keys are cut into shares (split-KV)
+    w = SMALL
+    T_max = P0 + Tq
+    q, kn, vn, kc, vc = synth.chunk_inputs(w, "cuda", P0=P0, Tq=Tq, T_max=T_max)
+    kc0, vc0 = to_bits(kc), to_bits(vc)
+    tab, th, ss = _tables(w)
+    k16, v16 = kc.to(torch.float16), vc.to(torch.float16)
+    kc2, vc2, k16b, v16b = kc.clone(), vc.clone(), k16.clone(), v16.clone()
+    lse = torch.empty(q.shape[:3], device="cuda")
+    o = api.attn_prefill_chunk_fp16cache(q, kn, vn, kc, vc, k16, v16, P0, P0, tab, window,
+                                         n_sink, lse=lse)
+    o1 = api.attn_prefill_chunk_fp16cache(q, kn, vn, kc2, vc2, k16b, v16b, P0, P0, tab, window,
+                                          n_sink, split=False)
+    api.device_status()
+    ro, rl, _ = oracle.prefill_chunk(to_bits(q), to_bits(kn), to_bits(vn), kc0, vc0, P0, th, ss,
+                                     window, n_sink)
+    emax, emean = err_stats(to_f64(o), ro)
+    assert emax <= O_MAX_ABS and emean <= O_MEAN_ABS, (emax, emean)
+    assert err_stats(to_f64(lse), rl)[0] <= LSE_ABS
+    # the same operands, merged in another order: within one bf16 rounding of each other
+    a, b = o.float(), o1.float()
+    assert torch.all((a - b).abs() <= b.abs() * 2.0 ** -8 + 2e-3)
+    assert torch.equal(kc, kc2) and torch.equal(k16, k16b)

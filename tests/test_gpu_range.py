@@ -4,7 +4,7 @@ The prefill kernels hand the rotated queries and keys, the values and the
 probabilities to the tensor cores as fp16 (11-bit significand, largest finite
 value 65504).  Three things are checked here against the fp64 oracle:
 
-* Peaked softmax (queries scaled by 8 and 30 with the 128K workload's YaRN table)
+* Peaked softmax (queries scaled by 8, 16 and 30 with the 128K workload's YaRN table)
   drives the online softmax through its tile-max and rescale path and makes a
   fresh row reject its trial reference of 0.  fp16 storage of a rotated operand
   moves a logit by up to ~2^-11 of its size, so with logits of tens of units the
@@ -87,9 +87,16 @@ def _run_gpu(q, k, v, tab, window=0, n_sink=0):
     return to_f64(o), to_f64(lse), to_f64(qrot)
 
 
-@pytest.mark.parametrize("cq", [8.0, 30.0])
+@pytest.mark.parametrize("cq,flip", [(8.0, 0.0), (16.0, 0.0), (30.0, 1e-2)])
 @pytest.mark.parametrize("window,n_sink", [(0, 0), (200, 4)])
-def test_peaked_softmax_matches_exact_attention_of_the_rounded_operands(cq, window, n_sink):
+def test_peaked_softmax_matches_exact_attention_of_the_rounded_operands(cq, flip, window,
+                                                                        n_sink):
+    # `flip`: the kernel rotates in fp32 (angle within ~3e-7 turns), the oracle in fp64;
+    # an element whose exact value lies that close to the midpoint between two fp16 values
+    # rounds to the other neighbour on the GPU.  At |q~| up to ~135 (x30) one such flip
+    # moves a logit by up to ss * 2^-4 * |k~_i| ~ 0.01, and in a row where two keys nearly
+    # tie that moves o by up to ~0.01 more; below 2^6 (x8, x16) the effect is within the
+    # stated tolerance already.
     w, T = W128K, 700
     q, k, v = _scaled_inputs(w, T, cq=cq)
     o, lse, qrot = _run_gpu(q, k, v, _table(w), window, n_sink)
@@ -101,7 +108,7 @@ def test_peaked_softmax_matches_exact_attention_of_the_rounded_operands(cq, wind
                                      n_sink)
     got = o.reshape(ro.shape)
     err = np.abs(got - ro)
-    assert np.all(err <= O_MAX_ABS + np.abs(ro) * 2.0 ** -8), float(err.max())
+    assert np.all(err <= O_MAX_ABS + flip + np.abs(ro) * 2.0 ** -8), float(err.max())
     assert err.mean() <= O_MEAN_ABS + np.abs(ro).mean() * 2.0 ** -9, float(err.mean())
     # a rotated operand the kernel computes in fp32 can land one fp16 step away from the
     # oracle's fp64 rotation rounded to fp16: a logit moves by up to 2^-11 of its size

@@ -17,13 +17,18 @@ from .build import LIB
 YR_OK, YR_EINVAL, YR_EUNSUPPORTED, YR_ECUDA, YR_ETIMEOUT, YR_ERANGE = 0, -1, -2, -3, -4, -5
 ROPE, PI, NTK, YARN = 0, 1, 2, 3
 NTK_DYNAMIC, YARN_DIMRAMP, FACTORS, ALIBI = 4, 5, 6, 7
+PAIR_INTERLEAVED, PAIR_HALF = 0, 1
+PAIRS = {"interleaved": PAIR_INTERLEAVED, "half": PAIR_HALF}
 METHODS = {"rope": ROPE, "pi": PI, "ntk": NTK, "yarn": YARN, "ntk_dynamic": NTK_DYNAMIC,
            "yarn_dimramp": YARN_DIMRAMP, "factors": FACTORS, "alibi": ALIBI}
 SYMBOLS = ("yr_rope_freq_table", "yr_attn_prefill_workspace_bytes", "yr_attn_prefill",
            "yr_prefill_prepare_kv", "yr_prefill_attend", "yr_attn_prefill_chunk",
-           "yr_prefill_prepare_kv_at", "yr_prefill_attend_block", "yr_attn_merge",
+           "yr_attn_prefill_chunk_fp16cache", "yr_attn_prefill_chunk_split_bytes",
+           "yr_prefill_prepare_kv_at",
+           "yr_prefill_attend_block", "yr_attn_merge",
            "yr_attn_decode_workspace_bytes", "yr_attn_decode", "yr_attn_decode_noalloc",
-           "yr_device_status", "yr_last_error", "yr_version")
+           "yr_host_prefill_workspace_bytes", "yr_host_prefill_create", "yr_host_prefill_run",
+           "yr_host_prefill_destroy", "yr_device_status", "yr_last_error", "yr_version")
 
 
 class YarnAttnError(RuntimeError):
@@ -36,14 +41,15 @@ class RopeParams(ctypes.Structure):
     _fields_ = [("head_dim", ctypes.c_int), ("base", ctypes.c_double), ("L_train", ctypes.c_int),
                 ("scale", ctypes.c_double), ("method", ctypes.c_int), ("alpha", ctypes.c_double),
                 ("beta", ctypes.c_double), ("L_cur", ctypes.c_int),
-                ("factors", ctypes.POINTER(ctypes.c_double)), ("attn_factor", ctypes.c_double)]
+                ("factors", ctypes.POINTER(ctypes.c_double)), ("attn_factor", ctypes.c_double),
+                ("pairs", ctypes.c_int)]
 
 
 class RopeTable(ctypes.Structure):
     _fields_ = [("head_dim", ctypes.c_int), ("method", ctypes.c_int),
                 ("inv_freq", ctypes.c_double * 64), ("turns", ctypes.c_double * 64),
                 ("mscale", ctypes.c_double), ("softmax_scale", ctypes.c_double),
-                ("digest", ctypes.c_uint64)]
+                ("digest", ctypes.c_uint64), ("pairs", ctypes.c_int)]
 
 
 _lib = None
@@ -78,6 +84,12 @@ def load(path: str | None = None, make_default: bool = False) -> ctypes.CDLL:
     lib.yr_attn_prefill_chunk.argtypes = ([vp] * 7 + [ci] * 7 +
                                           [ctypes.POINTER(RopeTable), ci, ci, vp, cs, vp])
     lib.yr_attn_prefill_chunk.restype = ci
+    lib.yr_attn_prefill_chunk_fp16cache.argtypes = ([vp] * 7 + [ci] + [vp] * 2 + [ci] * 7 +
+                                                    [ctypes.POINTER(RopeTable), ci, ci, vp, cs,
+                                                     vp])
+    lib.yr_attn_prefill_chunk_split_bytes.argtypes = [ci] * 4
+    lib.yr_attn_prefill_chunk_split_bytes.restype = cs
+    lib.yr_attn_prefill_chunk_fp16cache.restype = ci
     lib.yr_prefill_prepare_kv_at.argtypes = ([vp] * 4 + [ci] * 4 + [i64p] * 3 +
                                              [ctypes.POINTER(RopeTable), ci, vp, cs, vp])
     lib.yr_prefill_prepare_kv_at.restype = ci
@@ -94,6 +106,14 @@ def load(path: str | None = None, make_default: bool = False) -> ctypes.CDLL:
     lib.yr_attn_decode_noalloc.argtypes = ([vp] * 9 + [ci] * 5 +
                                            [ctypes.POINTER(RopeTable), ci, ci, vp])
     lib.yr_attn_decode_noalloc.restype = ci
+    lib.yr_host_prefill_workspace_bytes.argtypes = [ci] * 6
+    lib.yr_host_prefill_workspace_bytes.restype = cs
+    lib.yr_host_prefill_create.argtypes = [ctypes.POINTER(vp)] + [ci] * 6 + [vp, cs]
+    lib.yr_host_prefill_create.restype = ci
+    lib.yr_host_prefill_run.argtypes = [vp] * 5 + [ctypes.POINTER(RopeTable), ci, ci, ci, vp]
+    lib.yr_host_prefill_run.restype = ci
+    lib.yr_host_prefill_destroy.argtypes = [vp]
+    lib.yr_host_prefill_destroy.restype = ci
     lib.yr_device_status.argtypes = [vp]
     lib.yr_device_status.restype = ci
     lib.yr_last_error.argtypes = []
@@ -128,18 +148,20 @@ def _strides(t: torch.Tensor):
 
 def rope_freq_table(head_dim: int, base: float, L_train: int, scale: float, method,
                     alpha: float = 1.0, beta: float = 32.0, L_cur: int = 0, factors=None,
-                    attn_factor: float = 0.0) -> RopeTable:
+                    attn_factor: float = 0.0, pairs="interleaved") -> RopeTable:
     """Frequency/temperature table for one position method (host only).  L_cur is the
     current sequence length (dynamic NTK); factors the d/2 per-dimension divisors and
-    attn_factor the temperature of the factor method."""
+    attn_factor the temperature of the factor method; pairs "interleaved" (2i, 2i+1) or
+    "half" (i, i + d/2)."""
     m = METHODS[method] if isinstance(method, str) else int(method)
+    pr = PAIRS[pairs] if isinstance(pairs, str) else int(pairs)
     fac = None
     if factors is not None:
         fac = (ctypes.c_double * len(factors))(*[float(x) for x in factors])
     p = RopeParams(int(head_dim), float(base), int(L_train), float(scale), m, float(alpha),
                    float(beta), int(L_cur),
                    ctypes.cast(fac, ctypes.POINTER(ctypes.c_double)) if fac is not None else None,
-                   float(attn_factor))
+                   float(attn_factor), pr)
     out = RopeTable()
     _check(load().yr_rope_freq_table(ctypes.byref(p), ctypes.byref(out)))
     return out
@@ -176,79 +198,55 @@ def attn_prefill(q, k, v, table: RopeTable, causal: bool = True, window: int = 0
 
 
 class HostPrefill:
-    """Prefill from pinned host tensors into a pinned host output with the PCIe transfers
-    hidden behind the kernels.  The work is cut into (batch, KV-head group) units; unit i
-    is copied host->device on one stream, rotated and attended on a second (the caller's
-    stream) and copied back on a third, so the copies of later and earlier units run
-    while a unit computes.  Device buffers are allocated once for a given shape and
-    reused; call it repeatedly for a stream of prompts of that shape.  Successive calls
-    overlap too: a unit's copy-in waits only for the previous call's kernels on that unit,
-    and its kernels only for the previous call's copy-out of it."""
+    """Prefill from pinned host tensors into a pinned host output through the library's
+    host-buffer entry point (yr_host_prefill_*): the work is cut into (batch, KV-head
+    group) units whose host-to-device copies, kernels and device-to-host copies overlap
+    on three streams, and successive calls overlap unit by unit.  The device workspace
+    is allocated once here for the shape; call it repeatedly for prompts of that shape."""
 
     def __init__(self, B, Hq, Hkv, T, d, device="cuda", units_per_batch=None):
         self.shape = (B, Hq, Hkv, T, d)
-        self.g = Hq // Hkv
-        n = units_per_batch or min(Hkv, 8)
-        self.kv_per_unit = -(-Hkv // n)
-        dev = torch.device(device)
-        self.qd = torch.empty((B, Hq, T, d), dtype=torch.bfloat16, device=dev)
-        self.kd = torch.empty((B, Hkv, T, d), dtype=torch.bfloat16, device=dev)
-        self.vd = torch.empty_like(self.kd)
-        self.od = torch.empty_like(self.qd)
-        self.ws = torch.empty(attn_prefill_workspace_bytes(1, self.kv_per_unit, T, d),
-                              dtype=torch.uint8, device=dev)
-        self.h2d = torch.cuda.Stream(device=dev)
-        self.d2h = torch.cuda.Stream(device=dev)
-        self.units = [(b, kv0, min(kv0 + self.kv_per_unit, Hkv))
-                      for b in range(B) for kv0 in range(0, Hkv, self.kv_per_unit)]
-        self.computed = [None] * len(self.units)  # per unit: its kernels of the last call
-        self.copied_out = [None] * len(self.units)  # ... and its copy-out
+        lib = load()
+        n = int(units_per_batch or 0)
+        nbytes = int(lib.yr_host_prefill_workspace_bytes(B, Hq, Hkv, T, d, n))
+        if nbytes == 0:
+            raise ValueError("HostPrefill: invalid sizes")
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=torch.device(device))
+        self._lib = lib
+        self.plan = ctypes.c_void_p()
+        _check(lib.yr_host_prefill_create(ctypes.byref(self.plan), B, Hq, Hkv, T, d, n,
+                                          _ptr(self.ws), nbytes))
 
     def __call__(self, q, k, v, table: RopeTable, causal: bool = True, window: int = 0,
-                 n_sink: int = 0, out=None):
+                 n_sink: int = 0, out=None, stream=None):
         """q [B,Hq,T,d], k/v [B,Hkv,T,d] bf16 in pinned host memory, contiguous.  Returns
-        `out` (pinned, allocated if None).  All work is ordered before the caller's
-        current stream's later work; synchronise it before reading `out` or changing the
-        inputs."""
+        `out` (pinned, allocated if None).  All work is ordered before the stream's later
+        work; synchronise it before reading `out` or changing the inputs."""
         B, Hq, Hkv, T, d = self.shape
         if q.shape != (B, Hq, T, d) or k.shape != (B, Hkv, T, d) or v.shape != k.shape:
             raise ValueError("HostPrefill: tensor shapes differ from the ones it was built for")
         for t in (q, k, v):
-            if t.is_cuda or not t.is_pinned() or not t.is_contiguous():
-                raise ValueError("HostPrefill expects contiguous tensors in pinned host memory")
+            if t.is_cuda or not t.is_pinned() or not t.is_contiguous() or \
+                    t.dtype != torch.bfloat16:
+                raise ValueError("HostPrefill expects contiguous bf16 tensors in pinned host "
+                                 "memory")
         if out is None:
             out = torch.empty((B, Hq, T, d), dtype=torch.bfloat16).pin_memory()
-        comp = torch.cuda.current_stream(self.qd.device)
-        g = self.g
-        for u, (b, kv0, kv1) in enumerate(self.units):
-            q_sl = (b, slice(kv0 * g, kv1 * g))
-            kv_sl = (b, slice(kv0, kv1))
-            with torch.cuda.stream(self.h2d):
-                if self.computed[u] is not None:  # the unit's inputs were read by then
-                    self.h2d.wait_event(self.computed[u])
-                self.qd[q_sl].copy_(q[q_sl], non_blocking=True)
-                self.kd[kv_sl].copy_(k[kv_sl], non_blocking=True)
-                self.vd[kv_sl].copy_(v[kv_sl], non_blocking=True)
-                arrived = torch.cuda.Event()
-                arrived.record(self.h2d)
-            comp.wait_event(arrived)
-            if self.copied_out[u] is not None:  # the unit's last output has left
-                comp.wait_event(self.copied_out[u])
-            qu = self.qd[b:b + 1, kv0 * g:kv1 * g]
-            attn_prefill(qu, self.kd[b:b + 1, kv0:kv1], self.vd[b:b + 1, kv0:kv1], table,
-                         causal, window, n_sink, out=self.od[b:b + 1, kv0 * g:kv1 * g],
-                         workspace=self.ws, stream=comp)
-            done = torch.cuda.Event()
-            done.record(comp)
-            self.computed[u] = done
-            with torch.cuda.stream(self.d2h):
-                self.d2h.wait_event(done)
-                out[q_sl].copy_(self.od[q_sl], non_blocking=True)
-                left = torch.cuda.Event()
-                left.record(self.d2h)
-            self.copied_out[u] = left
-        comp.wait_stream(self.d2h)
+        _check(self._lib.yr_host_prefill_run(self.plan, _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                             ctypes.byref(table), int(bool(causal)), int(window),
+                                             int(n_sink), _stream(stream)))
         return out
+
+    def close(self):
+        if self.plan:
+            self._lib.yr_host_prefill_destroy(self.plan)
+            self.plan = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def prefill_prepare_kv(k, v, table: RopeTable, workspace, k_cache=None, k_rot_dbg=None,
@@ -348,6 +346,45 @@ def attn_prefill_chunk(q, k_new, v_new, k_cache, v_cache, P0: int, table: RopeTa
         _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
         B, Hq, Hkv, Tq, d, int(P0), T_max, ctypes.byref(table), int(window), int(n_sink),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc)
+    return out
+
+
+def attn_prefill_chunk_split_bytes(B: int, Hq: int, Tq: int, d: int) -> int:
+    return int(load().yr_attn_prefill_chunk_split_bytes(B, Hq, Tq, d))
+
+
+def attn_prefill_chunk_fp16cache(q, k_new, v_new, k_cache, v_cache, k_cache16, v_cache16,
+                                 cache16_len: int, P0: int, table: RopeTable, window: int = 0,
+                                 n_sink: int = 0, out=None, lse=None, workspace=None,
+                                 split: bool = True, stream=None):
+    """Chunked prefill that keeps an fp16 copy of the cache (k_cache16, v_cache16 fp16
+    [B,Hkv,T_max,d]) whose slots < cache16_len are already valid: only slots
+    cache16_len..P0-1 are converted, and the chunk's slots are written to both copies.
+    `workspace` holds split-KV partials (allocated here when None and split is True;
+    split=False runs one CTA per query block).  Returns the output [B,Hq,Tq,d] bf16;
+    afterwards slots < P0+Tq of the copy are valid."""
+    B, Hq, Tq, d = q.shape
+    Hkv, T_max = k_cache.shape[1], k_cache.shape[2]
+    for t in (q, k_new, v_new, k_cache, v_cache, k_cache16, v_cache16):
+        if not t.is_contiguous():
+            raise ValueError("attn_prefill_chunk_fp16cache expects contiguous tensors")
+    if k_cache16.dtype != torch.float16 or k_cache16.shape != k_cache.shape or \
+            v_cache16.dtype != torch.float16 or v_cache16.shape != v_cache.shape:
+        raise ValueError("the fp16 caches must be float16 tensors shaped like the caches")
+    if out is None:
+        out = torch.empty_like(q)
+    if split and workspace is None:
+        workspace = torch.empty(attn_prefill_chunk_split_bytes(B, Hq, Tq, d), dtype=torch.uint8,
+                                device=q.device)
+    if not split:
+        workspace = None
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().yr_attn_prefill_chunk_fp16cache(
+        _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(k_cache16),
+        _ptr(v_cache16), int(cache16_len), _ptr(out), _ptr(lse), B, Hq, Hkv, Tq, d, int(P0),
+        T_max, ctypes.byref(table), int(window), int(n_sink), _ptr(workspace), ws_bytes,
+        _stream(stream))
     _check(rc)
     return out
 

@@ -49,7 +49,8 @@ def build(force: bool = False, verbose: bool = False, fault_hooks: bool = False)
     common = ["-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include")]
     if fault_hooks:
         common += ["-DYR_FAULT_HOOKS"]
-    for src, extra in [("yarnattn.cu", ARCH + ["-lineinfo"]), ("rope_table.cpp", ARCH)]:
+    for src, extra in [("yarnattn.cu", ARCH + ["-lineinfo"]), ("rope_table.cpp", ARCH),
+                       ("host_prefill.cpp", ARCH)]:
         obj = os.path.join(OUT_DIR, src + tag + ".o")
         cmd = [NVCC] + common + extra + ["-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:

@@ -8,7 +8,8 @@
 // of bytes whatever the mix of cache lengths, and all finish together.  For each
 // segment piece it holds, a block
 //   * rotates the new query of each of the g = Hq/Hkv heads of the group at
-//     position L_b (fp64 angle reduction, fp32 sin/cos) and splits it into a
+//     position L_b (pairs (2i, 2i+1), or (i, i + d/2) in the half-split layout;
+//     fp64 angle reduction, fp32 sin/cos) and splits it into a
 //     bf16 high part and a bf16 remainder, so the product with the bf16 cache
 //     keeps ~16 significant bits of the rotated query;
 //   * if its piece ends at position L_b, rotates the new key and writes it, with
@@ -52,6 +53,7 @@ struct DecodeParams {
     int window, n_sink;
     float sl2;
     int alibi;  // 1: add the ALiBi bias -m_h (L - n) to the logits
+    int half_pairs;  // 1: rotated pairs are (i, i + d/2); 0: (2i, 2i+1)
     double turns[64];
 };
 
@@ -208,14 +210,20 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     const __nv_bfloat16 *vbase = p.v_cache + plane * HD;
 
     // ---- prologue: rotated queries (hi/lo split), the new key into slot L
+    // Elements (ia, ib) of pair i: (2i, 2i+1) interleaved, (i, i + d/2) half-split.
+    auto pair_elems = [&](int i, int &ia, int &ib) {
+        ia = p.half_pairs ? i : 2 * i;
+        ib = p.half_pairs ? i + HD / 2 : 2 * i + 1;
+    };
     for (int e = tid; e < 16 * (HD / 2); e += kDecThreads) {
         const int hh = e / (HD / 2), i = e % (HD / 2);
+        int ia, ib;
+        pair_elems(i, ia, ib);
         float y0 = 0.f, y1 = 0.f;
         if (hh < g && hh < 8 * NT) {
             const int hq = kvh * g + hh;
-            const __nv_bfloat162 q2 = *reinterpret_cast<const __nv_bfloat162 *>(
-                p.q_new + (static_cast<long long>(b) * p.Hq + hq) * HD + 2 * i);
-            const float a = __bfloat162float(q2.x), c = __bfloat162float(q2.y);
+            const __nv_bfloat16 *qrow = p.q_new + (static_cast<long long>(b) * p.Hq + hq) * HD;
+            const float a = __bfloat162float(qrow[ia]), c = __bfloat162float(qrow[ib]);
             const double tr = static_cast<double>(L) * p.turns[i];
             const double frac = tr - rint(tr);
             float sn, cs;
@@ -223,32 +231,34 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             y0 = a * cs - c * sn;
             y1 = a * sn + c * cs;
             if (p.q_dbg != nullptr && has_L) {
-                float *d = p.q_dbg + (static_cast<long long>(b) * p.Hq + hq) * HD + 2 * i;
-                d[0] = y0;
-                d[1] = y1;
+                float *d = p.q_dbg + (static_cast<long long>(b) * p.Hq + hq) * HD;
+                d[ia] = y0;
+                d[ib] = y1;
             }
         }
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(y0, y1);
-        const __nv_bfloat162 lo =
-            __floats2bfloat162_rn(y0 - __bfloat162float(hi.x), y1 - __bfloat162float(hi.y));
-        *reinterpret_cast<__nv_bfloat162 *>(&sm->q_hi[hh][2 * i]) = hi;
-        *reinterpret_cast<__nv_bfloat162 *>(&sm->q_lo[hh][2 * i]) = lo;
+        const __nv_bfloat16 hi0 = __float2bfloat16_rn(y0), hi1 = __float2bfloat16_rn(y1);
+        sm->q_hi[hh][ia] = hi0;
+        sm->q_hi[hh][ib] = hi1;
+        sm->q_lo[hh][ia] = __float2bfloat16_rn(y0 - __bfloat162float(hi0));
+        sm->q_lo[hh][ib] = __float2bfloat16_rn(y1 - __bfloat162float(hi1));
     }
     if (has_L) {
         for (int i = tid; i < HD / 2; i += kDecThreads) {
-            const long long src = (static_cast<long long>(b) * p.Hkv + kvh) * HD + 2 * i;
-            const __nv_bfloat162 k2 = *reinterpret_cast<const __nv_bfloat162 *>(p.k_new + src);
-            const float a = __bfloat162float(k2.x), c = __bfloat162float(k2.y);
+            int ia, ib;
+            pair_elems(i, ia, ib);
+            const long long src = (static_cast<long long>(b) * p.Hkv + kvh) * HD;
+            const float a = __bfloat162float(p.k_new[src + ia]);
+            const float c = __bfloat162float(p.k_new[src + ib]);
             const double tr = static_cast<double>(L) * p.turns[i];
             const double frac = tr - rint(tr);
             float sn, cs;
             __sincosf(static_cast<float>(frac * 6.283185307179586), &sn, &cs);
-            __nv_bfloat16 *kd = p.k_cache + (plane + L) * HD + 2 * i;
-            *reinterpret_cast<__nv_bfloat162 *>(kd) =
-                __floats2bfloat162_rn(a * cs - c * sn, a * sn + c * cs);
-            __nv_bfloat16 *vd = p.v_cache + (plane + L) * HD + 2 * i;
-            *reinterpret_cast<__nv_bfloat162 *>(vd) =
-                *reinterpret_cast<const __nv_bfloat162 *>(p.v_new + src);
+            __nv_bfloat16 *kd = p.k_cache + (plane + L) * HD;
+            kd[ia] = __float2bfloat16_rn(a * cs - c * sn);
+            kd[ib] = __float2bfloat16_rn(a * sn + c * cs);
+            __nv_bfloat16 *vd = p.v_cache + (plane + L) * HD;
+            vd[ia] = p.v_new[src + ia];
+            vd[ib] = p.v_new[src + ib];
         }
     }
     __syncthreads();  // orders the slot-L writes before the copies below

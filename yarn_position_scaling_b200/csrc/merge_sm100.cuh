@@ -83,4 +83,59 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const __grid_constant__
     }
 }
 
+// Split-KV prefill: n_split partials per row, each normalised over its share of the
+// keys with its log-sum-exp, combined into the bf16 output (and the lse):
+//     M = max_s lse_s,  o = sum_s e^(lse_s - M) o_s / sum_s e^(lse_s - M),
+//     lse = M + log sum_s e^(lse_s - M).
+// A share with no visible key for the row has lse_s = -inf and is not read.  One
+// lane per 8 elements of a row; HBM-bound (4d bytes per row and share read, 2d written).
+struct SplitMergeParams {
+    const float *o_part;    // [n_split][rows][d]
+    const float *lse_part;  // [n_split][rows]
+    __nv_bfloat16 *o;       // [rows][d]
+    float *lse;             // [rows] or null
+    long long rows;
+    int d, n_split;
+};
+
+__global__ void __launch_bounds__(256) split_merge_kernel(const __grid_constant__ SplitMergeParams p) {
+    const int cpr = p.d >> 3;
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+         g < p.rows * cpr; g += stride) {
+        const long long row = g / cpr;
+        const int c = static_cast<int>(g % cpr);
+        float M = -INFINITY;
+        for (int s = 0; s < p.n_split; ++s) M = fmaxf(M, p.lse_part[s * p.rows + row]);
+        float r[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float sum = 0.f;
+        if (M > -INFINITY) {
+            for (int s = 0; s < p.n_split; ++s) {
+                const float ls = p.lse_part[s * p.rows + row];
+                if (ls == -INFINITY) continue;
+                const float w = expf(ls - M);
+                sum += w;
+                const float4 *src =
+                    reinterpret_cast<const float4 *>(p.o_part + (s * p.rows + row) * p.d + c * 8);
+                const float4 a = src[0], bq = src[1];
+                r[0] = fmaf(w, a.x, r[0]); r[1] = fmaf(w, a.y, r[1]);
+                r[2] = fmaf(w, a.z, r[2]); r[3] = fmaf(w, a.w, r[3]);
+                r[4] = fmaf(w, bq.x, r[4]); r[5] = fmaf(w, bq.y, r[5]);
+                r[6] = fmaf(w, bq.z, r[6]); r[7] = fmaf(w, bq.w, r[7]);
+            }
+            const float inv = 1.0f / sum;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) r[i] *= inv;
+        }
+        uint32_t pk[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(r[2 * i], r[2 * i + 1]);
+            pk[i] = *reinterpret_cast<uint32_t *>(&b2);
+        }
+        *reinterpret_cast<uint4 *>(p.o + row * p.d + c * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        if (p.lse != nullptr && c == 0) p.lse[row] = M > -INFINITY ? M + logf(sum) : -INFINITY;
+    }
+}
+
 }  // namespace yr

@@ -22,6 +22,8 @@
 //   ALiBi  no rotation (theta' = 0); the kernels add the per-head linear bias
 //          (ALiBi slide)
 //   softmax_scale = mscale^2 / sqrt(d): the temperature on both rotated q and k.
+//   The pair layout (interleaved (2i, 2i+1) or half-split (i, i + d/2)) is
+//   carried in the table for the kernels; it does not change any frequency.
 // The table also carries theta'_i / (2 pi) (rotations per position), which the
 // kernels multiply by the position in fp64 to reduce the angle exactly.
 #include <algorithm>
@@ -80,6 +82,10 @@ extern "C" int yr_rope_freq_table(const yr_rope_params *p, yr_rope_table *out) {
         yr_host::set_error("yr_rope_freq_table: dynamic NTK needs L_train >= 1 and L_cur >= 1");
         return YR_EINVAL;
     }
+    if (p->pairs != YR_PAIR_INTERLEAVED && p->pairs != YR_PAIR_HALF) {
+        yr_host::set_error("yr_rope_freq_table: pairs must be YR_PAIR_INTERLEAVED or YR_PAIR_HALF");
+        return YR_EINVAL;
+    }
     if (p->method == YR_FACTORS) {
         if (p->factors == nullptr) {
             yr_host::set_error("yr_rope_freq_table: YR_FACTORS needs d/2 factors");
@@ -96,6 +102,7 @@ extern "C" int yr_rope_freq_table(const yr_rope_params *p, yr_rope_table *out) {
     std::memset(&t, 0, sizeof t);
     t.head_dim = d;
     t.method = p->method;
+    t.pairs = p->pairs;
     const double two_pi = 2.0 * M_PI;
     const double ln_base = std::log(p->base);
     const double s = p->scale;
@@ -171,6 +178,7 @@ extern "C" int yr_rope_freq_table(const yr_rope_params *p, yr_rope_table *out) {
     hsh = fnv1a(hsh, fields_i, sizeof fields_i);
     hsh = fnv1a(hsh, fields_d, sizeof fields_d);
     if (fac) hsh = fnv1a(hsh, p->factors, sizeof(double) * (d / 2));
+    if (p->pairs != YR_PAIR_INTERLEAVED) hsh = fnv1a(hsh, &p->pairs, sizeof p->pairs);
     t.digest = hsh;
     *out = t;
     return YR_OK;

@@ -209,8 +209,14 @@ int encode(CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base,
     return YR_OK;
 }
 
-size_t prefill_ws_bytes(long long B, long long Hkv, long long T, long long d) {
+// Prefill workspace: the rotated keys and the values in fp16, then 256 bytes that hold
+// the work counter of the persistent attention grid.
+constexpr size_t kCounterBytes = 256;
+size_t prefill_planes_bytes(long long B, long long Hkv, long long T, long long d) {
     return static_cast<size_t>(2 * B * Hkv * T * d * 2);
+}
+size_t prefill_ws_bytes(long long B, long long Hkv, long long T, long long d) {
+    return prefill_planes_bytes(B, Hkv, T, d) + kCounterBytes;
 }
 
 // Partial-result slots per (b, KV head): a block of the balanced split holds at least
@@ -266,6 +272,8 @@ int check_common(const char *fn, int B, int Hkv, int T, int d, const yr_rope_tab
     if (B < 1 || Hkv < 1 || T < 1) return fail(YR_EINVAL, f + ": B, Hkv and T must be >= 1");
     if (d != 64 && d != 128) return fail(YR_EUNSUPPORTED, f + ": d must be 64 or 128");
     if (tab->head_dim != d) return fail(YR_EINVAL, f + ": table head_dim != d");
+    if (tab->pairs != YR_PAIR_INTERLEAVED && tab->pairs != YR_PAIR_HALF)
+        return fail(YR_EINVAL, f + ": table pairs must be YR_PAIR_INTERLEAVED or YR_PAIR_HALF");
     const size_t need = prefill_ws_bytes(B, Hkv, T, d);
     if (workspace_bytes < need)
         return fail(YR_EINVAL, f + ": workspace too small (need " + std::to_string(need) + " bytes)");
@@ -307,7 +315,7 @@ int check_attend(const void *q, const void *o, const float *lse, const float *q_
     if (window < 0 || n_sink < 0) return fail(YR_EINVAL, f + ": window and n_sink must be >= 0");
     if (window > 0 && !causal) return fail(YR_EINVAL, f + ": a window needs causal=1");
     if (n_sink > 0 && window == 0) return fail(YR_EINVAL, f + ": sinks need a window");
-    if (static_cast<long long>(B) * Hq * ((T + 255) / 256) >= (1ll << 31))
+    if (static_cast<long long>(B) * Hq * ((T + 255) / 256) * 16 >= (1ll << 31))
         return fail(YR_EINVAL, f + ": problem too large for one launch");
     for (const void *ptr : {q, o, static_cast<const void *>(q_rot_dbg)})
         if (ptr && !aligned(ptr, 16)) return fail(YR_EINVAL, f + ": pointers must be 16-byte aligned");
@@ -338,33 +346,52 @@ int launch_prepare(const void *k, const void *v, void *k_cache, float *k_rot_dbg
     kp.k_dbg = k_rot_dbg;
     kp.Hkv = Hkv; kp.T = T; kp.d = d;
     kp.pos0 = pos0;
-    kp.n_items = static_cast<long long>(B) * Hkv * T * (d / 8);
+    const bool half = tab->pairs == YR_PAIR_HALF;
+    kp.n_items = static_cast<long long>(B) * Hkv * T * (half ? d / 16 : d / 8);
     for (int i = 0; i < d / 2; ++i) kp.turns[i] = tab->turns[i];
     long long blocks = (kp.n_items + 255) / 256;
     const long long cap = static_cast<long long>(sm_count) * 16;
     if (blocks > cap) blocks = cap;
-    yr::kv_prep_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(kp);
+    if (half)
+        yr::kv_prep_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(kp);
+    else
+        yr::kv_prep_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(kp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("kv_prep_kernel launch", e);
     return YR_OK;
 }
 
-// T query rows against Tk keys laid out in the workspace as fp16 [B*Hkv][Tk][d]
-// rotated keys, then the same for values.  Key n sits at position k_pos0 + n and
+// The fp16 rotated keys and values the attention kernel reads: planes of ld16 rows
+// of d elements, one per (b, KV head), keys [0, Tk) of each.
+// `counter` (nullable): device int the persistent grid takes work units from.
+struct KvPlanes {
+    const __half *k16;
+    const __half *v16;
+    long long ld16;
+    int *counter;
+};
+// The layout of a prefill workspace: K [B*Hkv][Tk][d], then V the same, then the
+// counter.
+KvPlanes workspace_planes(const void *workspace, int B, int Hkv, int Tk, int d) {
+    const __half *k16 = static_cast<const __half *>(workspace);
+    int *counter = reinterpret_cast<int *>(static_cast<char *>(const_cast<void *>(workspace)) +
+                                           prefill_planes_bytes(B, Hkv, Tk, d));
+    return {k16, k16 + static_cast<size_t>(B) * Hkv * Tk * d, Tk, counter};
+}
+
+// T query rows against the Tk keys of `kv`.  Key n sits at position k_pos0 + n and
 // query row r at k_pos0 + q_off + r; masks use the offsets relative to key 0.
 int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, int Hq, int Hkv,
                   int T, int d, const long long qs[3], const long long os[3],
                   const yr_rope_table *tab, int causal, int window, int n_sink,
-                  const void *workspace, cudaStream_t st, int Tk, int q_off, int k_pos0 = 0,
-                  float *o32 = nullptr) {
+                  const KvPlanes &kv, cudaStream_t st, int Tk, int q_off, int k_pos0 = 0,
+                  float *o32 = nullptr, int n_split = 1) {
     DeviceState ds;
     int rc = prepare_device(nullptr, &ds);
     if (rc != YR_OK) return rc;
     if (!ds.prefill_regs_ok)
         return fail(YR_EUNSUPPORTED, "prefill kernel was built with too few registers per thread "
                                      "for its warpgroup register split");
-    const __half *k16 = static_cast<const __half *>(workspace);
-    const __half *v16 = k16 + static_cast<size_t>(B) * Hkv * Tk * d;
     yr::PrefillParams pp;
     std::memset(&pp, 0, sizeof pp);
     {
@@ -381,12 +408,12 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
         const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(Tk),
                                     static_cast<cuuint64_t>(B) * Hkv};
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                                       static_cast<cuuint64_t>(Tk) * d * 2};
+                                       static_cast<cuuint64_t>(kv.ld16) * d * 2};
         const cuuint32_t box[3] = {64, 128, 1};
-        rc = encode(&pp.tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, k16, dims, strides, box,
+        rc = encode(&pp.tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, kv.k16, dims, strides, box,
                     "rotated k");
         if (rc != YR_OK) return rc;
-        rc = encode(&pp.tm_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, v16, dims, strides, box, "v");
+        rc = encode(&pp.tm_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, kv.v16, dims, strides, box, "v");
         if (rc != YR_OK) return rc;
     }
     pp.o = static_cast<__nv_bfloat16 *>(o);
@@ -398,10 +425,13 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     pp.Tk = Tk; pp.q_off = q_off; pp.k_pos0 = k_pos0;
     pp.causal = causal; pp.window = window; pp.n_sink = n_sink;
     pp.n_qblocks = (T + 255) / 256;
+    pp.n_split = n_split;
+    pp.split_rows = static_cast<long long>(B) * Hq * T;
     // Grouped query heads read each K/V tile several times: order the CTAs by KV head
     // so that re-reads hit L2 (measured: +2.7% at the 128K GQA workload, neutral for MHA).
     pp.kv_major = pp.group > 1 ? 1 : 0;
     pp.alibi = tab->method == YR_ALIBI ? 1 : 0;
+    pp.half_pairs = tab->pairs == YR_PAIR_HALF ? 1 : 0;
     pp.sl2 = static_cast<float>(tab->softmax_scale * 1.4426950408889634);
     pp.timeout_ns = wait_timeout_ns();
 #ifdef YR_FAULT_HOOKS
@@ -412,7 +442,17 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     pp.fault_drop_tile = -1;
 #endif
     for (int i = 0; i < d / 2; ++i) pp.turns[i] = tab->turns[i];
-    const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * Hq * pp.n_qblocks);
+    const long long n_units = static_cast<long long>(B) * Hq * pp.n_qblocks * n_split;
+    pp.n_units = static_cast<int>(n_units);
+    // Persistent grid: one CTA per SM (the kernel needs a whole SM's TMEM and most of its
+    // shared memory), each taking units from the counter until none is left.
+    pp.work_counter = kv.counter;
+    unsigned grid = static_cast<unsigned>(n_units);
+    if (kv.counter != nullptr) {
+        if (n_units > ds.sm_count) grid = static_cast<unsigned>(ds.sm_count);
+        cudaError_t me = cudaMemsetAsync(kv.counter, 0, sizeof(int), st);
+        if (me != cudaSuccess) return cuda_fail("cudaMemsetAsync(work counter)", me);
+    }
     if (d == 128)
         yr::prefill_attn_kernel<128>
             <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<128>(), st>>>(pp);
@@ -458,7 +498,8 @@ extern "C" int yr_prefill_attend(const void *q, void *o, float *lse, float *q_ro
     rc = prepare_device(nullptr);
     if (rc != YR_OK) return rc;
     return launch_attend(q, o, lse, q_rot_dbg, B, Hq, Hkv, T, d, qs, os, tab, causal, window,
-                         n_sink, workspace, static_cast<cudaStream_t>(stream), T, 0);
+                         n_sink, workspace_planes(workspace, B, Hkv, T, d),
+                         static_cast<cudaStream_t>(stream), T, 0);
 }
 
 extern "C" int yr_attn_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
@@ -485,8 +526,121 @@ extern "C" int yr_attn_prefill(const void *q, const void *k, const void *v, void
                         sm_count, st);
     if (rc != YR_OK) return rc;
     return launch_attend(q, o, lse, q_rot_dbg, B, Hq, Hkv, T, d, qs, os, tab, causal, window,
-                         n_sink, workspace, st, T, 0);
+                         n_sink, workspace_planes(workspace, B, Hkv, T, d), st, T, 0);
 }
+
+namespace yr_host {
+
+// The shared body of the two chunked-prefill entry points: argument checks, the
+// chunk pass into (k16, v16) with plane stride ld16 starting at slot `first`, then
+// the attention over those planes.
+// Bytes of one split-KV share's partials: fp32 o [B*Hq*Tq][d] and lse [B*Hq*Tq].
+size_t split_share_bytes(long long B, long long Hq, long long Tq, long long d) {
+    return static_cast<size_t>(B * Hq * Tq * (d + 1) * 4);
+}
+
+// Shares per item for a prefill of Tq query rows after P0 cached keys: enough CTAs
+// for two waves when the items alone are too few, each share at least 4 key tiles,
+// at most kMaxSplit and at most what the split workspace holds.
+constexpr int kMaxSplit = 16;
+int choose_split(int sm_count, int B, int Hq, int Tq, int P0, int window, size_t ws_bytes,
+                 size_t share_bytes) {
+    const long long items = static_cast<long long>(B) * Hq * ((Tq + 255) / 256);
+    if (items >= 2ll * sm_count || share_bytes == 0) return 1;
+    int keys = P0 + (Tq < 256 ? Tq : 256);  // the first query block's keys (the fewest)
+    if (window > 0 && window < keys) keys = window + 256;
+    const int tiles = (keys + 127) / 128;
+    long long s = (2ll * sm_count + items - 1) / items;
+    if (s > kMaxSplit) s = kMaxSplit;
+    if (s > tiles / 4) s = tiles / 4;
+    if (s > static_cast<long long>(ws_bytes / share_bytes)) s = ws_bytes / share_bytes;
+    return s < 2 ? 1 : static_cast<int>(s);
+}
+
+int chunk_call(const char *fn, const void *q, const void *k_new, const void *v_new,
+               void *k_cache, void *v_cache, void *o, float *lse, int B, int Hq, int Hkv,
+               int Tq, int d, int P0, int T_max, const yr_rope_table *tab, int window,
+               int n_sink, __half *k16, __half *v16, long long ld16, int first,
+               int *counter, void *split_ws, size_t split_ws_bytes, void *stream) {
+    const std::string f(fn);
+    if (!q || !k_new || !v_new || !k_cache || !v_cache || !o || !tab)
+        return fail(YR_EINVAL, f + ": NULL pointer argument");
+    if (B < 1 || Hq < 1 || Hkv < 1 || Tq < 1) return fail(YR_EINVAL, f + ": B, Hq, Hkv and Tq must be >= 1");
+    if (P0 < 0 || T_max < 1 || static_cast<long long>(P0) + Tq > T_max)
+        return fail(YR_EINVAL, f + ": need 0 <= P0 and P0 + Tq <= T_max");
+    const int Tk = P0 + Tq;
+    long long qs[3], os[3];
+    // check_attend and check_common want a workspace: hand them the fp16 planes, sized
+    // for the keys they must hold (the planes' own size is checked by the callers).
+    const size_t planes = prefill_ws_bytes(B, Hkv, Tk, d);
+    int rc = check_attend(q, o, lse, nullptr, B, Hq, Hkv, Tq, d, nullptr, nullptr, tab, 1, window,
+                          n_sink, k16, planes, fn, qs, os);
+    if (rc != YR_OK) return rc;
+    for (const void *ptr : {k_new, v_new, static_cast<const void *>(k_cache),
+                            static_cast<const void *>(v_cache), static_cast<const void *>(v16)})
+        if (!aligned(ptr, 16)) return fail(YR_EINVAL, f + ": pointers must be 16-byte aligned");
+    int sm_count = 0;
+    rc = prepare_device(&sm_count);
+    if (rc != YR_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool half = tab->pairs == YR_PAIR_HALF;
+    if (Tk > first) {
+        yr::ChunkPrepParams cp;
+        std::memset(&cp, 0, sizeof cp);
+        cp.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+        cp.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+        cp.kc = static_cast<__nv_bfloat16 *>(k_cache);
+        cp.vc = static_cast<__nv_bfloat16 *>(v_cache);
+        cp.k16 = k16;
+        cp.v16 = v16;
+        cp.Tq = Tq; cp.P0 = P0; cp.Tk = Tk; cp.T_max = T_max; cp.d = d;
+        cp.first = first;
+        cp.ld16 = ld16;
+        cp.n_items = static_cast<long long>(B) * Hkv * (Tk - first) * (half ? d / 16 : d / 8);
+        for (int i = 0; i < d / 2; ++i) cp.turns[i] = tab->turns[i];
+        long long blocks = (cp.n_items + 255) / 256;
+        const long long cap = static_cast<long long>(sm_count) * 16;
+        if (blocks > cap) blocks = cap;
+        if (half)
+            yr::chunk_prep_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(cp);
+        else
+            yr::chunk_prep_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(cp);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail("chunk_prep_kernel launch", e);
+    }
+    const size_t share = split_share_bytes(B, Hq, Tq, d);
+    const int n_split = split_ws ? choose_split(sm_count, B, Hq, Tq, P0, window, split_ws_bytes,
+                                                share)
+                                 : 1;
+    const KvPlanes kv{k16, v16, ld16, counter};
+    if (n_split == 1)
+        return launch_attend(q, o, lse, nullptr, B, Hq, Hkv, Tq, d, qs, os, tab, 1, window,
+                             n_sink, kv, st, Tk, P0);
+    // Split-KV: the shares' fp32 partials, then their log-sum-exp merge into o.
+    const long long rows = static_cast<long long>(B) * Hq * Tq;
+    float *o_part = static_cast<float *>(split_ws);
+    float *lse_part = o_part + n_split * rows * d;
+    rc = launch_attend(q, nullptr, lse_part, nullptr, B, Hq, Hkv, Tq, d, qs, os, tab, 1, window,
+                       n_sink, kv, st, Tk, P0, 0, o_part, n_split);
+    if (rc != YR_OK) return rc;
+    yr::SplitMergeParams mp;
+    mp.o_part = o_part;
+    mp.lse_part = lse_part;
+    mp.o = static_cast<__nv_bfloat16 *>(o);
+    mp.lse = lse;
+    mp.rows = rows;
+    mp.d = d;
+    mp.n_split = n_split;
+    long long blocks = (rows * (d / 8) + 255) / 256;
+    const long long cap = static_cast<long long>(sm_count) * 16;
+    if (blocks > cap) blocks = cap;
+    yr::split_merge_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(mp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("split_merge_kernel launch", e);
+    return YR_OK;
+}
+
+}  // namespace yr_host
 
 extern "C" int yr_attn_prefill_chunk(const void *q, const void *k_new, const void *v_new,
                                      void *k_cache, void *v_cache, void *o, float *lse, int B,
@@ -494,45 +648,54 @@ extern "C" int yr_attn_prefill_chunk(const void *q, const void *k_new, const voi
                                      const yr_rope_table *tab, int window, int n_sink,
                                      void *workspace, size_t workspace_bytes, void *stream) {
     set_error("");
-    const std::string f("yr_attn_prefill_chunk");
-    if (!q || !k_new || !v_new || !k_cache || !v_cache || !o)
-        return fail(YR_EINVAL, f + ": NULL pointer argument");
-    if (B < 1 || Hq < 1 || Hkv < 1 || Tq < 1) return fail(YR_EINVAL, f + ": B, Hq, Hkv and Tq must be >= 1");
-    if (P0 < 0 || T_max < 1 || static_cast<long long>(P0) + Tq > T_max)
-        return fail(YR_EINVAL, f + ": need 0 <= P0 and P0 + Tq <= T_max");
+    const char *fn = "yr_attn_prefill_chunk";
+    if (!workspace) return fail(YR_EINVAL, std::string(fn) + ": workspace must be non-NULL");
+    if (B < 1 || Hkv < 1 || Tq < 1 || P0 < 0 || static_cast<long long>(P0) + Tq > (1ll << 30))
+        return fail(YR_EINVAL, std::string(fn) + ": B, Hkv, Tq >= 1 and 0 <= P0 needed");
     const int Tk = P0 + Tq;
-    long long qs[3], os[3];
-    int rc = check_attend(q, o, lse, nullptr, B, Hq, Hkv, Tq, d, nullptr, nullptr, tab, 1, window,
-                          n_sink, workspace, workspace_bytes, "yr_attn_prefill_chunk", qs, os);
-    if (rc != YR_OK) return rc;
-    rc = check_common("yr_attn_prefill_chunk", B, Hkv, Tk, d, tab, workspace, workspace_bytes);
-    if (rc != YR_OK) return rc;
-    for (const void *ptr : {k_new, v_new, static_cast<const void *>(k_cache),
-                            static_cast<const void *>(v_cache)})
-        if (!aligned(ptr, 16)) return fail(YR_EINVAL, f + ": pointers must be 16-byte aligned");
-    int sm_count = 0;
-    rc = prepare_device(&sm_count);
-    if (rc != YR_OK) return rc;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    yr::ChunkPrepParams cp;
-    std::memset(&cp, 0, sizeof cp);
-    cp.k_new = static_cast<const __nv_bfloat16 *>(k_new);
-    cp.v_new = static_cast<const __nv_bfloat16 *>(v_new);
-    cp.kc = static_cast<__nv_bfloat16 *>(k_cache);
-    cp.vc = static_cast<__nv_bfloat16 *>(v_cache);
-    cp.k16 = static_cast<__half *>(workspace);
-    cp.v16 = cp.k16 + static_cast<size_t>(B) * Hkv * Tk * d;
-    cp.Tq = Tq; cp.P0 = P0; cp.Tk = Tk; cp.T_max = T_max; cp.d = d;
-    cp.n_items = static_cast<long long>(B) * Hkv * Tk * (d / 8);
-    for (int i = 0; i < d / 2; ++i) cp.turns[i] = tab->turns[i];
-    long long blocks = (cp.n_items + 255) / 256;
-    const long long cap = static_cast<long long>(sm_count) * 16;
-    if (blocks > cap) blocks = cap;
-    yr::chunk_prep_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(cp);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail("chunk_prep_kernel launch", e);
-    return launch_attend(q, o, lse, nullptr, B, Hq, Hkv, Tq, d, qs, os, tab, 1, window, n_sink,
-                         workspace, st, Tk, P0);
+    const size_t need = prefill_ws_bytes(B, Hkv, Tk, d);
+    if (workspace_bytes < need)
+        return fail(YR_EINVAL, std::string(fn) + ": workspace too small (need " +
+                                   std::to_string(need) + " bytes)");
+    if (!aligned(workspace, 256))
+        return fail(YR_EINVAL, std::string(fn) + ": workspace must be 256-byte aligned");
+    const KvPlanes kv = workspace_planes(workspace, B, Hkv, Tk, d);
+    return chunk_call(fn, q, k_new, v_new, k_cache, v_cache, o, lse, B, Hq, Hkv, Tq, d, P0,
+                      T_max, tab, window, n_sink, const_cast<__half *>(kv.k16),
+                      const_cast<__half *>(kv.v16), Tk, 0, kv.counter, nullptr, 0, stream);
+}
+
+extern "C" size_t yr_attn_prefill_chunk_split_bytes(int B, int Hq, int Tq, int d) {
+    if (B < 1 || Hq < 1 || Tq < 1 || (d != 64 && d != 128)) return 0;
+    return kCounterBytes + kMaxSplit * split_share_bytes(B, Hq, Tq, d);
+}
+
+extern "C" int yr_attn_prefill_chunk_fp16cache(const void *q, const void *k_new,
+                                               const void *v_new, void *k_cache, void *v_cache,
+                                               void *k_cache16, void *v_cache16, int cache16_len,
+                                               void *o, float *lse, int B, int Hq, int Hkv,
+                                               int Tq, int d, int P0, int T_max,
+                                               const yr_rope_table *tab, int window, int n_sink,
+                                               void *workspace, size_t workspace_bytes,
+                                               void *stream) {
+    set_error("");
+    const char *fn = "yr_attn_prefill_chunk_fp16cache";
+    if (!k_cache16 || !v_cache16)
+        return fail(YR_EINVAL, std::string(fn) + ": k_cache16 and v_cache16 must be non-NULL");
+    if (!aligned(k_cache16, 256) || !aligned(v_cache16, 256))
+        return fail(YR_EINVAL, std::string(fn) + ": the fp16 caches must be 256-byte aligned");
+    if (cache16_len < 0 || cache16_len > P0)
+        return fail(YR_EINVAL, std::string(fn) + ": need 0 <= cache16_len <= P0");
+    if (workspace && !aligned(workspace, 256))
+        return fail(YR_EINVAL, std::string(fn) + ": workspace must be 256-byte aligned");
+    // The workspace starts with the work counter; the split partials follow it.
+    const bool has_ws = workspace != nullptr && workspace_bytes >= kCounterBytes;
+    int *counter = has_ws ? static_cast<int *>(workspace) : nullptr;
+    void *split_ws = has_ws ? static_cast<char *>(workspace) + kCounterBytes : nullptr;
+    return chunk_call(fn, q, k_new, v_new, k_cache, v_cache, o, lse, B, Hq, Hkv, Tq, d, P0,
+                      T_max, tab, window, n_sink, static_cast<__half *>(k_cache16),
+                      static_cast<__half *>(v_cache16), T_max, cache16_len, counter, split_ws,
+                      has_ws ? workspace_bytes - kCounterBytes : 0, stream);
 }
 
 extern "C" int yr_prefill_prepare_kv_at(const void *k, const void *v, void *k_cache,
@@ -583,8 +746,8 @@ extern "C" int yr_prefill_attend_block(const void *q, float *o, float *lse, int 
     // coordinates they are keys [0, n_sink - k_pos0).
     const int sinks_here = n_sink > k_pos0 ? n_sink - k_pos0 : 0;
     return launch_attend(q, nullptr, lse, nullptr, B, Hq, Hkv, T, d, qs, os, tab, causal, window,
-                         sinks_here, workspace, static_cast<cudaStream_t>(stream), Tk,
-                         q_pos0 - k_pos0, k_pos0, o);
+                         sinks_here, workspace_planes(workspace, B, Hkv, Tk, d),
+                         static_cast<cudaStream_t>(stream), Tk, q_pos0 - k_pos0, k_pos0, o);
 }
 
 extern "C" int yr_attn_merge(const float *o_part, const float *lse_part, float *o_acc,
@@ -638,6 +801,8 @@ extern "C" int yr_attn_decode(const void *q_new, const void *k_new, const void *
     if (d != 64 && d != 128) return fail(YR_EUNSUPPORTED, "yr_attn_decode: d must be 64 or 128");
     if (Hq / Hkv > 16) return fail(YR_EUNSUPPORTED, "yr_attn_decode: at most 16 query heads per KV head");
     if (tab->head_dim != d) return fail(YR_EINVAL, "yr_attn_decode: table head_dim != d");
+    if (tab->pairs != YR_PAIR_INTERLEAVED && tab->pairs != YR_PAIR_HALF)
+        return fail(YR_EINVAL, "yr_attn_decode: table pairs must be YR_PAIR_INTERLEAVED or YR_PAIR_HALF");
     if (window < 0 || n_sink < 0) return fail(YR_EINVAL, "yr_attn_decode: window and n_sink must be >= 0");
     if (n_sink > 0 && window == 0) return fail(YR_EINVAL, "yr_attn_decode: sinks need a window");
     const size_t need = decode_ws_bytes(B, Hq, Hkv, d, T_max);
@@ -672,6 +837,7 @@ extern "C" int yr_attn_decode(const void *q_new, const void *k_new, const void *
     dp.window = window; dp.n_sink = n_sink;
     dp.sl2 = static_cast<float>(tab->softmax_scale * 1.4426950408889634);
     dp.alibi = tab->method == YR_ALIBI ? 1 : 0;
+    dp.half_pairs = tab->pairs == YR_PAIR_HALF ? 1 : 0;
     for (int i = 0; i < d / 2; ++i) dp.turns[i] = tab->turns[i];
     if (d == 128) {
         if (g <= 8) {
