@@ -131,10 +131,8 @@ int yr_rope_freq_table(const yr_rope_params *p, yr_rope_table *out);
 
 /*
  * attn_prefill_workspace_bytes -- bytes of device workspace yr_attn_prefill
- * needs: the rotated keys and the values, each [B, Hkv, T, d] in fp16, then 256
- * bytes for the work counter of the persistent attention grid (one CTA per SM,
- * each taking the next 256-row query block of a (batch, head) from the counter,
- * heaviest first).  Returns 0 for invalid sizes.
+ * needs: the rotated keys and the values, each [B, Hkv, T, d] in fp16.
+ * Returns 0 for invalid sizes.
  */
 size_t yr_attn_prefill_workspace_bytes(int B, int Hkv, int T, int d);
 
@@ -257,9 +255,7 @@ int yr_attn_prefill_chunk(const void *q, const void *k_new, const void *v_new,
  *     passes cache16_len = P0 + Tq.  Slots a decode step appended to the bf16
  *     cache in between are picked up by passing the last valid length.
  *   0 <= cache16_len <= P0.
- *   workspace (nullable, 256-byte aligned): 256 bytes for the persistent grid's
- *     work counter (without it, one CTA per query block), then room for split-KV
- *     partials.  A short
+ *   workspace (nullable, 256-byte aligned): room for split-KV partials.  A short
  *     chunk after a long prefix has few (sequence, head, 256-row query block)
  *     items -- 32 for one 256-token chunk of a 32-head model -- too few for the
  *     GPU's SMs; with a workspace the call cuts each item's keys into up to 16

@@ -179,10 +179,10 @@ def test_decode_rejects_bad_arguments_on_host(lib, kw, code):
 
 
 def test_workspace_sizes(lib):
-    # rotated keys and values in fp16, then 256 bytes for the persistent grid's work counter
-    assert api.attn_prefill_workspace_bytes(1, 8, 131072, 128) == 2 * 8 * 131072 * 128 * 2 + 256
-    # the chunk's split-KV workspace: the counter, then up to 16 shares of fp32 o and lse
-    assert api.attn_prefill_chunk_split_bytes(1, 32, 256, 128) == 256 + 16 * 32 * 256 * 129 * 4
+    # rotated keys and values in fp16
+    assert api.attn_prefill_workspace_bytes(1, 8, 131072, 128) == 2 * 8 * 131072 * 128 * 2
+    # the chunk's split-KV workspace: up to 16 shares of fp32 o and lse
+    assert api.attn_prefill_chunk_split_bytes(1, 32, 256, 128) == 16 * 32 * 256 * 129 * 4
     # one partial slot per block of the balanced split that can hold part of a segment:
     # blocks hold at least 2048 keys, so a segment of T_max keys touches ceil(T_max/2048)+1
     parts = (131073 + 2047) // 2048 + 1
@@ -201,11 +201,10 @@ def test_table_rejects_unknown_pair_layout(lib):
 
 def test_host_prefill_plan_checks_arguments_before_any_cuda_call(lib):
     # sizes: q and o [B,Hq,T,d], k and v [B,Hkv,T,d] bf16, each rounded up to 256 bytes,
-    # plus one unit's prefill workspace (rotated keys and values of its KV heads, fp16, and
-    # the work counter)
+    # plus one unit's prefill workspace (rotated keys and values of its KV heads, fp16)
     B, Hq, Hkv, T, d = 2, 4, 2, 16, 64
     r = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    want = 2 * r(B * Hq * T * d * 2) + 2 * r(B * Hkv * T * d * 2) + r(4 * 1 * T * d + 256)
+    want = 2 * r(B * Hq * T * d * 2) + 2 * r(B * Hkv * T * d * 2) + r(4 * 1 * T * d)
     assert lib.yr_host_prefill_workspace_bytes(B, Hq, Hkv, T, d, 2) == want  # 1 KV head a unit
     assert lib.yr_host_prefill_workspace_bytes(1, 3, 2, 16, 64, 0) == 0      # Hq % Hkv
     assert lib.yr_host_prefill_workspace_bytes(1, 4, 2, 16, 96, 0) == 0      # head size

@@ -32,7 +32,7 @@
 //
 // Rotation ("Arch_03_Long_Context", RoPE slide): pair (2i, 2i+1) of the query
 // at position m turns by m * theta'_i (or pair (i, i + d/2) in the half-split
-// layout).  Each softmax warp reduces the angle of
+// layout, a separate instantiation of the kernel).  Each softmax warp reduces the angle of
 // every pair at its first row in fp64 (turns minus the nearest integer); a row
 // adds lane * theta'_i / (2 pi) in fp32 and takes fp32 sin/cos.  A rotated value
 // that does not fit fp16 sets the range bit of the device status word.  Rarely run
@@ -86,19 +86,12 @@ struct alignas(64) PrefillParams {
     int n_qblocks;
     int kv_major;  // CTA order: 1 = by KV head first (grouped heads), 0 = by query block
     int alibi;     // 1: add the ALiBi bias -m_h (i - j) to the logits
-    int half_pairs;  // 1: rotated pairs are (i, i + d/2); 0: (2i, 2i+1)
     // Split-KV: each (batch, head, query block) item is cut into n_split CTAs that take
     // equal shares of its key tiles; CTA s writes its normalised fp32 partial to
     // o32 + s * split_rows * d and its log-sum-exp to lse + s * split_rows, and a merge
     // kernel combines them.  n_split = 1: one CTA per item.
     int n_split;
     long long split_rows;
-    // Work units (item, share) in the CTA order below: n_units = B * Hq * n_qblocks *
-    // n_split.  With work_counter set the grid is persistent -- at most one CTA per SM,
-    // each taking the next unit from the counter (zeroed before the launch) until none
-    // is left -- otherwise CTA u runs unit u alone.
-    int n_units;
-    int *work_counter;
     float sl2;  // softmax_scale * log2(e)
     unsigned long long timeout_ns;
     // Failure-detection test hook, compiled only into the test build (YR_FAULT_HOOKS):
@@ -118,12 +111,6 @@ struct PrefillSmem {
     uint64_t k_full[kKStages], k_empty[kKStages];
     uint64_t v_full[kVStages], v_empty[kVStages];
     uint64_t s_full[kQTiles], p_full[kQTiles], o_done[kQTiles];
-    // Between units: Q_t's buffer may be reloaded once its unit's last S_t is done
-    // (q_free), O_t overwritten once the epilogue has read it (o_free).  The producer
-    // hands every unit (or the end marker -1) to the other roles through a two-slot ring.
-    uint64_t q_free[kQTiles], o_free[kQTiles];
-    uint64_t item_full[2], item_empty[2];
-    int item[2];
     // Q rotation: per softmax warp, the angle (turns, reduced) of each pair at the
     // warp's first row, and the pair's rotations per position in fp32.
     float q_base[8][kMaxPairs], q_turn[8][kMaxPairs];
@@ -188,56 +175,6 @@ __device__ __forceinline__ bool tile_full(const PrefillParams &p, int r_lo, int 
     return true;
 }
 
-// One work unit: a 256-row query block of one (batch, head), or one share of its key
-// tiles under split-KV.
-struct Unit {
-    int b, h, kvh, split;
-    int r_lo[kQTiles], r_hi[kQTiles];  // query positions of the two tiles (r_lo > r_hi: none)
-    TilePlan tp;
-};
-
-// Unit u in launch order.  With grouped heads: one (batch, KV head) after another,
-// its query blocks heaviest first and the query heads of its group adjacent, so the
-// CTAs working at any time read the K/V of one or two KV heads, which stay in L2.
-// Otherwise heaviest causal blocks first, the heads of one query block adjacent.  The
-// shares of one item are adjacent.
-__device__ __forceinline__ Unit unit_at(const PrefillParams &p, int u) {
-    Unit un;
-    un.split = p.n_split > 1 ? u % p.n_split : 0;
-    const int item = p.n_split > 1 ? u / p.n_split : u;
-    int qb;
-    if (p.kv_major) {
-        const int per_kv = p.n_qblocks * p.group;
-        const int bk = item / per_kv;
-        const int rem = item % per_kv;
-        qb = p.n_qblocks - 1 - rem / p.group;
-        un.b = bk / p.Hkv;
-        un.h = (bk % p.Hkv) * p.group + rem % p.group;
-    } else {
-        const int bh_count = p.B * p.Hq;
-        qb = p.n_qblocks - 1 - item / bh_count;
-        const int rem = item % bh_count;
-        un.b = rem / p.Hq;
-        un.h = rem % p.Hq;
-    }
-    un.kvh = un.h / p.group;
-    // Query tiles by position: row r of the query tensor sits at position q_off + r.
-    const int q0 = p.q_off + qb * (kQTiles * kBlockM);
-    const int last_pos = min(q0 + kQTiles * kBlockM - 1, p.q_off + p.T - 1);
-    un.tp = plan_tiles(p, q0, last_pos);
-    if (p.n_split > 1) {
-        const int per = (un.tp.n + p.n_split - 1) / p.n_split;
-        un.tp.first = min(un.split * per, un.tp.n);
-        un.tp.n = min(per, un.tp.n - un.tp.first);
-    }
-#pragma unroll
-    for (int t = 0; t < kQTiles; ++t) {
-        un.r_lo[t] = q0 + t * kBlockM;
-        un.r_hi[t] = min(un.r_lo[t] + kBlockM - 1, last_pos);
-    }
-    return un;
-}
-
 // Bits 0..min(c, 31) set (0 for c < 0): columns at or below c of a 32-column word.
 __device__ __forceinline__ uint32_t cols_upto(int c) {
     if (c < 0) return 0u;
@@ -277,7 +214,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
         : "memory");
 }
 
-template <int HD>
+template <int HD, bool kHalfPairs>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_attn_kernel(const __grid_constant__ PrefillParams p) {
     using Smem = PrefillSmem<HD>;
@@ -288,6 +225,46 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    // Split-KV: the shares of one item are adjacent CTAs.
+    const int split = p.n_split > 1 ? static_cast<int>(blockIdx.x) % p.n_split : 0;
+    const int item = p.n_split > 1 ? static_cast<int>(blockIdx.x) / p.n_split
+                                   : static_cast<int>(blockIdx.x);
+    int qb, b, h;
+    if (p.kv_major) {
+        // Grouped heads: one (batch, KV head) after another, its query blocks
+        // heaviest first and the query heads of its group adjacent, so the CTAs
+        // resident at any time read the K/V of one or two KV heads, which stay in L2.
+        const int per_kv = p.n_qblocks * p.group;
+        const int bk = item / per_kv;
+        const int rem = item % per_kv;
+        qb = p.n_qblocks - 1 - rem / p.group;
+        b = bk / p.Hkv;
+        h = (bk % p.Hkv) * p.group + rem % p.group;
+    } else {
+        // Heaviest causal blocks first, the heads of one query block adjacent.
+        const int bh_count = p.B * p.Hq;
+        qb = p.n_qblocks - 1 - item / bh_count;
+        const int rem = item % bh_count;
+        b = rem / p.Hq;
+        h = rem % p.Hq;
+    }
+    const int kvh = h / p.group;
+    // Query tiles by position: row r of the query tensor sits at position q_off + r.
+    const int q0 = p.q_off + qb * (kQTiles * kBlockM);
+    const int last_pos = min(q0 + kQTiles * kBlockM - 1, p.q_off + p.T - 1);
+    TilePlan tp = plan_tiles(p, q0, last_pos);
+    if (p.n_split > 1) {
+        const int per = (tp.n + p.n_split - 1) / p.n_split;
+        tp.first = min(split * per, tp.n);
+        tp.n = min(per, tp.n - tp.first);
+    }
+    int r_lo[kQTiles], r_hi[kQTiles];
+#pragma unroll
+    for (int t = 0; t < kQTiles; ++t) {
+        r_lo[t] = q0 + t * kBlockM;
+        r_hi[t] = min(r_lo[t] + kBlockM - 1, last_pos);
+    }
+
     if (threadIdx.x == 0) {
         for (int t = 0; t < kQTiles; ++t) {
             mbar_init(&sm->q_full[t], 1);
@@ -295,12 +272,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             mbar_init(&sm->s_full[t], 1);
             mbar_init(&sm->p_full[t], kBlockM / 32);
             mbar_init(&sm->o_done[t], 1);
-            mbar_init(&sm->q_free[t], 1);
-            mbar_init(&sm->o_free[t], kBlockM / 32);
-        }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&sm->item_full[s], 1);
-            mbar_init(&sm->item_empty[s], 1 + 2 * kBlockM / 32);  // MMA warp + softmax warps
         }
         for (int s = 0; s < kKStages; ++s) {
             mbar_init(&sm->k_full[s], 1);
@@ -338,62 +309,35 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const uint64_t pol_q = l2_policy_evict_first();
             const uint64_t pol_kv = l2_policy_evict_last();
             bool ok = true;
-            uint32_t n_pub = 0, kc = 0, vc = 0;  // units published, K and V tiles loaded
-            int qc[kQTiles] = {0, 0};             // loads of each Q tile
+            for (int t = 0; t < kQTiles; ++t) {
+                if (r_lo[t] > r_hi[t]) continue;
+                mbar_arrive_expect_tx(&sm->q_full[t], kSub * kSubTileBytes);
+                for (int s = 0; s < kSub; ++s)
+                    tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64, r_lo[t] - p.q_off, h,
+                                b, pol_q);
+            }
+            const int kv_plane = b * p.Hkv + kvh;
             int issued_k[kKStages] = {}, issued_v[kVStages] = {};
-            for (;;) {
-                int u = p.work_counter != nullptr ? atomicAdd(p.work_counter, 1)
-                                                  : (n_pub == 0 ? static_cast<int>(blockIdx.x)
-                                                                : p.n_units);
-                if (u >= p.n_units) u = -1;
-                const int slot = n_pub & 1;
-                ok = mbar_wait(&sm->item_empty[slot], ((n_pub >> 1) & 1) ^ 1, abort, p.timeout_ns);
-                if (!ok) break;
-                sm->item[slot] = u;
-                mbar_arrive(&sm->item_full[slot]);
-                ++n_pub;
-                if (u < 0) break;
-                const Unit un = unit_at(p, u);
-                for (int t = 0; t < kQTiles && ok; ++t) {
-                    if (un.r_lo[t] > un.r_hi[t]) continue;
-                    // the previous unit's last S_t has read this buffer
-                    ok = mbar_wait(&sm->q_free[t], (qc[t] & 1) ^ 1, abort, p.timeout_ns);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(&sm->q_full[t], kSub * kSubTileBytes);
-                    for (int s = 0; s < kSub; ++s)
-                        tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64,
-                                    un.r_lo[t] - p.q_off, un.h, un.b, pol_q);
-                    ++qc[t];
-                }
-                const int kv_plane = un.b * p.Hkv + un.kvh;
-                for (int idx = 0; idx < un.tp.n && ok; ++idx) {
-                    const int j = tile_at(un.tp, idx);
-                    const int ks = kc % kKStages, vs = vc % kVStages;
+            for (int idx = 0; idx < tp.n && ok; ++idx) {
+                const int j = tile_at(tp, idx);
+                const int ks = idx % kKStages, vs = idx % kVStages;
 #ifdef YR_FAULT_HOOKS
-                    if (idx == p.fault_drop_tile && blockIdx.x == 0 && n_pub == 1) {
-                        ++kc;
-                        ++vc;
-                        continue;
-                    }
+                if (idx == p.fault_drop_tile && blockIdx.x == 0) continue;
 #endif
-                    ok = mbar_wait(&sm->k_empty[ks], ((kc / kKStages) & 1) ^ 1, abort, p.timeout_ns);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(&sm->k_full[ks], kSub * kSubTileBytes);
-                    for (int s = 0; s < kSub; ++s)
-                        tma_load_3d(sm->k[ks][s], &p.tm_k, &sm->k_full[ks], s * 64, j * kBlockN,
-                                    kv_plane, pol_kv);
-                    ++issued_k[ks];
-                    ++kc;
-                    ok = mbar_wait(&sm->v_empty[vs], ((vc / kVStages) & 1) ^ 1, abort, p.timeout_ns);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(&sm->v_full[vs], kSub * kSubTileBytes);
-                    for (int s = 0; s < kSub; ++s)
-                        tma_load_3d(sm->v[vs][s], &p.tm_v, &sm->v_full[vs], s * 64, j * kBlockN,
-                                    kv_plane, pol_kv);
-                    ++issued_v[vs];
-                    ++vc;
-                }
+                ok = mbar_wait(&sm->k_empty[ks], ((idx / kKStages) & 1) ^ 1, abort, p.timeout_ns);
                 if (!ok) break;
+                mbar_arrive_expect_tx(&sm->k_full[ks], kSub * kSubTileBytes);
+                for (int s = 0; s < kSub; ++s)
+                    tma_load_3d(sm->k[ks][s], &p.tm_k, &sm->k_full[ks], s * 64, j * kBlockN,
+                                kv_plane, pol_kv);
+                ++issued_k[ks];
+                ok = mbar_wait(&sm->v_empty[vs], ((idx / kVStages) & 1) ^ 1, abort, p.timeout_ns);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&sm->v_full[vs], kSub * kSubTileBytes);
+                for (int s = 0; s < kSub; ++s)
+                    tma_load_3d(sm->v[vs][s], &p.tm_v, &sm->v_full[vs], s * 64, j * kBlockN,
+                                kv_plane, pol_kv);
+                ++issued_v[vs];
             }
             if (!ok) {
                 raise_status(kStatusTimeoutLoad);
@@ -402,7 +346,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             // Drain: every copy this thread issued must land before the CTA exits.
             bool drained = true;
             for (int t = 0; t < kQTiles; ++t)
-                if (qc[t]) drained &= mbar_wait_drain(&sm->q_full[t], (qc[t] - 1) & 1, p.timeout_ns);
+                if (r_lo[t] <= r_hi[t]) drained &= mbar_wait_drain(&sm->q_full[t], 0, p.timeout_ns);
             for (int s = 0; s < kKStages; ++s)
                 if (issued_k[s])
                     drained &= mbar_wait_drain(&sm->k_full[s], (issued_k[s] - 1) & 1, p.timeout_ns);
@@ -426,139 +370,87 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const uint64_t desc_k = sw128_desc(smem_u32(sm->k[0][0]), 16, 1024);
         const uint64_t desc_v = sw128_desc(smem_u32(sm->v[0][0]), kSubTileBytes, 1024);
         bool ok = true;
-        uint32_t n_con = 0, kc = 0, vc = 0;  // units taken, K and V tiles consumed
-        int qc[kQTiles] = {0, 0};             // rotated Q tiles waited for
-        int pv_total[kQTiles] = {0, 0};       // PV_t issued (phases of p_full / o_done)
-        int o_units[kQTiles] = {0, 0};        // units whose O_t the epilogue has read
-        for (;;) {
-            const int slot = n_con & 1;
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(&sm->item_full[slot], (n_con >> 1) & 1, abort, p.timeout_ns));
-            if (!ok) break;
-            const int u = sm->item[slot];
-            __syncwarp();
-            if (leader) mbar_arrive(&sm->item_empty[slot]);
-            ++n_con;
-            if (u < 0) break;
-            const Unit un = unit_at(p, u);
-            bool live[kQTiles], vis[kQTiles];
-            int last_s[kQTiles];  // plan index of the unit's last S_t (-1: none)
-            int pv_unit[kQTiles] = {0, 0};
-            for (int t = 0; t < kQTiles; ++t) {
-                live[t] = un.r_lo[t] <= un.r_hi[t];
-                last_s[t] = -1;
-                if (!live[t]) continue;
-                for (int idx = un.tp.n - 1; idx >= 0; --idx)
-                    if (tile_visible(p, un.r_lo[t], un.r_hi[t], tile_at(un.tp, idx))) {
-                        last_s[t] = idx;
-                        break;
-                    }
-            }
-            for (int t = 0; t < kQTiles; ++t)
-                if (ok && live[t]) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(&sm->q_ready[t], qc[t] & 1, abort, p.timeout_ns));
-                    ++qc[t];
+        bool vis[kQTiles];
+        int pv_count[kQTiles] = {0, 0};
+        for (int t = 0; t < kQTiles; ++t)
+            if (ok && r_lo[t] <= r_hi[t])
+                ok = __all_sync(0xffffffffu, mbar_wait(&sm->q_ready[t], 0, abort, p.timeout_ns));
+        tc_fence_after();
+
+        // Descriptors advance by (byte offset >> 4) in their start-address field.
+        auto issue_s = [&](int t, int ks) {
+            const uint64_t da = t == 0 ? desc_q0 : desc_q1;
+            const uint64_t db = desc_k + ((ks * kStageBytes) >> 4);
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * kSubTileBytes + (kk & 3) * 32) >> 4;
+                    mma_ss(tmem + t * kBlockN, da + off, db + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
+                mma_commit(&sm->s_full[t]);
+            }
+            __syncwarp();
+        };
+        auto issue_pv = [&](int t, int vs) -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm->p_full[t], pv_count[t] & 1, abort, p.timeout_ns)))
+                return false;
+            tc_fence_after();
+            const uint64_t db = desc_v + ((vs * kStageBytes) >> 4);
+            const uint32_t first = pv_count[t] > 0 ? 1u : 0u;
+            if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < kBlockN / 16; ++kk)
+                    mma_ts(tmem + 2 * kBlockN + t * HD, tmem + t * kBlockN + kk * 8,
+                           db + ((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : first);
+                mma_commit(&sm->o_done[t]);
+            }
+            __syncwarp();
+            ++pv_count[t];
+            return true;
+        };
+
+        // Tensor-pipe order: S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) ...
+        // S_t(i+1) overwrites the P that PV_t(i) reads; tcgen05 MMAs from one thread
+        // run in issue order, so it is issued right behind PV_t(i), with nothing in
+        // between: the next tile's bookkeeping and its K and V waits are done while
+        // this tile's softmax runs, before the wait for P.
+        if (tp.n > 0) {
+            const int j = tile_at(tp, 0);
+            for (int t = 0; t < kQTiles; ++t) vis[t] = tile_visible(p, r_lo[t], r_hi[t], j);
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm->k_full[0], 0, abort, p.timeout_ns));
+            if (ok) {
+                tc_fence_after();
+                if (vis[0]) issue_s(0, 0);
+                if (vis[1]) issue_s(1, 0);
+                if (leader) mma_commit(&sm->k_empty[0]);
+                __syncwarp();
+            }
+        }
+        for (int idx = 0; idx < tp.n && ok; ++idx) {
+            const int vs = idx % kVStages;
+            const int ks1 = (idx + 1) % kKStages;
+            const bool has_next = idx + 1 < tp.n;
+            bool vis1[kQTiles] = {false, false};
+            if (has_next) {
+                const int j1 = tile_at(tp, idx + 1);
+                for (int t = 0; t < kQTiles; ++t) vis1[t] = tile_visible(p, r_lo[t], r_hi[t], j1);
+            }
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(&sm->v_full[vs], (idx / kVStages) & 1, abort, p.timeout_ns));
+            if (ok && has_next)
+                ok = __all_sync(0xffffffffu, mbar_wait(&sm->k_full[ks1], ((idx + 1) / kKStages) & 1,
+                                                       abort, p.timeout_ns));
             if (!ok) break;
             tc_fence_after();
-
-            // Descriptors advance by (byte offset >> 4) in their start-address field.
-            auto issue_s = [&](int t, int ks, int idx) {
-                const uint64_t da = t == 0 ? desc_q0 : desc_q1;
-                const uint64_t db = desc_k + ((ks * kStageBytes) >> 4);
-                if (leader) {
-#pragma unroll
-                    for (int kk = 0; kk < HD / 16; ++kk) {
-                        const uint32_t off = ((kk >> 2) * kSubTileBytes + (kk & 3) * 32) >> 4;
-                        mma_ss(tmem + t * kBlockN, da + off, db + off, idesc_s, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&sm->s_full[t]);
-                    // the unit's last S_t: Q_t's buffer is free once it completes
-                    if (idx == last_s[t]) mma_commit(&sm->q_free[t]);
-                }
-                __syncwarp();
-            };
-            auto issue_pv = [&](int t, int vs) -> bool {
-                // The unit's first PV_t overwrites O_t: the previous unit's epilogue must
-                // have read it.
-                if (pv_unit[t] == 0 && o_units[t] > 0 &&
-                    !__all_sync(0xffffffffu, mbar_wait(&sm->o_free[t], (o_units[t] - 1) & 1, abort,
-                                                       p.timeout_ns)))
-                    return false;
-                if (!__all_sync(0xffffffffu, mbar_wait(&sm->p_full[t], pv_total[t] & 1, abort, p.timeout_ns)))
-                    return false;
-                tc_fence_after();
-                const uint64_t db = desc_v + ((vs * kStageBytes) >> 4);
-                const uint32_t first = pv_unit[t] > 0 ? 1u : 0u;
-                if (leader) {
-#pragma unroll
-                    for (int kk = 0; kk < kBlockN / 16; ++kk)
-                        mma_ts(tmem + 2 * kBlockN + t * HD, tmem + t * kBlockN + kk * 8,
-                               db + ((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : first);
-                    mma_commit(&sm->o_done[t]);
-                }
-                __syncwarp();
-                ++pv_total[t];
-                ++pv_unit[t];
-                return true;
-            };
-
-            // Tensor-pipe order: S0(0) S1(0) | PV0(0) S0(1) PV1(0) S1(1) | PV0(1) S0(2) ...
-            // S_t(i+1) overwrites the P that PV_t(i) reads; tcgen05 MMAs from one thread
-            // run in issue order, so it is issued right behind PV_t(i), with nothing in
-            // between: the next tile's bookkeeping and its K and V waits are done while
-            // this tile's softmax runs, before the wait for P.
-            if (un.tp.n > 0) {
-                const int j = tile_at(un.tp, 0);
-                for (int t = 0; t < kQTiles; ++t) vis[t] = tile_visible(p, un.r_lo[t], un.r_hi[t], j);
-                const int ks = kc % kKStages;
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait(&sm->k_full[ks], (kc / kKStages) & 1, abort, p.timeout_ns));
-                if (ok) {
-                    tc_fence_after();
-                    if (vis[0]) issue_s(0, ks, 0);
-                    if (vis[1]) issue_s(1, ks, 0);
-                    if (leader) mma_commit(&sm->k_empty[ks]);
-                    __syncwarp();
-                    ++kc;
-                }
-            }
-            for (int idx = 0; idx < un.tp.n && ok; ++idx) {
-                const int vs = vc % kVStages;
-                const int ks1 = kc % kKStages;
-                const bool has_next = idx + 1 < un.tp.n;
-                bool vis1[kQTiles] = {false, false};
-                if (has_next) {
-                    const int j1 = tile_at(un.tp, idx + 1);
-                    for (int t = 0; t < kQTiles; ++t)
-                        vis1[t] = tile_visible(p, un.r_lo[t], un.r_hi[t], j1);
-                }
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait(&sm->v_full[vs], (vc / kVStages) & 1, abort, p.timeout_ns));
-                if (ok && has_next)
-                    ok = __all_sync(0xffffffffu, mbar_wait(&sm->k_full[ks1], (kc / kKStages) & 1,
-                                                           abort, p.timeout_ns));
-                if (!ok) break;
-                tc_fence_after();
-                if (vis[0] && !(ok = issue_pv(0, vs))) break;
-                if (vis1[0]) issue_s(0, ks1, idx + 1);
-                if (vis[1] && !(ok = issue_pv(1, vs))) break;
-                if (leader) mma_commit(&sm->v_empty[vs]);
-                ++vc;
-                if (vis1[1]) issue_s(1, ks1, idx + 1);
-                if (leader && has_next) mma_commit(&sm->k_empty[ks1]);
-                if (has_next) ++kc;
-                __syncwarp();
-                vis[0] = vis1[0];
-                vis[1] = vis1[1];
-            }
-            if (!ok) break;
-            for (int t = 0; t < kQTiles; ++t) {
-                // A live Q tile with no S in this unit still hands its buffer back.
-                if (live[t] && last_s[t] < 0 && leader) mma_commit(&sm->q_free[t]);
-                if (pv_unit[t] > 0) ++o_units[t];
-            }
+            if (vis[0] && !(ok = issue_pv(0, vs))) break;
+            if (vis1[0]) issue_s(0, ks1);
+            if (vis[1] && !(ok = issue_pv(1, vs))) break;
+            if (leader) mma_commit(&sm->v_empty[vs]);
+            if (vis1[1]) issue_s(1, ks1);
+            if (leader && has_next) mma_commit(&sm->k_empty[ks1]);
             __syncwarp();
+            vis[0] = vis1[0];
+            vis[1] = vis1[1];
         }
         if (!ok) {
             if (leader) {
@@ -576,40 +468,23 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // ------------------------------------------------- softmax warpgroups
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
         const int t = warp >> 2;
+        const int my_lo = t == 0 ? r_lo[0] : r_lo[1];
+        const int my_hi = t == 0 ? r_hi[0] : r_hi[1];
         const int lane_base = (warp & 3) * 32;
         const int r = lane_base + lane;  // row within the tile = TMEM lane
+        const int pos = my_lo + r;       // position of this thread's query row
+        const int row = pos - p.q_off;   // its index in the query tensor
         const uint32_t tm_lane = static_cast<uint32_t>(lane_base) << 16;
         const uint32_t tm_s = tmem + tm_lane + t * kBlockN;
         const uint32_t tm_o = tmem + tm_lane + 2 * kBlockN + t * HD;
-        const float sl2 = p.sl2;
+        const bool tile_live = my_lo <= my_hi;
         bool ok = true;
-        uint32_t n_con = 0;  // units taken
-        int qc = 0;          // Q_t loads waited for
-        int it = 0;          // S_t tiles processed (phases of s_full / p_full / o_done)
-        for (;;) {
-            const int slot = n_con & 1;
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(&sm->item_full[slot], (n_con >> 1) & 1, abort, p.timeout_ns));
-            if (!ok) break;
-            const int u = sm->item[slot];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm->item_empty[slot]);
-            ++n_con;
-            if (u < 0) break;
-            const Unit un = unit_at(p, u);
-            const int b = un.b, h = un.h, split = un.split;
-            const TilePlan &tp = un.tp;
-            const int my_lo = t == 0 ? un.r_lo[0] : un.r_lo[1];
-            const int my_hi = t == 0 ? un.r_hi[0] : un.r_hi[1];
-            const int pos = my_lo + r;      // position of this thread's query row
-            const int row = pos - p.q_off;  // its index in the query tensor
-            const bool tile_live = my_lo <= my_hi;
 
-            if (tile_live) {
-                // Rotate this row of Q in shared memory: bf16 in, fp16 out, in place.
-                ok = __all_sync(0xffffffffu, mbar_wait(&sm->q_full[t], qc & 1, abort, p.timeout_ns));
-                ++qc;
-                if (!ok) break;
+        if (tile_live) {
+            // Rotate this row of Q in shared memory: bf16 in, fp16 out, in place.
+            ok = mbar_wait(&sm->q_full[t], 0, abort, p.timeout_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
                 float *dbg = (p.q_dbg != nullptr && row < p.T)
                                  ? p.q_dbg + ((static_cast<long long>(b) * p.Hq + h) * p.T + row) * HD
                                  : nullptr;
@@ -638,7 +513,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     return reinterpret_cast<uint4 *>(sm->q[t][g >> 3] + r * 128 +
                                                      (((g & 7) ^ (r & 7)) << 4));
                 };
-                if (p.half_pairs) {
+                if constexpr (kHalfPairs) {
                     // Pairs (i, i + d/2): chunk c holds the first elements of pairs
                     // 8c .. 8c+7, chunk c + d/16 their second elements.
 #pragma unroll 1
@@ -673,13 +548,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         }
                     }
                 } else {
+                    // Pairs (2i, 2i+1): chunk c holds pairs 4c .. 4c+3.
 #pragma unroll 1
-                for (int s = 0; s < kSub; ++s) {
-#pragma unroll 1
-                    for (int c = 0; c < 8; ++c) {
-                        uint4 *ptr = reinterpret_cast<uint4 *>(sm->q[t][s] + r * 128 +
-                                                               ((c ^ (r & 7)) << 4));
-                        uint4 raw = *ptr;
+                    for (int c = 0; c < HD / 8; ++c) {
+                        uint4 *ptr = q_chunk(c);
+                        const uint4 raw = *ptr;
                         const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
                         uint32_t out[4];
                         float y[8];
@@ -688,7 +561,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                             const float a = __uint_as_float(w[pp] << 16);
                             const float bb = __uint_as_float(w[pp] & 0xFFFF0000u);
                             float sn, cs;
-                            pair_sincos(s * 32 + c * 4 + pp, sn, cs);
+                            pair_sincos(c * 4 + pp, sn, cs);
                             y[2 * pp] = a * cs - bb * sn;
                             y[2 * pp + 1] = a * sn + bb * cs;
                             bad |= f16_out_of_range(y[2 * pp]) | f16_out_of_range(y[2 * pp + 1]);
@@ -696,231 +569,222 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         }
                         *ptr = make_uint4(out[0], out[1], out[2], out[3]);
                         if (dbg) {
-                            float4 *d4 = reinterpret_cast<float4 *>(dbg + s * 64 + c * 8);
+                            float4 *d4 = reinterpret_cast<float4 *>(dbg + c * 8);
                             d4[0] = make_float4(y[0], y[1], y[2], y[3]);
                             d4[1] = make_float4(y[4], y[5], y[6], y[7]);
                         }
                     }
-                }
                 }
                 if (__any_sync(0xffffffffu, bad) && lane == 0) raise_status(kStatusRange);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm->q_ready[t]);
             }
+        }
 
-            // ALiBi slope of this head, m_h = 2^(-8 (h+1) / Hq), over the softmax scale.
-            const float alibi_coef =
-                p.alibi ? exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(p.Hq)) *
-                              1.4426950408889634f / p.sl2
-                        : 0.0f;
-            float m_run = -INFINITY;  // reference max of this row, log2 units (score * sl2)
-            float l_run = 0.0f;       // sum of exp2(score * sl2 - m_run) so far
-            int it_unit = 0;          // tiles of this unit processed
-            for (int idx = 0; idx < tp.n && ok && tile_live; ++idx) {
-                const int j = tile_at(tp, idx);
-                if (!tile_visible(p, my_lo, my_hi, j)) continue;
-                ok = mbar_wait(&sm->s_full[t], it & 1, abort, p.timeout_ns);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-                tc_fence_after();
-                float s[kBlockN];
-                {
-                    uint32_t raw[kBlockN / 32][32];
-#pragma unroll
-                    for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tm_s + c * 32, raw[c]);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int c = 0; c < kBlockN / 32; ++c) {
-                        reg_fence32(raw[c]);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[c][e]);
-                    }
-                }
-                if (p.alibi) {
-                    // ALiBi: logit - m_h (pos - n), folded into the raw score as
-                    // s + (m_h / softmax_scale) (n - pos).  Far keys get a large negative
-                    // score whose rounding does not matter: their weight is ~0.
-                    const float b0 = alibi_coef * static_cast<float>(j * kBlockN - pos);
-#pragma unroll
-                    for (int c = 0; c < kBlockN; ++c) s[c] += fmaf(alibi_coef, static_cast<float>(c), b0);
-                }
-                if (!tile_full(p, my_lo, my_hi, j)) {
-                    // Visible columns of this row as a bit mask: c <= c_hi (causal, in range)
-                    // and (c >= c_lo or c < c_sink) (window, sinks); one select per score.
-                    const int k0 = j * kBlockN;
-                    int c_hi = p.Tk - 1 - k0;
-                    if (p.causal) c_hi = min(c_hi, pos - k0);
-                    const int c_lo = p.window > 0 ? pos - p.window + 1 - k0 : -(1 << 30);
-                    const int c_sink = p.window > 0 ? p.n_sink - k0 : -(1 << 30);
-#pragma unroll
-                    for (int w32 = 0; w32 < kBlockN / 32; ++w32) {
-                        const uint32_t vis = cols_upto(c_hi - 32 * w32) &
-                                             (~cols_upto(c_lo - 1 - 32 * w32) | cols_upto(c_sink - 1 - 32 * w32));
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (!((vis >> e) & 1u)) s[w32 * 32 + e] = -INFINITY;
-                    }
-                }
-                auto exps_to_tmem = [&](float m_ref_in) -> float {
-                    // Scalar FMAs feed the scalar ex2 (measured on sm_100a, a packed f32x2
-                    // FMA there costs about twice as many cycles per element); the row
-                    // sums take packed adds.
-                    const float m_ref = (m_ref_in == -INFINITY) ? 0.0f : m_ref_in;
-                    const float neg_m = -m_ref;
-                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int c = 0; c < kBlockN / 32; ++c) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const float p0 = ex2(fmaf(s[c * 32 + 2 * e], sl2, neg_m));
-                            const float p1 = ex2(fmaf(s[c * 32 + 2 * e + 1], sl2, neg_m));
-                            add_f32x2(acc[(2 * e) & 7], acc[(2 * e + 1) & 7], p0, p1);
-                            pk[e] = pack_half2(p0, p1);
-                        }
-                        tmem_st16(tm_s + c * 16, pk);
-                    }
-                    return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-                };
-                // A row with a reference max takes its exponentials against it without
-                // looking at this tile's max: P only has to fit fp16, and since every
-                // p <= l_tile, l_tile <= kPBound proves it does.  A row with no reference
-                // yet tries 0 (log2 units) and keeps it when kBlockN <= l_tile <= kPBound:
-                // then its largest p is at least 1, as with the exact max, so the small p
-                // keep the precision they would have had.
-                // Rows that fail, in warps where any row fails, take the tile max, move
-                // their reference to it and redo P (rare: a row's running max grows
-                // slowly, and typical scores pass the first test).
-                const bool fresh = m_run == -INFINITY;
-                float l_tile = exps_to_tmem(m_run);  // reference 0 for a fresh row
-                bool over = fresh ? !(l_tile >= static_cast<float>(kBlockN) && l_tile <= kPBound)
-                                  : !(l_tile <= kPBound);
-                if (fresh && !over) m_run = 0.0f;
-                if (__any_sync(0xffffffffu, over)) {
-                    // Tile max in four independent chains of three-input max: s[0..3] start
-                    // the chains, s[4..123] go eight per step, s[124..127] close them.
-                    static_assert(kBlockN % 8 == 0, "tile max covers the tile in steps of 8");
-                    float m4[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-                    for (int c = 4; c + 8 <= kBlockN - 4; c += 8) {
-                        m4[0] = fmax3(m4[0], s[c], s[c + 1]);
-                        m4[1] = fmax3(m4[1], s[c + 2], s[c + 3]);
-                        m4[2] = fmax3(m4[2], s[c + 4], s[c + 5]);
-                        m4[3] = fmax3(m4[3], s[c + 6], s[c + 7]);
-                    }
-                    m4[0] = fmax3(m4[0], s[kBlockN - 4], s[kBlockN - 3]);
-                    m4[1] = fmax3(m4[1], s[kBlockN - 2], s[kBlockN - 1]);
-                    const float m_tile = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * sl2;
-                    const bool first = m_run == -INFINITY;
-                    const bool move = first || (over && m_tile > m_run);
-                    const float m_new = move ? fmaxf(m_run, m_tile) : m_run;
-                    const bool rescale = !first && m_new > m_run;
-                    const float alpha = rescale ? ex2(m_run - m_new) : 1.0f;
-                    tmem_st_wait();
-                    l_tile = exps_to_tmem(m_new);
-                    if (it_unit > 0 && __any_sync(0xffffffffu, rescale)) {
-                        // O holds P V up to the previous tile: wait for it, then rescale.
-                        ok = mbar_wait(&sm->o_done[t], (it - 1) & 1, abort, p.timeout_ns);
-                        ok = __all_sync(0xffffffffu, ok);
-                        if (!ok) break;
-                        tc_fence_after();
-                        uint32_t raw[32];
-#pragma unroll
-                        for (int c = 0; c < HD / 32; ++c) {
-                            tmem_ld32_sync(tm_o + c * 32, raw);
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
-                            tmem_st32(tm_o + c * 32, raw);
-                        }
-                    }
-                    // Rows seen for the first time have O = 0 and l = 0: nothing to rescale.
-                    l_run *= alpha;
-                    m_run = m_new;
-                }
-                l_run += l_tile;
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm->p_full[t]);
-                ++it;
-                ++it_unit;
-            }
+        // ALiBi slope of this head, m_h = 2^(-8 (h+1) / Hq), over the softmax scale.
+        const float alibi_coef =
+            p.alibi ? exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(p.Hq)) *
+                          1.4426950408889634f / p.sl2
+                    : 0.0f;
+        float m_run = -INFINITY;  // reference max of this row, log2 units (score * sl2)
+        float l_run = 0.0f;       // sum of exp2(score * sl2 - m_run) so far
+        int it = 0;
+        const float sl2 = p.sl2;
+        for (int idx = 0; idx < tp.n && ok && tile_live; ++idx) {
+            const int j = tile_at(tp, idx);
+            if (!tile_visible(p, my_lo, my_hi, j)) continue;
+            ok = mbar_wait(&sm->s_full[t], it & 1, abort, p.timeout_ns);
+            ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
-            // Epilogue: O / l -> bf16 (or fp32), and the log-sum-exp in natural-log units.
-            const long long orow_idx =
-                (static_cast<long long>(b) * p.Hq + h) * p.T + row + split * p.split_rows;
-            if (ok && tile_live && it_unit > 0) {
-                ok = mbar_wait(&sm->o_done[t], (it - 1) & 1, abort, p.timeout_ns);
-                ok = __all_sync(0xffffffffu, ok);
-                if (ok) {
+            tc_fence_after();
+            float s[kBlockN];
+            {
+                uint32_t raw[kBlockN / 32][32];
+#pragma unroll
+                for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tm_s + c * 32, raw[c]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < kBlockN / 32; ++c) {
+                    reg_fence32(raw[c]);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[c][e]);
+                }
+            }
+            if (p.alibi) {
+                // ALiBi: logit - m_h (pos - n), folded into the raw score as
+                // s + (m_h / softmax_scale) (n - pos).  Far keys get a large negative
+                // score whose rounding does not matter: their weight is ~0.
+                const float b0 = alibi_coef * static_cast<float>(j * kBlockN - pos);
+#pragma unroll
+                for (int c = 0; c < kBlockN; ++c) s[c] += fmaf(alibi_coef, static_cast<float>(c), b0);
+            }
+            if (!tile_full(p, my_lo, my_hi, j)) {
+                // Visible columns of this row as a bit mask: c <= c_hi (causal, in range)
+                // and (c >= c_lo or c < c_sink) (window, sinks); one select per score.
+                const int k0 = j * kBlockN;
+                int c_hi = p.Tk - 1 - k0;
+                if (p.causal) c_hi = min(c_hi, pos - k0);
+                const int c_lo = p.window > 0 ? pos - p.window + 1 - k0 : -(1 << 30);
+                const int c_sink = p.window > 0 ? p.n_sink - k0 : -(1 << 30);
+#pragma unroll
+                for (int w32 = 0; w32 < kBlockN / 32; ++w32) {
+                    const uint32_t vis = cols_upto(c_hi - 32 * w32) &
+                                         (~cols_upto(c_lo - 1 - 32 * w32) | cols_upto(c_sink - 1 - 32 * w32));
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (!((vis >> e) & 1u)) s[w32 * 32 + e] = -INFINITY;
+                }
+            }
+            auto exps_to_tmem = [&](float m_ref_in) -> float {
+                // Scalar FMAs feed the scalar ex2 (measured on sm_100a, a packed f32x2
+                // FMA there costs about twice as many cycles per element); the row
+                // sums take packed adds.
+                const float m_ref = (m_ref_in == -INFINITY) ? 0.0f : m_ref_in;
+                const float neg_m = -m_ref;
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c = 0; c < kBlockN / 32; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = ex2(fmaf(s[c * 32 + 2 * e], sl2, neg_m));
+                        const float p1 = ex2(fmaf(s[c * 32 + 2 * e + 1], sl2, neg_m));
+                        add_f32x2(acc[(2 * e) & 7], acc[(2 * e + 1) & 7], p0, p1);
+                        pk[e] = pack_half2(p0, p1);
+                    }
+                    tmem_st16(tm_s + c * 16, pk);
+                }
+                return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+            };
+            // A row with a reference max takes its exponentials against it without
+            // looking at this tile's max: P only has to fit fp16, and since every
+            // p <= l_tile, l_tile <= kPBound proves it does.  A row with no reference
+            // yet tries 0 (log2 units) and keeps it when kBlockN <= l_tile <= kPBound:
+            // then its largest p is at least 1, as with the exact max, so the small p
+            // keep the precision they would have had.
+            // Rows that fail, in warps where any row fails, take the tile max, move
+            // their reference to it and redo P (rare: a row's running max grows
+            // slowly, and typical scores pass the first test).
+            const bool fresh = m_run == -INFINITY;
+            float l_tile = exps_to_tmem(m_run);  // reference 0 for a fresh row
+            bool over = fresh ? !(l_tile >= static_cast<float>(kBlockN) && l_tile <= kPBound)
+                              : !(l_tile <= kPBound);
+            if (fresh && !over) m_run = 0.0f;
+            if (__any_sync(0xffffffffu, over)) {
+                // Tile max in four independent chains of three-input max: s[0..3] start
+                // the chains, s[4..123] go eight per step, s[124..127] close them.
+                static_assert(kBlockN % 8 == 0, "tile max covers the tile in steps of 8");
+                float m4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+                for (int c = 4; c + 8 <= kBlockN - 4; c += 8) {
+                    m4[0] = fmax3(m4[0], s[c], s[c + 1]);
+                    m4[1] = fmax3(m4[1], s[c + 2], s[c + 3]);
+                    m4[2] = fmax3(m4[2], s[c + 4], s[c + 5]);
+                    m4[3] = fmax3(m4[3], s[c + 6], s[c + 7]);
+                }
+                m4[0] = fmax3(m4[0], s[kBlockN - 4], s[kBlockN - 3]);
+                m4[1] = fmax3(m4[1], s[kBlockN - 2], s[kBlockN - 1]);
+                const float m_tile = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * sl2;
+                const bool first = m_run == -INFINITY;
+                const bool move = first || (over && m_tile > m_run);
+                const float m_new = move ? fmaxf(m_run, m_tile) : m_run;
+                const bool rescale = !first && m_new > m_run;
+                const float alpha = rescale ? ex2(m_run - m_new) : 1.0f;
+                tmem_st_wait();
+                l_tile = exps_to_tmem(m_new);
+                if (it > 0 && __any_sync(0xffffffffu, rescale)) {
+                    // O holds P V up to the previous tile: wait for it, then rescale.
+                    ok = mbar_wait(&sm->o_done[t], (it - 1) & 1, abort, p.timeout_ns);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
                     tc_fence_after();
-                    const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
-                    __nv_bfloat16 *orow = p.o + b * p.osb + h * p.osh + static_cast<long long>(row) * p.ost;
                     uint32_t raw[32];
 #pragma unroll
                     for (int c = 0; c < HD / 32; ++c) {
                         tmem_ld32_sync(tm_o + c * 32, raw);
-                        if (row < p.T && p.o32 != nullptr) {
-                            float4 *dst = reinterpret_cast<float4 *>(p.o32 + orow_idx * HD + c * 32);
 #pragma unroll
-                            for (int q4 = 0; q4 < 8; ++q4)
-                                dst[q4] = make_float4(__uint_as_float(raw[4 * q4]) * inv_l,
-                                                      __uint_as_float(raw[4 * q4 + 1]) * inv_l,
-                                                      __uint_as_float(raw[4 * q4 + 2]) * inv_l,
-                                                      __uint_as_float(raw[4 * q4 + 3]) * inv_l);
-                        } else if (row < p.T) {
-#pragma unroll
-                            for (int q4 = 0; q4 < 4; ++q4) {
-                                uint32_t pk[4];
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    __nv_bfloat162 v2 = __floats2bfloat162_rn(
-                                        __uint_as_float(raw[q4 * 8 + 2 * e]) * inv_l,
-                                        __uint_as_float(raw[q4 * 8 + 2 * e + 1]) * inv_l);
-                                    pk[e] = *reinterpret_cast<uint32_t *>(&v2);
-                                }
-                                *reinterpret_cast<uint4 *>(orow + c * 32 + q4 * 8) =
-                                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                            }
-                        }
+                        for (int e = 0; e < 32; ++e)
+                            raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
+                        tmem_st32(tm_o + c * 32, raw);
                     }
-                    if (p.lse != nullptr && row < p.T) {
-                        const float m_ref = (m_run == -INFINITY) ? 0.0f : m_run;
-                        p.lse[orow_idx] = (l_run > 0.0f) ? (m_ref + __log2f(l_run)) * 0.69314718055994531f
-                                                         : -INFINITY;
-                    }
-                } else {
-                    raise_status(kStatusTimeoutSoftmax);
-                    sm->abort = 1;
                 }
-            } else if (ok && tile_live && row < p.T) {
-                // No key of this call is visible to the whole query tile (possible only when
-                // the keys are one block of a longer sequence): o = 0, lse = -inf.
-                if (p.o32 != nullptr) {
-                    float4 *dst = reinterpret_cast<float4 *>(p.o32 + orow_idx * HD);
-#pragma unroll 1
-                    for (int c = 0; c < HD / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-                } else {
-                    __nv_bfloat16 *orow = p.o + b * p.osb + h * p.osh + static_cast<long long>(row) * p.ost;
-#pragma unroll 1
-                    for (int c = 0; c < HD / 8; ++c)
-                        *reinterpret_cast<uint4 *>(orow + c * 8) = make_uint4(0u, 0u, 0u, 0u);
-                }
-                if (p.lse != nullptr) p.lse[orow_idx] = -INFINITY;
+                // Rows seen for the first time have O = 0 and l = 0: nothing to rescale.
+                l_run *= alpha;
+                m_run = m_new;
             }
-            if (!ok) break;
-            if (tile_live && it_unit > 0) {
-                // O_t has been read: the next unit's first PV_t may overwrite it.
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm->o_free[t]);
-            }
+            l_run += l_tile;
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm->p_full[t]);
+            ++it;
         }
         if (!ok) {
             raise_status(kStatusTimeoutSoftmax);
             sm->abort = 1;
+        }
+        // Epilogue: O / l -> bf16 (or fp32), and the log-sum-exp in natural-log units.
+        const long long orow_idx =
+            (static_cast<long long>(b) * p.Hq + h) * p.T + row + split * p.split_rows;
+        if (ok && tile_live && it > 0) {
+            ok = mbar_wait(&sm->o_done[t], (it - 1) & 1, abort, p.timeout_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                tc_fence_after();
+                const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
+                __nv_bfloat16 *orow = p.o + b * p.osb + h * p.osh + static_cast<long long>(row) * p.ost;
+                uint32_t raw[32];
+#pragma unroll
+                for (int c = 0; c < HD / 32; ++c) {
+                    tmem_ld32_sync(tm_o + c * 32, raw);
+                    if (row < p.T && p.o32 != nullptr) {
+                        float4 *dst = reinterpret_cast<float4 *>(p.o32 + orow_idx * HD + c * 32);
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4)
+                            dst[q4] = make_float4(__uint_as_float(raw[4 * q4]) * inv_l,
+                                                  __uint_as_float(raw[4 * q4 + 1]) * inv_l,
+                                                  __uint_as_float(raw[4 * q4 + 2]) * inv_l,
+                                                  __uint_as_float(raw[4 * q4 + 3]) * inv_l);
+                    } else if (row < p.T) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                __nv_bfloat162 v2 = __floats2bfloat162_rn(
+                                    __uint_as_float(raw[q4 * 8 + 2 * e]) * inv_l,
+                                    __uint_as_float(raw[q4 * 8 + 2 * e + 1]) * inv_l);
+                                pk[e] = *reinterpret_cast<uint32_t *>(&v2);
+                            }
+                            *reinterpret_cast<uint4 *>(orow + c * 32 + q4 * 8) =
+                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
+                }
+                if (p.lse != nullptr && row < p.T) {
+                    const float m_ref = (m_run == -INFINITY) ? 0.0f : m_run;
+                    p.lse[orow_idx] = (l_run > 0.0f) ? (m_ref + __log2f(l_run)) * 0.69314718055994531f
+                                                     : -INFINITY;
+                }
+            } else {
+                raise_status(kStatusTimeoutSoftmax);
+                sm->abort = 1;
+            }
+        } else if (ok && tile_live && row < p.T) {
+            // No key of this call is visible to the whole query tile (possible only when
+            // the keys are one block of a longer sequence): o = 0, lse = -inf.
+            if (p.o32 != nullptr) {
+                float4 *dst = reinterpret_cast<float4 *>(p.o32 + orow_idx * HD);
+#pragma unroll 1
+                for (int c = 0; c < HD / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+                __nv_bfloat16 *orow = p.o + b * p.osb + h * p.osh + static_cast<long long>(row) * p.ost;
+#pragma unroll 1
+                for (int c = 0; c < HD / 8; ++c)
+                    *reinterpret_cast<uint4 *>(orow + c * 8) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            if (p.lse != nullptr) p.lse[orow_idx] = -INFINITY;
         }
     }
 

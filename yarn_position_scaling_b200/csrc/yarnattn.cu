@@ -134,9 +134,13 @@ int prepare_device(int *sm_count, DeviceState *out = nullptr) {
                 const void *fn;
                 size_t bytes;
             } attrs[] = {
-                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128>),
+                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, false>),
                  yr::prefill_smem_bytes<128>()},
-                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64>),
+                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, true>),
+                 yr::prefill_smem_bytes<128>()},
+                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, false>),
+                 yr::prefill_smem_bytes<64>()},
+                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, true>),
                  yr::prefill_smem_bytes<64>()},
                 {reinterpret_cast<const void *>(&yr::decode_split_kernel<128, 1>),
                  yr::decode_smem_bytes<128>()},
@@ -155,8 +159,10 @@ int prepare_device(int *sm_count, DeviceState *out = nullptr) {
             // The prefill kernel re-splits its registers between warpgroups
             // (setmaxnreg); that only works if the launch reserves enough of them.
             st.prefill_regs_ok = true;
-            for (const void *fn : {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128>),
-                                   reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64>)}) {
+            for (const void *fn : {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, false>),
+                                   reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, true>),
+                                   reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, false>),
+                                   reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, true>)}) {
                 cudaFuncAttributes fa;
                 e = cudaFuncGetAttributes(&fa, fn);
                 if (e != cudaSuccess) return cuda_fail("cudaFuncGetAttributes", e);
@@ -209,14 +215,9 @@ int encode(CUtensorMap *map, CUtensorMapDataType dt, int rank, const void *base,
     return YR_OK;
 }
 
-// Prefill workspace: the rotated keys and the values in fp16, then 256 bytes that hold
-// the work counter of the persistent attention grid.
-constexpr size_t kCounterBytes = 256;
-size_t prefill_planes_bytes(long long B, long long Hkv, long long T, long long d) {
-    return static_cast<size_t>(2 * B * Hkv * T * d * 2);
-}
+// Prefill workspace: the rotated keys and the values in fp16.
 size_t prefill_ws_bytes(long long B, long long Hkv, long long T, long long d) {
-    return prefill_planes_bytes(B, Hkv, T, d) + kCounterBytes;
+    return static_cast<size_t>(2 * B * Hkv * T * d * 2);
 }
 
 // Partial-result slots per (b, KV head): a block of the balanced split holds at least
@@ -363,20 +364,15 @@ int launch_prepare(const void *k, const void *v, void *k_cache, float *k_rot_dbg
 
 // The fp16 rotated keys and values the attention kernel reads: planes of ld16 rows
 // of d elements, one per (b, KV head), keys [0, Tk) of each.
-// `counter` (nullable): device int the persistent grid takes work units from.
 struct KvPlanes {
     const __half *k16;
     const __half *v16;
     long long ld16;
-    int *counter;
 };
-// The layout of a prefill workspace: K [B*Hkv][Tk][d], then V the same, then the
-// counter.
+// The layout of a prefill workspace: K [B*Hkv][Tk][d], then V the same.
 KvPlanes workspace_planes(const void *workspace, int B, int Hkv, int Tk, int d) {
     const __half *k16 = static_cast<const __half *>(workspace);
-    int *counter = reinterpret_cast<int *>(static_cast<char *>(const_cast<void *>(workspace)) +
-                                           prefill_planes_bytes(B, Hkv, Tk, d));
-    return {k16, k16 + static_cast<size_t>(B) * Hkv * Tk * d, Tk, counter};
+    return {k16, k16 + static_cast<size_t>(B) * Hkv * Tk * d, Tk};
 }
 
 // T query rows against the Tk keys of `kv`.  Key n sits at position k_pos0 + n and
@@ -431,7 +427,7 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     // so that re-reads hit L2 (measured: +2.7% at the 128K GQA workload, neutral for MHA).
     pp.kv_major = pp.group > 1 ? 1 : 0;
     pp.alibi = tab->method == YR_ALIBI ? 1 : 0;
-    pp.half_pairs = tab->pairs == YR_PAIR_HALF ? 1 : 0;
+    const bool half = tab->pairs == YR_PAIR_HALF;
     pp.sl2 = static_cast<float>(tab->softmax_scale * 1.4426950408889634);
     pp.timeout_ns = wait_timeout_ns();
 #ifdef YR_FAULT_HOOKS
@@ -442,22 +438,19 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     pp.fault_drop_tile = -1;
 #endif
     for (int i = 0; i < d / 2; ++i) pp.turns[i] = tab->turns[i];
-    const long long n_units = static_cast<long long>(B) * Hq * pp.n_qblocks * n_split;
-    pp.n_units = static_cast<int>(n_units);
-    // Persistent grid: one CTA per SM (the kernel needs a whole SM's TMEM and most of its
-    // shared memory), each taking units from the counter until none is left.
-    pp.work_counter = kv.counter;
-    unsigned grid = static_cast<unsigned>(n_units);
-    if (kv.counter != nullptr) {
-        if (n_units > ds.sm_count) grid = static_cast<unsigned>(ds.sm_count);
-        cudaError_t me = cudaMemsetAsync(kv.counter, 0, sizeof(int), st);
-        if (me != cudaSuccess) return cuda_fail("cudaMemsetAsync(work counter)", me);
-    }
-    if (d == 128)
-        yr::prefill_attn_kernel<128>
+    const unsigned grid =
+        static_cast<unsigned>(static_cast<long long>(B) * Hq * pp.n_qblocks * n_split);
+    if (d == 128 && !half)
+        yr::prefill_attn_kernel<128, false>
             <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<128>(), st>>>(pp);
+    else if (d == 128)
+        yr::prefill_attn_kernel<128, true>
+            <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<128>(), st>>>(pp);
+    else if (!half)
+        yr::prefill_attn_kernel<64, false>
+            <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<64>(), st>>>(pp);
     else
-        yr::prefill_attn_kernel<64>
+        yr::prefill_attn_kernel<64, true>
             <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<64>(), st>>>(pp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("prefill_attn_kernel launch", e);
@@ -561,7 +554,7 @@ int chunk_call(const char *fn, const void *q, const void *k_new, const void *v_n
                void *k_cache, void *v_cache, void *o, float *lse, int B, int Hq, int Hkv,
                int Tq, int d, int P0, int T_max, const yr_rope_table *tab, int window,
                int n_sink, __half *k16, __half *v16, long long ld16, int first,
-               int *counter, void *split_ws, size_t split_ws_bytes, void *stream) {
+               void *split_ws, size_t split_ws_bytes, void *stream) {
     const std::string f(fn);
     if (!q || !k_new || !v_new || !k_cache || !v_cache || !o || !tab)
         return fail(YR_EINVAL, f + ": NULL pointer argument");
@@ -612,7 +605,7 @@ int chunk_call(const char *fn, const void *q, const void *k_new, const void *v_n
     const int n_split = split_ws ? choose_split(sm_count, B, Hq, Tq, P0, window, split_ws_bytes,
                                                 share)
                                  : 1;
-    const KvPlanes kv{k16, v16, ld16, counter};
+    const KvPlanes kv{k16, v16, ld16};
     if (n_split == 1)
         return launch_attend(q, o, lse, nullptr, B, Hq, Hkv, Tq, d, qs, os, tab, 1, window,
                              n_sink, kv, st, Tk, P0);
@@ -662,12 +655,12 @@ extern "C" int yr_attn_prefill_chunk(const void *q, const void *k_new, const voi
     const KvPlanes kv = workspace_planes(workspace, B, Hkv, Tk, d);
     return chunk_call(fn, q, k_new, v_new, k_cache, v_cache, o, lse, B, Hq, Hkv, Tq, d, P0,
                       T_max, tab, window, n_sink, const_cast<__half *>(kv.k16),
-                      const_cast<__half *>(kv.v16), Tk, 0, kv.counter, nullptr, 0, stream);
+                      const_cast<__half *>(kv.v16), Tk, 0, nullptr, 0, stream);
 }
 
 extern "C" size_t yr_attn_prefill_chunk_split_bytes(int B, int Hq, int Tq, int d) {
     if (B < 1 || Hq < 1 || Tq < 1 || (d != 64 && d != 128)) return 0;
-    return kCounterBytes + kMaxSplit * split_share_bytes(B, Hq, Tq, d);
+    return kMaxSplit * split_share_bytes(B, Hq, Tq, d);
 }
 
 extern "C" int yr_attn_prefill_chunk_fp16cache(const void *q, const void *k_new,
@@ -688,14 +681,10 @@ extern "C" int yr_attn_prefill_chunk_fp16cache(const void *q, const void *k_new,
         return fail(YR_EINVAL, std::string(fn) + ": need 0 <= cache16_len <= P0");
     if (workspace && !aligned(workspace, 256))
         return fail(YR_EINVAL, std::string(fn) + ": workspace must be 256-byte aligned");
-    // The workspace starts with the work counter; the split partials follow it.
-    const bool has_ws = workspace != nullptr && workspace_bytes >= kCounterBytes;
-    int *counter = has_ws ? static_cast<int *>(workspace) : nullptr;
-    void *split_ws = has_ws ? static_cast<char *>(workspace) + kCounterBytes : nullptr;
     return chunk_call(fn, q, k_new, v_new, k_cache, v_cache, o, lse, B, Hq, Hkv, Tq, d, P0,
                       T_max, tab, window, n_sink, static_cast<__half *>(k_cache16),
-                      static_cast<__half *>(v_cache16), T_max, cache16_len, counter, split_ws,
-                      has_ws ? workspace_bytes - kCounterBytes : 0, stream);
+                      static_cast<__half *>(v_cache16), T_max, cache16_len, workspace,
+                      workspace ? workspace_bytes : 0, stream);
 }
 
 extern "C" int yr_prefill_prepare_kv_at(const void *k, const void *v, void *k_cache,
