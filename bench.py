@@ -72,9 +72,9 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {
-    "prefill_attn_kernel<128>": ["prefill_sm100.cuh"],
-    "kv_prep_kernel": ["kvprep_sm100.cuh"],
-    "decode_split_kernel<128,1>": ["decode_sm100.cuh"],
+    "prefill_attn_kernel<128, false>": ["prefill_sm100.cuh"],
+    "kv_prep_kernel<false>": ["kvprep_sm100.cuh"],
+    "decode_split_kernel<128, 1>": ["decode_sm100.cuh"],
 }
 
 
@@ -628,14 +628,14 @@ def main():
                    "l2": "no flush: q+k+v+o = %.0f MB per step > 126 MB L2" %
                          ((2 * wp.B * wp.Hq + 2 * wp.B * wp.Hkv) * wp.T * wp.d * 2 / 2 ** 20),
                    "step": "yr_prefill_prepare_kv + yr_prefill_attend (= yr_attn_prefill)"},
-        "roofline": {"bound": "tensor", "kernel": "prefill_attn_kernel<128>",
+        "roofline": {"bound": "tensor", "kernel": "prefill_attn_kernel<128, false>",
                      "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": attn_tflops / peak_t,
                      "peak_source": f"{peak_src} bf16 "
                                     f"{'sustained' if long_step else 'burst'} (of {peak_src}; "
                                     "the fp16 tensor rate equals bf16)",
                      "frac_of_burst": attn_tflops / peak_burst, "peak_burst": peak_burst,
-                     "traffic": ncu_traffic("prefill_attn_kernel<128>"),
+                     "traffic": ncu_traffic("prefill_attn_kernel<128, false>"),
                      "algorithmic_flops_per_launch": flops_step,
                      "kernel_ms": attn_ms_max / steps,
                      "kv_prep_ms": prep_ms_max / steps},
@@ -651,11 +651,11 @@ def main():
             "metric": "decode KV-read GB/s", "value": d_gbs, "unit": "GB/s", "steps": dsteps,
             "ms_per_step": dtotal_ms / dsteps, "workload": wd.name,
             "cache_len": lens,
-            "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<128,1> + merge",
+            "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<128, 1> + merge",
                          "achieved": d_call_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": d_call_gbs / peaks["hbm_gbs"],
                          "peak_source": f"{peak_src} HBM copy",
-                         "traffic": ncu_traffic("decode_split_kernel<128,1>"),
+                         "traffic": ncu_traffic("decode_split_kernel<128, 1>"),
                          "algorithmic_bytes_per_launch": dbytes}}, 5),
     }
     if dist.rank == 0:

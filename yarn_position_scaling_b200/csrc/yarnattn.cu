@@ -532,9 +532,12 @@ size_t split_share_bytes(long long B, long long Hq, long long Tq, long long d) {
     return static_cast<size_t>(B * Hq * Tq * (d + 1) * 4);
 }
 
-// Shares per item for a prefill of Tq query rows after P0 cached keys: enough CTAs
-// for two waves when the items alone are too few, each share at least 4 key tiles,
-// at most kMaxSplit and at most what the split workspace holds.
+// Shares per item for a prefill of Tq query rows after P0 cached keys, when the items
+// alone leave SMs idle.  Each CTA holds a whole SM, so the grid runs in waves of
+// sm_count CTAs, and a share costs its key tiles plus a CTA's fixed cost (set-up, Q
+// rotation, epilogue: about five tiles' time): the count with the least
+// waves x (tiles per share + 5) wins.  Each share keeps at least 4 key tiles; at most kMaxSplit shares
+// and at most what the split workspace holds.
 constexpr int kMaxSplit = 16;
 int choose_split(int sm_count, int B, int Hq, int Tq, int P0, int window, size_t ws_bytes,
                  size_t share_bytes) {
@@ -543,11 +546,22 @@ int choose_split(int sm_count, int B, int Hq, int Tq, int P0, int window, size_t
     int keys = P0 + (Tq < 256 ? Tq : 256);  // the first query block's keys (the fewest)
     if (window > 0 && window < keys) keys = window + 256;
     const int tiles = (keys + 127) / 128;
-    long long s = (2ll * sm_count + items - 1) / items;
-    if (s > kMaxSplit) s = kMaxSplit;
-    if (s > tiles / 4) s = tiles / 4;
-    if (s > static_cast<long long>(ws_bytes / share_bytes)) s = ws_bytes / share_bytes;
-    return s < 2 ? 1 : static_cast<int>(s);
+    long long s_max = kMaxSplit;
+    if (s_max > tiles / 4) s_max = tiles / 4;
+    if (s_max > static_cast<long long>(ws_bytes / share_bytes)) s_max = ws_bytes / share_bytes;
+    // Time of a split in tile steps: waves x (tiles of a share + the fixed cost).
+    int best = 1;
+    double best_time = 0.0;
+    for (long long s = 1; s <= s_max || s == 1; ++s) {
+        const long long waves = (items * s + sm_count - 1) / sm_count;
+        const double time = static_cast<double>(waves) *
+                            (static_cast<double>(tiles) / static_cast<double>(s) + 5.0);
+        if (s == 1 || time < best_time * 0.9999) {
+            best_time = time;
+            best = static_cast<int>(s);
+        }
+    }
+    return best;
 }
 
 int chunk_call(const char *fn, const void *q, const void *k_new, const void *v_new,
