@@ -426,7 +426,7 @@ def chunk_fp16cache_bench(w, Tq, steps, stream, dist, peak_t):
     return {"tflops": tf, "frac": tf / peak_t, "ms": call_ms / steps}
 
 
-def ring_bench(w, world, steps, stream, dist, peak_t):
+def ring_bench(w, world, steps, stream, dist, peak_t, layout="contiguous"):
     """Ring attention over `world` ranks emulated in one process on this GPU: every rank's
     block kernels (keys prepared at their positions, one attention call per visible
     block, fp32 partials folded by the log-sum-exp merge) run in turn, without the
@@ -440,7 +440,8 @@ def ring_bench(w, world, steps, stream, dist, peak_t):
         e = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
         with torch.cuda.stream(stream):
             e[0].record(stream)
-            ring.ring_prefill_emulated(q, k, v, tab, world, w.causal, w.window, w.n_sink)
+            ring.ring_prefill_emulated(q, k, v, tab, world, w.causal, w.window, w.n_sink,
+                                       layout=layout)
             e[1].record(stream)
         return [(e[0], e[1])]
 
@@ -454,7 +455,10 @@ def ring_bench(w, world, steps, stream, dist, peak_t):
     call_ms = dist.max(call_ms)
     flops = metrics.prefill_flops(w.B, w.Hq, w.T, w.d, w.causal, w.window, w.n_sink)
     tf = flops / (call_ms / steps * 1e-3) / 1e12
-    return {"ranks_emulated": world, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "method": w.method,
+    # causal work per rank in (query chunk, key chunk) pairs: the multi-GPU balance
+    work = [len(ring.rank_pairs(r, world, layout, w.causal)) for r in range(world)]
+    return {"ranks_emulated": world, "layout": layout,
+            "rank_work_max_over_mean": max(work) / (sum(work) / world), "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "method": w.method,
             "flops_per_step": flops, "steps": steps, "call_ms": call_ms / steps,
             "call_tflops": tf, "frac_of_peak": tf / peak_t,
             "timed_over": "all ranks' block preparation, block attention and merge launches, "
@@ -462,9 +466,10 @@ def ring_bench(w, world, steps, stream, dist, peak_t):
 
 
 def e2e_prefill(w, steps, warmup, stream):
-    """Through the public API with host buffers: `api.HostPrefill` takes pinned host q, k, v
-    and returns the pinned host output; the H2D copies, the kernels and the D2H copy of
-    each (batch, KV-head group) unit overlap those of the other units."""
+    """Through the C ABI's host-buffer entry point (yr_host_prefill_run, wrapped by
+    `api.HostPrefill`): pinned host q, k, v in, the pinned host output out; the H2D copies,
+    the kernels and the D2H copy of each (batch, KV-head group) unit overlap those of the
+    other units."""
     from yarn_position_scaling_b200 import api
     qh, kh, vh = [t.pin_memory() for t in synth.prefill_inputs(w, "cpu")]
     oh = torch.empty(qh.shape, dtype=torch.bfloat16).pin_memory()
@@ -569,10 +574,12 @@ def main():
             synth.CHUNK, 256, max(args.other_steps, 10), stream, dist, peak_burst)
         torch.cuda.empty_cache()
         wr = synth.LLAMA3_128K
-        r = ring_bench(wr, 8, args.other_steps, stream, dist, peak_burst)
-        others["ring_128k_8_emulated_ranks"] = {"tflops": r["call_tflops"],
-                                                "frac": r["frac_of_peak"]}
-        torch.cuda.empty_cache()
+        for layout in ("contiguous", "zigzag"):
+            r = ring_bench(wr, 8, args.other_steps, stream, dist, peak_burst, layout)
+            others[f"ring_128k_8_emulated_{layout}"] = {
+                "tflops": r["call_tflops"], "frac": r["frac_of_peak"],
+                "rank_work_max_over_mean": r["rank_work_max_over_mean"]}
+            torch.cuda.empty_cache()
         w16 = synth.LLAMA2_16K
         r = workload_prefill(w16, max(args.other_steps, 20), stream, dist, peak_burst)
         prefill_16k = {"workload": w16.name, "step_tflops": r["step_tflops"],
@@ -644,7 +651,9 @@ def main():
         "clocks": clk,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": esteps,
-                "path": "api.HostPrefill: pinned host q/k/v in, pinned host o out"},
+                "path": "yr_host_prefill_run (C ABI, through api.HostPrefill): pinned host "
+                        "q/k/v in, pinned host o out, copies and kernels overlapped per "
+                        "(batch, KV-head group)"},
         "other_workloads": _r(others, 4),
         "prefill_16k": _r(prefill_16k, 5),
         "decode": _r({

@@ -184,3 +184,26 @@ def test_merge_kernel_against_numpy(d, init):
     ob = to_f64(out)
     np.testing.assert_allclose(ob[live], got_o[live], rtol=2.0 ** -8, atol=1e-6)
     assert np.all(ob[both_empty] == 0.0)
+
+
+@pytest.mark.parametrize("world,T,window,n_sink", [(2, 512, 0, 0), (4, 1024, 0, 0),
+                                                   (4, 1024, 300, 4)])
+def test_zigzag_ring_matches_oracle(world, T, window, n_sink):
+    # zigzag layout: rank r's queries are chunks r and 2 world - 1 - r of T / (2 world)
+    w = dataclasses.replace(synth.LLAMA3_128K, Hq=8, Hkv=2)
+    q, k, v = synth.prefill_inputs(w, "cuda", T=T)
+    tab, th, ss = _tables(w)
+    outs = ring.ring_prefill_emulated(q, k, v, tab, world, True, window, n_sink,
+                                      layout="zigzag")
+    api.device_status()
+    ro, rl, _ = oracle.attn_rows(to_bits(q), to_bits(k), to_bits(v), th, ss, True, window,
+                                 n_sink)
+    B, Hq, d = q.shape[0], q.shape[1], q.shape[3]
+    ro = torch.from_numpy(ro.reshape(B, Hq, T, d))
+    rl = torch.from_numpy(rl.reshape(B, Hq, T, 1))
+    for rank, (o_r, lse_r) in enumerate(outs):
+        want = ring.zigzag_gather(ro, world, rank).numpy()
+        emax, emean = err_stats(to_f64(o_r), want)
+        assert emax <= O_MAX_ABS and emean <= O_MEAN_ABS, (rank, emax, emean)
+        wl = ring.zigzag_gather(rl, world, rank).numpy()[..., 0]
+        assert err_stats(to_f64(lse_r), wl)[0] <= LSE_ABS

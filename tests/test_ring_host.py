@@ -135,7 +135,7 @@ def _free_port():
     return port
 
 
-def _worker(rank, world, port, causal, window, n_sink, out):
+def _worker(rank, world, port, causal, window, n_sink, out, layout="contiguous"):
     import sys
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
@@ -146,9 +146,13 @@ def _worker(rank, world, port, causal, window, n_sink, out):
         C = CASE["C"]
         th, _, ss = oracle.rope_theta(CASE["d"], CASE["base"], CASE["L_train"], CASE["s"],
                                       CASE["method"])
-        sl = slice(rank * C, (rank + 1) * C)
-        o, lse = ring.ring_prefill(q[:, :, sl], k[:, :, sl], v[:, :, sl], None, causal=causal,
-                                   window=window, n_sink=n_sink, ops=CpuBlockOps(th, ss))
+        if layout == "zigzag":
+            share = [ring.zigzag_gather(x, world, rank) for x in (q, k, v)]
+        else:
+            sl = slice(rank * C, (rank + 1) * C)
+            share = [x[:, :, sl] for x in (q, k, v)]
+        o, lse = ring.ring_prefill(*share, None, causal=causal, window=window, n_sink=n_sink,
+                                   ops=CpuBlockOps(th, ss), layout=layout)
         out.put((rank, o.numpy(), lse.numpy()))
     finally:
         dist.destroy_process_group()
@@ -199,3 +203,46 @@ def test_ring_rejects_unequal_slices():
             ring.ring_prefill(q, k, k, None, ops=CpuBlockOps(np.zeros(8), 1.0))
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,causal,window,n_sink", [
+    (2, True, 0, 0), (3, True, 0, 0), (3, False, 0, 0), (4, True, 30, 3)])
+def test_zigzag_ring_over_gloo_equals_exact_attention(world, causal, window, n_sink):
+    # zigzag layout: rank r holds chunks r and 2 world - 1 - r of C / 2 tokens each
+    ctx = mp.get_context("spawn")
+    qu = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, causal, window, n_sink, qu,
+                                               "zigzag"))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted((qu.get(timeout=180) for _ in range(world)), key=lambda t: t[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    q, k, v = _inputs(world, **CASE)
+    th, _, ss = oracle.rope_theta(CASE["d"], CASE["base"], CASE["L_train"], CASE["s"],
+                                  CASE["method"])
+    ro, rl, _ = oracle.attn_rows(to_bits(q), to_bits(k), to_bits(v), th, ss, causal, window,
+                                 n_sink)
+    B, Hq, d, C = CASE["B"], CASE["Hq"], CASE["d"], CASE["C"]
+    T = world * C
+    ro = torch.from_numpy(ro.reshape(B, Hq, T, d))
+    rl = torch.from_numpy(rl.reshape(B, Hq, T, 1))
+    for rank, o, lse in got:
+        np.testing.assert_allclose(o, ring.zigzag_gather(ro, world, rank).numpy(), atol=1e-10)
+        np.testing.assert_allclose(lse, ring.zigzag_gather(rl, world, rank).numpy()[..., 0],
+                                   atol=1e-10)
+
+
+@pytest.mark.parametrize("world", [2, 4, 8])
+def test_zigzag_balances_causal_work(world):
+    # contiguous slices: rank r attends r + 1 of world blocks; zigzag: every rank attends
+    # 2 world + 1 (query chunk, key chunk) pairs, i.e. the same share of the causal work
+    zz = [len(ring.rank_pairs(r, world, "zigzag")) for r in range(world)]
+    assert zz == [2 * world + 1] * world
+    assert sum(zz) == (2 * world) * (2 * world + 1) // 2   # every causal chunk pair once
+    co = [len(ring.rank_pairs(r, world, "contiguous")) for r in range(world)]
+    assert co == list(range(1, world + 1))
+
