@@ -259,6 +259,17 @@ def oracle_sample(w, seconds: float, seed: int = 0):
     return done_flops, wall, threads, desc
 
 
+def workload_config(w, n: int) -> dict:
+    """The `config` of the JSON line for prefill workload w on n GPUs (both arms)."""
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T,
+            "method": w.method, "base": w.base, "L_train": w.L_train, "scale": w.scale,
+            "causal": w.causal, "window": w.window, "n_sink": w.n_sink, "io_dtype": "bf16",
+            "mma_operands": "fp16", "accumulate": "fp32", "parallelism": f"replicas x{n}",
+            "l2": "no flush: q+k+v+o = %.0f MB per step > 126 MB L2" %
+                  ((2 * w.B * w.Hq + 2 * w.B * w.Hkv) * w.T * w.d * 2 / 2 ** 20),
+            "step": "yr_prefill_prepare_kv + yr_prefill_attend (= yr_attn_prefill)"}
+
+
 def reference_arm(args, dist: Dist):
     w = synth.ALL[args.headline]
     line = {"impl": "reference"}
@@ -280,9 +291,7 @@ def reference_arm(args, dist: Dist):
         "n_gpus": 1, "steps": steps, "warmup": warm, "ms_per_step": wall / steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic N(0,1) bf16 inputs, seeded",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T,
-                   "method": w.method, "base": w.base, "L_train": w.L_train, "scale": w.scale,
-                   "causal": True, "parallelism": "replicas"},
+        "config": workload_config(w, 1),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": f"each step ~{per_step:.1f}s of oracle work: {desc}"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -627,14 +636,7 @@ def main():
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp16",
         "data": "synthetic: seeded i.i.d. N(0,1) inputs rounded to bf16",
-        "config": {"workload": wp.name, "B": wp.B, "Hq": wp.Hq, "Hkv": wp.Hkv, "d": wp.d,
-                   "T": wp.T, "method": wp.method, "base": wp.base, "L_train": wp.L_train,
-                   "scale": wp.scale, "causal": wp.causal, "window": wp.window,
-                   "n_sink": wp.n_sink, "io_dtype": "bf16", "mma_operands": "fp16",
-                   "accumulate": "fp32", "parallelism": f"replicas x{n}",
-                   "l2": "no flush: q+k+v+o = %.0f MB per step > 126 MB L2" %
-                         ((2 * wp.B * wp.Hq + 2 * wp.B * wp.Hkv) * wp.T * wp.d * 2 / 2 ** 20),
-                   "step": "yr_prefill_prepare_kv + yr_prefill_attend (= yr_attn_prefill)"},
+        "config": workload_config(wp, n),
         "roofline": {"bound": "tensor", "kernel": "prefill_attn_kernel<128, false>",
                      "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": attn_tflops / peak_t,
