@@ -249,3 +249,27 @@ def test_fp16cache_split_kv_against_the_oracle_and_unsplit(P0, Tq, window, n_sin
     a, b = o.float(), o1.float()
     assert torch.all((a - b).abs() <= b.abs() * 2.0 ** -8 + 2e-3)
     assert torch.equal(kc, kc2) and torch.equal(k16, k16b)
+
+
+def test_fp16cache_alibi_and_range_check():
+    # ALiBi through the fp16-copy form; a prefix value past the fp16 limit in the slots the
+    # call converts is reported as YR_ERANGE
+    w = dataclasses.replace(SMALL, method="alibi")
+    P0, Tq, T_max = 3000, 100, 3100
+    q, kn, vn, kc, vc = synth.chunk_inputs(w, "cuda", P0=P0, Tq=Tq, T_max=T_max)
+    kc0, vc0 = to_bits(kc), to_bits(vc)
+    tab = api.rope_freq_table(w.d, w.base, w.L_train, w.scale, "alibi")
+    k16 = torch.zeros(kc.shape, dtype=torch.float16, device="cuda")
+    v16 = torch.zeros(vc.shape, dtype=torch.float16, device="cuda")
+    o = api.attn_prefill_chunk_fp16cache(q, kn, vn, kc, vc, k16, v16, 0, P0, tab)
+    api.device_status()
+    ro, _, _ = oracle.prefill_chunk(to_bits(q), to_bits(kn), to_bits(vn), kc0, vc0, P0,
+                                    np.zeros(w.d // 2), 1.0 / np.sqrt(w.d),
+                                    slopes=oracle.alibi_slopes(w.Hq))
+    emax, emean = err_stats(to_f64(o), ro)
+    assert emax <= O_MAX_ABS and emean <= O_MEAN_ABS, (emax, emean)
+    vc[0, 1, 17, 3] = 70000.0
+    api.attn_prefill_chunk_fp16cache(q, kn, vn, kc, vc, k16, v16, 10, P0, tab)
+    with pytest.raises(api.YarnAttnError) as ei:
+        api.device_status()
+    assert ei.value.code == api.YR_ERANGE
