@@ -68,10 +68,12 @@ struct yr_host_prefill {
     struct Unit {
         int b, kv0, kv1;
         cudaEvent_t arrived = nullptr, computed = nullptr, copied_out = nullptr;
+        // recorded by an earlier call (kept per unit, so that a call that stopped on an
+        // error half-way still orders the next call behind the work it did queue)
+        bool has_computed = false, has_copied_out = false;
     };
     std::vector<Unit> units;
     cudaEvent_t all_out = nullptr;
-    bool ran = false;  // a previous call recorded the per-unit events
 };
 
 namespace {
@@ -163,7 +165,7 @@ extern "C" int yr_host_prefill_run(yr_host_prefill *p, const void *q, const void
         const size_t kv_off = (static_cast<size_t>(u.b) * p->Hkv + u.kv0) * row;
         const size_t kv_len = static_cast<size_t>(nkv) * row;
         // copy-in: once the previous call's kernels on this unit have read its inputs
-        if (p->ran && (e = cudaStreamWaitEvent(p->h2d, u.computed, 0)) != cudaSuccess)
+        if (u.has_computed && (e = cudaStreamWaitEvent(p->h2d, u.computed, 0)) != cudaSuccess)
             return cuda_fail("cudaStreamWaitEvent", e);
         if ((e = cudaMemcpyAsync(p->qd + q_off, static_cast<const char *>(q) + q_off, q_len,
                                  cudaMemcpyHostToDevice, p->h2d)) != cudaSuccess ||
@@ -175,7 +177,7 @@ extern "C" int yr_host_prefill_run(yr_host_prefill *p, const void *q, const void
             return cuda_fail("copy-in", e);
         // kernels: once the inputs have arrived and the previous output has left
         if ((e = cudaStreamWaitEvent(comp, u.arrived, 0)) != cudaSuccess ||
-            (p->ran && (e = cudaStreamWaitEvent(comp, u.copied_out, 0)) != cudaSuccess))
+            (u.has_copied_out && (e = cudaStreamWaitEvent(comp, u.copied_out, 0)) != cudaSuccess))
             return cuda_fail("cudaStreamWaitEvent", e);
         const int rc = yr_attn_prefill(p->qd + q_off, p->kd + kv_off, p->vd + kv_off,
                                        p->od + q_off, nullptr, nullptr, nullptr, nullptr, 1,
@@ -185,14 +187,15 @@ extern "C" int yr_host_prefill_run(yr_host_prefill *p, const void *q, const void
         if (rc != YR_OK) return rc;  // its message is already set
         if ((e = cudaEventRecord(u.computed, comp)) != cudaSuccess)
             return cuda_fail("cudaEventRecord", e);
+        u.has_computed = true;
         // copy-out
         if ((e = cudaStreamWaitEvent(p->d2h, u.computed, 0)) != cudaSuccess ||
             (e = cudaMemcpyAsync(static_cast<char *>(o) + q_off, p->od + q_off, q_len,
                                  cudaMemcpyDeviceToHost, p->d2h)) != cudaSuccess ||
             (e = cudaEventRecord(u.copied_out, p->d2h)) != cudaSuccess)
             return cuda_fail("copy-out", e);
+        u.has_copied_out = true;
     }
-    p->ran = true;
     if ((e = cudaEventRecord(p->all_out, p->d2h)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(comp, p->all_out, 0)) != cudaSuccess)
         return cuda_fail("joining the caller's stream", e);
