@@ -600,16 +600,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             tc_fence_after();
             float s[kBlockN];
             {
-                uint32_t raw[kBlockN / 32][32];
-#pragma unroll
-                for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tm_s + c * 32, raw[c]);
+                // The whole score row in one TMEM load (measured ~1% faster at 128K than
+                // four 32-column loads).
+                static_assert(kBlockN == 128, "one 128-column TMEM load per score row");
+                uint32_t raw[kBlockN];
+                tmem_ld128(tm_s, raw);
                 tmem_ld_wait();
+                reg_fence128(raw);
 #pragma unroll
-                for (int c = 0; c < kBlockN / 32; ++c) {
-                    reg_fence32(raw[c]);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[c][e]);
-                }
+                for (int e = 0; e < kBlockN; ++e) s[e] = __uint_as_float(raw[e]);
             }
             if (p.alibi) {
                 // ALiBi: logit - m_h (pos - n), folded into the raw score as

@@ -169,6 +169,33 @@ __device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
                    "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
                    "+r"(r[30]), "+r"(r[31]));
 }
+// 32 lanes x 32 bits, 128 consecutive columns in one instruction (a whole 128-key
+// score tile of one row per thread).
+#define YR_TM_OUT4(b) "=r"(r[b]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3])
+#define YR_TM_OUT16(b) YR_TM_OUT4(b), YR_TM_OUT4(b + 4), YR_TM_OUT4(b + 8), YR_TM_OUT4(b + 12)
+#define YR_TM_IO4(b) "+r"(r[b]), "+r"(r[b + 1]), "+r"(r[b + 2]), "+r"(r[b + 3])
+#define YR_TM_IO16(b) YR_TM_IO4(b), YR_TM_IO4(b + 4), YR_TM_IO4(b + 8), YR_TM_IO4(b + 12)
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
+        "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,"
+        "%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,"
+        "%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%128];"
+        : YR_TM_OUT16(0), YR_TM_OUT16(16), YR_TM_OUT16(32), YR_TM_OUT16(48), YR_TM_OUT16(64),
+          YR_TM_OUT16(80), YR_TM_OUT16(96), YR_TM_OUT16(112)
+        : "r"(taddr));
+}
+// reg_fence32 for the 128 registers of tmem_ld128.
+__device__ __forceinline__ void reg_fence128(uint32_t (&r)[128]) {
+    asm volatile(""
+                 : YR_TM_IO16(0), YR_TM_IO16(16), YR_TM_IO16(32), YR_TM_IO16(48), YR_TM_IO16(64),
+                   YR_TM_IO16(80), YR_TM_IO16(96), YR_TM_IO16(112));
+}
+#undef YR_TM_OUT4
+#undef YR_TM_OUT16
+#undef YR_TM_IO4
+#undef YR_TM_IO16
 // Load 32 columns and wait for them.
 __device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]) {
     tmem_ld32(taddr, r);
