@@ -336,31 +336,6 @@ int yr_attn_merge(const float *o_part, const float *lse_part, float *o_acc, floa
                   void *o_out, long long rows, int d, int init, void *stream);
 
 /*
- * prefill_attend_block_merge -- yr_prefill_attend_block and yr_attn_merge in one
- * kernel, for ring attention ("long-context-models", context parallelism: each
- * worker folds the block it holds into its running maxima, sums and outputs;
- * "Long context (engineering 100k+ tokens)", sec. 3): the attention kernel's
- * epilogue folds each query row of this block into the running (o_acc, lse_acc)
- * with the same weights and the same operations as yr_attn_merge, so the result is
- * bit-identical to yr_prefill_attend_block into temporaries followed by
- * yr_attn_merge(o_part, lse_part, o_acc, lse_acc, o_out, B * Hq * T, d, init), without
- * writing and re-reading the block's fp32 partial.
- * Arguments: as yr_prefill_attend_block, with o and lse replaced by
- *   o_acc fp32 [B, Hq, T, d] and lse_acc fp32 [B, Hq, T] (contiguous, device, read
- *   and written in place; not read when init != 0), o_out bf16 [B, Hq, T, d]
- *   (contiguous, nullable: the merged rows rounded to bf16, e.g. on the last block),
- *   init 0 or 1.  o_acc and o_out 16-byte aligned, lse_acc 4-byte aligned.
- * Errors: those of yr_prefill_attend_block, and YR_EINVAL for NULL o_acc or
- *   lse_acc, a misaligned o_acc, o_out or lse_acc, or init not 0/1.
- */
-int yr_prefill_attend_block_merge(const void *q, float *o_acc, float *lse_acc, void *o_out,
-                                  int init, int B, int Hq, int Hkv, int T, int Tk, int d,
-                                  const int64_t *q_strides,
-                                  const yr_rope_table *tab, int causal, int window, int n_sink,
-                                  int q_pos0, int k_pos0,
-                                  const void *workspace, size_t workspace_bytes, void *stream);
-
-/*
  * host_prefill -- prefill of prompts that live in host memory: q, k, v are read
  * from host buffers and o is written to a host buffer, with the copies inside the
  * call ("LLM context window mechanics", production lessons: a 128K prompt's first

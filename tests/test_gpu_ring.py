@@ -207,66 +207,3 @@ def test_zigzag_ring_matches_oracle(world, T, window, n_sink):
         assert emax <= O_MAX_ABS and emean <= O_MEAN_ABS, (rank, emax, emean)
         wl = ring.zigzag_gather(rl, world, rank).numpy()[..., 0]
         assert err_stats(to_f64(lse_r), wl)[0] <= LSE_ABS
-
-
-@pytest.mark.parametrize("layout,world,T,causal,window,n_sink,d,Hq,Hkv,pairs", [
-    ("contiguous", 4, 1024, True, 0, 0, 128, 8, 2, "interleaved"),
-    ("contiguous", 4, 1024, True, 300, 4, 128, 8, 2, "interleaved"),
-    ("contiguous", 3, 771, False, 0, 0, 64, 6, 3, "half"),
-    ("zigzag", 4, 1024, True, 0, 0, 128, 8, 2, "interleaved"),
-    ("zigzag", 2, 640, True, 200, 3, 64, 4, 4, "half"),
-])
-def test_fused_block_merge_is_the_separate_calls_bit_for_bit(layout, world, T, causal, window,
-                                                             n_sink, d, Hq, Hkv, pairs):
-    # The fused kernel folds each block into the running rows with the merge kernel's own
-    # operations: every output, every running lse and the final bf16 rows are identical.
-    w = dataclasses.replace(synth.LLAMA3_128K, Hq=Hq, Hkv=Hkv, d=d)
-    q, k, v = synth.prefill_inputs(w, "cuda", T=T)
-    tab = api.rope_freq_table(d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta,
-                              pairs=pairs)
-
-    class Separate(ring.BlockOps):
-        def __getattribute__(self, name):
-            if name == "attend_into":
-                raise AttributeError(name)
-            return super().__getattribute__(name)
-
-    fused = ring.ring_prefill_emulated(q, k, v, tab, world, causal, window, n_sink,
-                                       layout=layout)
-    sep = ring.ring_prefill_emulated(q, k, v, tab, world, causal, window, n_sink,
-                                     ops=Separate(), layout=layout)
-    api.device_status()
-    assert len(fused) == len(sep) == world
-    for (of, lf), (os_, ls) in zip(fused, sep):
-        assert torch.equal(of, os_)
-        assert torch.equal(lf, ls)
-
-
-def test_fused_block_merge_single_blocks_and_empty_rows():
-    # One query block against key blocks it sees wholly, partly, and not at all (rows
-    # before the block under a causal mask, or past a window), folded into a running
-    # result that starts empty, holds some rows, and ends with the bf16 copy.
-    w = dataclasses.replace(synth.LLAMA3_128K, Hq=8, Hkv=2)
-    C = 384
-    q, k, v = synth.prefill_inputs(w, "cuda", T=3 * C)
-    tab, _, _ = _tables(w)
-    ops = ring.BlockOps()
-    blocks = [ops.prepare(k[:, :, i * C:(i + 1) * C], v[:, :, i * C:(i + 1) * C], tab, i * C)
-              for i in range(3)]
-    qb = q[:, :, 2 * C:]
-    for window, n_sink in [(0, 0), (200, 5), (500, 0)]:
-        acc_f, acc_s = ops.new_acc(qb), ops.new_acc(qb)
-        for n, src in enumerate([2, 0, 1]):
-            first, last = n == 0, n == 2
-            o_p, lse_p = api.prefill_attend_block(qb, w.Hkv, C, tab, blocks[src], 2 * C, src * C,
-                                                  True, window, n_sink)
-            api.attn_merge(o_p, lse_p, acc_s[0], acc_s[1], out=acc_s[2] if last else None,
-                           init=first)
-            api.prefill_attend_block_merge(qb, w.Hkv, C, tab, blocks[src], 2 * C, src * C,
-                                           acc_f[0], acc_f[1], True, window, n_sink,
-                                           out=acc_f[2] if last else None, init=first)
-            api.device_status()
-            assert torch.equal(acc_f[1], acc_s[1])
-            live = torch.isfinite(acc_s[1])
-            assert torch.equal(acc_f[0][live], acc_s[0][live])
-        assert torch.equal(acc_f[2], acc_s[2])

@@ -25,7 +25,7 @@ SYMBOLS = ("yr_rope_freq_table", "yr_attn_prefill_workspace_bytes", "yr_attn_pre
            "yr_prefill_prepare_kv", "yr_prefill_attend", "yr_attn_prefill_chunk",
            "yr_attn_prefill_chunk_fp16cache", "yr_attn_prefill_chunk_split_bytes",
            "yr_prefill_prepare_kv_at",
-           "yr_prefill_attend_block", "yr_attn_merge", "yr_prefill_attend_block_merge",
+           "yr_prefill_attend_block", "yr_attn_merge",
            "yr_attn_decode_workspace_bytes", "yr_attn_decode", "yr_attn_decode_noalloc",
            "yr_host_prefill_workspace_bytes", "yr_host_prefill_create", "yr_host_prefill_run",
            "yr_host_prefill_destroy", "yr_device_status", "yr_last_error", "yr_version")
@@ -98,10 +98,6 @@ def load(path: str | None = None, make_default: bool = False) -> ctypes.CDLL:
     lib.yr_prefill_attend_block.restype = ci
     lib.yr_attn_merge.argtypes = [vp] * 5 + [ctypes.c_longlong, ci, ci, vp]
     lib.yr_attn_merge.restype = ci
-    lib.yr_prefill_attend_block_merge.argtypes = ([vp] * 4 + [ci] * 7 + [i64p] +
-                                                  [ctypes.POINTER(RopeTable)] + [ci] * 5 +
-                                                  [vp, cs, vp])
-    lib.yr_prefill_attend_block_merge.restype = ci
     lib.yr_attn_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci]
     lib.yr_attn_decode_workspace_bytes.restype = cs
     lib.yr_attn_decode.argtypes = ([vp] * 9 + [ci] * 5 +
@@ -326,27 +322,6 @@ def attn_merge(o_part, lse_part, o_acc, lse_acc, out=None, init: bool = False, s
             raise ValueError("attn_merge expects contiguous tensors")
     rc = load().yr_attn_merge(_ptr(o_part), _ptr(lse_part), _ptr(o_acc), _ptr(lse_acc),
                               _ptr(out), rows, d, int(bool(init)), _stream(stream))
-    _check(rc)
-    return o_acc, lse_acc
-
-
-def prefill_attend_block_merge(q, Hkv: int, Tk: int, table: RopeTable, workspace, q_pos0: int,
-                               k_pos0: int, o_acc, lse_acc, causal: bool = True, window: int = 0,
-                               n_sink: int = 0, out=None, init: bool = False, stream=None):
-    """prefill_attend_block followed by attn_merge into (o_acc fp32 [B,Hq,T,d], lse_acc fp32
-    [B,Hq,T]) in one kernel; `out` (bf16 [B,Hq,T,d]) optionally receives the merged rows.
-    Bit-identical to the two calls."""
-    B, Hq, T, d = q.shape
-    for t in (o_acc, lse_acc) + ((out,) if out is not None else ()):
-        if not t.is_contiguous():
-            raise ValueError("prefill_attend_block_merge expects contiguous o_acc, lse_acc, out")
-    if o_acc.dtype != torch.float32 or lse_acc.dtype != torch.float32:
-        raise ValueError("prefill_attend_block_merge accumulates in fp32")
-    rc = load().yr_prefill_attend_block_merge(
-        _ptr(q), _ptr(o_acc), _ptr(lse_acc), _ptr(out), int(bool(init)), B, Hq, Hkv, T, int(Tk),
-        d, _strides(q), ctypes.byref(table), int(bool(causal)), int(window), int(n_sink),
-        int(q_pos0), int(k_pos0), _ptr(workspace), workspace.numel() * workspace.element_size(),
-        _stream(stream))
     _check(rc)
     return o_acc, lse_acc
 

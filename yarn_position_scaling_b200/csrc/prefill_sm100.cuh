@@ -98,12 +98,6 @@ struct alignas(64) PrefillParams {
     // CTA 0's producer issues no copy for this key tile index (-1: off), so a wait that
     // nothing will complete runs out of time.
     int fault_drop_tile;
-    // Ring merge (the kMerge instantiation): o32 and lse hold the running output and
-    // log-sum-exp of the rows and are updated in place, the block's rows folded in with
-    // the online-softmax weights; merge_init: the running values are empty (not read);
-    // acc_out: if set, the bf16 copy of the merged rows ([B][Hq][T][d], contiguous).
-    int merge_init;
-    __nv_bfloat16 *acc_out;
     double turns[64];
 };
 
@@ -220,7 +214,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
         : "memory");
 }
 
-template <int HD, bool kHalfPairs, bool kMerge = false>
+template <int HD, bool kHalfPairs>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_attn_kernel(const __grid_constant__ PrefillParams p) {
     using Smem = PrefillSmem<HD>;
@@ -732,135 +726,64 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // Epilogue: O / l -> bf16 (or fp32), and the log-sum-exp in natural-log units.
         const long long orow_idx =
             (static_cast<long long>(b) * p.Hq + h) * p.T + row + split * p.split_rows;
-        if constexpr (kMerge) {
-            // Fold this block's rows into the running ones (ring attention): with
-            // L = log(e^la + e^lb), o <- e^(la - L) o + e^(lb - L) o_b, lse <- L, in the
-            // same operations as the merge kernel, so the result is the same bit for bit
-            // as writing the block's partial and merging it.  A row that saw no key of
-            // this block has lb = -inf and o_b = 0.
-            const bool have_o = ok && tile_live && it > 0;
-            if (have_o) {
-                ok = mbar_wait(&sm->o_done[t], (it - 1) & 1, abort, p.timeout_ns);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) {
-                    raise_status(kStatusTimeoutSoftmax);
-                    sm->abort = 1;
-                } else {
-                    tc_fence_after();
-                }
-            }
-            if (ok && tile_live) {
-                const float m_ref = (m_run == -INFINITY) ? 0.0f : m_run;
-                const bool seen = have_o && l_run > 0.0f;
-                const float lb = seen ? (m_ref + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
-                const float inv_l = seen ? 1.0f / l_run : 0.0f;
-                const bool in_range = row < p.T;
-                const float la = (p.merge_init || !in_range) ? -INFINITY : p.lse[orow_idx];
-                const float mx = fmaxf(la, lb);
-                float ca = 0.0f, cb = 0.0f, l_new = -INFINITY;
-                if (mx > -INFINITY) {
-                    const float wa = expf(la - mx), wb = expf(lb - mx);
-                    const float sum = wa + wb;
-                    l_new = mx + logf(sum);
-                    ca = wa / sum;
-                    cb = wb / sum;
-                }
-                float *acc = p.o32 + orow_idx * HD;
-                __nv_bfloat16 *out = p.acc_out != nullptr ? p.acc_out + orow_idx * HD : nullptr;
+        if (ok && tile_live && it > 0) {
+            ok = mbar_wait(&sm->o_done[t], (it - 1) & 1, abort, p.timeout_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                tc_fence_after();
+                const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
+                __nv_bfloat16 *orow = p.o + b * p.osb + h * p.osh + static_cast<long long>(row) * p.ost;
                 uint32_t raw[32];
-#pragma unroll 1
+#pragma unroll
                 for (int c = 0; c < HD / 32; ++c) {
-                    if (have_o) tmem_ld32_sync(tm_o + c * 32, raw);
-                    if (!in_range) continue;
-                    if (mx > -INFINITY) {
+                    tmem_ld32_sync(tm_o + c * 32, raw);
+                    if (row < p.T && p.o32 != nullptr) {
+                        float4 *dst = reinterpret_cast<float4 *>(p.o32 + orow_idx * HD + c * 32);
 #pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4) {
-                            const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-                            float4 *a4 = reinterpret_cast<float4 *>(acc + c * 32 + q4 * 4);
-                            const float4 a = la > -INFINITY ? *a4 : z;
-                            float bv[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                bv[e] = have_o ? __uint_as_float(raw[4 * q4 + e]) * inv_l : 0.0f;
-                            const float4 r = make_float4(fmaf(ca, a.x, cb * bv[0]), fmaf(ca, a.y, cb * bv[1]),
-                                                         fmaf(ca, a.z, cb * bv[2]), fmaf(ca, a.w, cb * bv[3]));
-                            *a4 = r;
-                            if (out != nullptr) {
-                                __nv_bfloat162 b01 = __floats2bfloat162_rn(r.x, r.y);
-                                __nv_bfloat162 b23 = __floats2bfloat162_rn(r.z, r.w);
-                                *reinterpret_cast<uint2 *>(out + c * 32 + q4 * 4) =
-                                    make_uint2(*reinterpret_cast<uint32_t *>(&b01),
-                                               *reinterpret_cast<uint32_t *>(&b23));
-                            }
-                        }
-                    } else if (out != nullptr) {
-#pragma unroll 1
                         for (int q4 = 0; q4 < 8; ++q4)
-                            *reinterpret_cast<uint2 *>(out + c * 32 + q4 * 4) = make_uint2(0u, 0u);
-                    }
-                }
-                if (in_range) p.lse[orow_idx] = l_new;
-            }
-        } else {
-            if (ok && tile_live && it > 0) {
-                ok = mbar_wait(&sm->o_done[t], (it - 1) & 1, abort, p.timeout_ns);
-                ok = __all_sync(0xffffffffu, ok);
-                if (ok) {
-                    tc_fence_after();
-                    const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
-                    __nv_bfloat16 *orow = p.o + b * p.osb + h * p.osh + static_cast<long long>(row) * p.ost;
-                    uint32_t raw[32];
+                            dst[q4] = make_float4(__uint_as_float(raw[4 * q4]) * inv_l,
+                                                  __uint_as_float(raw[4 * q4 + 1]) * inv_l,
+                                                  __uint_as_float(raw[4 * q4 + 2]) * inv_l,
+                                                  __uint_as_float(raw[4 * q4 + 3]) * inv_l);
+                    } else if (row < p.T) {
 #pragma unroll
-                    for (int c = 0; c < HD / 32; ++c) {
-                        tmem_ld32_sync(tm_o + c * 32, raw);
-                        if (row < p.T && p.o32 != nullptr) {
-                            float4 *dst = reinterpret_cast<float4 *>(p.o32 + orow_idx * HD + c * 32);
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint32_t pk[4];
 #pragma unroll
-                            for (int q4 = 0; q4 < 8; ++q4)
-                                dst[q4] = make_float4(__uint_as_float(raw[4 * q4]) * inv_l,
-                                                      __uint_as_float(raw[4 * q4 + 1]) * inv_l,
-                                                      __uint_as_float(raw[4 * q4 + 2]) * inv_l,
-                                                      __uint_as_float(raw[4 * q4 + 3]) * inv_l);
-                        } else if (row < p.T) {
-#pragma unroll
-                            for (int q4 = 0; q4 < 4; ++q4) {
-                                uint32_t pk[4];
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    __nv_bfloat162 v2 = __floats2bfloat162_rn(
-                                        __uint_as_float(raw[q4 * 8 + 2 * e]) * inv_l,
-                                        __uint_as_float(raw[q4 * 8 + 2 * e + 1]) * inv_l);
-                                    pk[e] = *reinterpret_cast<uint32_t *>(&v2);
-                                }
-                                *reinterpret_cast<uint4 *>(orow + c * 32 + q4 * 8) =
-                                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            for (int e = 0; e < 4; ++e) {
+                                __nv_bfloat162 v2 = __floats2bfloat162_rn(
+                                    __uint_as_float(raw[q4 * 8 + 2 * e]) * inv_l,
+                                    __uint_as_float(raw[q4 * 8 + 2 * e + 1]) * inv_l);
+                                pk[e] = *reinterpret_cast<uint32_t *>(&v2);
                             }
+                            *reinterpret_cast<uint4 *>(orow + c * 32 + q4 * 8) =
+                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         }
                     }
-                    if (p.lse != nullptr && row < p.T) {
-                        const float m_ref = (m_run == -INFINITY) ? 0.0f : m_run;
-                        p.lse[orow_idx] = (l_run > 0.0f) ? (m_ref + __log2f(l_run)) * 0.69314718055994531f
-                                                         : -INFINITY;
-                    }
-                } else {
-                    raise_status(kStatusTimeoutSoftmax);
-                    sm->abort = 1;
                 }
-            } else if (ok && tile_live && row < p.T) {
-                // No key of this call is visible to the whole query tile (possible only when
-                // the keys are one block of a longer sequence): o = 0, lse = -inf.
-                if (p.o32 != nullptr) {
-                    float4 *dst = reinterpret_cast<float4 *>(p.o32 + orow_idx * HD);
-#pragma unroll 1
-                    for (int c = 0; c < HD / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-                } else {
-                    __nv_bfloat16 *orow = p.o + b * p.osb + h * p.osh + static_cast<long long>(row) * p.ost;
-#pragma unroll 1
-                    for (int c = 0; c < HD / 8; ++c)
-                        *reinterpret_cast<uint4 *>(orow + c * 8) = make_uint4(0u, 0u, 0u, 0u);
+                if (p.lse != nullptr && row < p.T) {
+                    const float m_ref = (m_run == -INFINITY) ? 0.0f : m_run;
+                    p.lse[orow_idx] = (l_run > 0.0f) ? (m_ref + __log2f(l_run)) * 0.69314718055994531f
+                                                     : -INFINITY;
                 }
-                if (p.lse != nullptr) p.lse[orow_idx] = -INFINITY;
+            } else {
+                raise_status(kStatusTimeoutSoftmax);
+                sm->abort = 1;
             }
+        } else if (ok && tile_live && row < p.T) {
+            // No key of this call is visible to the whole query tile (possible only when
+            // the keys are one block of a longer sequence): o = 0, lse = -inf.
+            if (p.o32 != nullptr) {
+                float4 *dst = reinterpret_cast<float4 *>(p.o32 + orow_idx * HD);
+#pragma unroll 1
+                for (int c = 0; c < HD / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+                __nv_bfloat16 *orow = p.o + b * p.osb + h * p.osh + static_cast<long long>(row) * p.ost;
+#pragma unroll 1
+                for (int c = 0; c < HD / 8; ++c)
+                    *reinterpret_cast<uint4 *>(orow + c * 8) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            if (p.lse != nullptr) p.lse[orow_idx] = -INFINITY;
         }
     }
 

@@ -142,14 +142,6 @@ int prepare_device(int *sm_count, DeviceState *out = nullptr) {
                  yr::prefill_smem_bytes<64>()},
                 {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, true>),
                  yr::prefill_smem_bytes<64>()},
-                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, false, true>),
-                 yr::prefill_smem_bytes<128>()},
-                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, true, true>),
-                 yr::prefill_smem_bytes<128>()},
-                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, false, true>),
-                 yr::prefill_smem_bytes<64>()},
-                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, true, true>),
-                 yr::prefill_smem_bytes<64>()},
                 {reinterpret_cast<const void *>(&yr::decode_split_kernel<128, 1>),
                  yr::decode_smem_bytes<128>()},
                 {reinterpret_cast<const void *>(&yr::decode_split_kernel<128, 2>),
@@ -170,11 +162,7 @@ int prepare_device(int *sm_count, DeviceState *out = nullptr) {
             for (const void *fn : {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, false>),
                                    reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, true>),
                                    reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, false>),
-                                   reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, true>),
-                                   reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, false, true>),
-                                   reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, true, true>),
-                                   reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, false, true>),
-                                   reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, true, true>)}) {
+                                   reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, true>)}) {
                 cudaFuncAttributes fa;
                 e = cudaFuncGetAttributes(&fa, fn);
                 if (e != cudaSuccess) return cuda_fail("cudaFuncGetAttributes", e);
@@ -393,8 +381,7 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
                   int T, int d, const long long qs[3], const long long os[3],
                   const yr_rope_table *tab, int causal, int window, int n_sink,
                   const KvPlanes &kv, cudaStream_t st, int Tk, int q_off, int k_pos0 = 0,
-                  float *o32 = nullptr, int n_split = 1, bool merge = false, int merge_init = 0,
-                  __nv_bfloat16 *acc_out = nullptr) {
+                  float *o32 = nullptr, int n_split = 1) {
     DeviceState ds;
     int rc = prepare_device(nullptr, &ds);
     if (rc != YR_OK) return rc;
@@ -450,20 +437,21 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
 #else
     pp.fault_drop_tile = -1;
 #endif
-    pp.merge_init = merge_init;
-    pp.acc_out = acc_out;
     for (int i = 0; i < d / 2; ++i) pp.turns[i] = tab->turns[i];
     const unsigned grid =
         static_cast<unsigned>(static_cast<long long>(B) * Hq * pp.n_qblocks * n_split);
-    const size_t smem = d == 128 ? yr::prefill_smem_bytes<128>() : yr::prefill_smem_bytes<64>();
-    // (head size, pair layout, ring merge) -> instantiation
-    void (*kernels[8])(const yr::PrefillParams) = {
-        yr::prefill_attn_kernel<64, false>,        yr::prefill_attn_kernel<64, true>,
-        yr::prefill_attn_kernel<128, false>,       yr::prefill_attn_kernel<128, true>,
-        yr::prefill_attn_kernel<64, false, true>,  yr::prefill_attn_kernel<64, true, true>,
-        yr::prefill_attn_kernel<128, false, true>, yr::prefill_attn_kernel<128, true, true>};
-    kernels[(merge ? 4 : 0) + (d == 128 ? 2 : 0) + (half ? 1 : 0)]
-        <<<grid, yr::kPrefillThreads, smem, st>>>(pp);
+    if (d == 128 && !half)
+        yr::prefill_attn_kernel<128, false>
+            <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<128>(), st>>>(pp);
+    else if (d == 128)
+        yr::prefill_attn_kernel<128, true>
+            <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<128>(), st>>>(pp);
+    else if (!half)
+        yr::prefill_attn_kernel<64, false>
+            <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<64>(), st>>>(pp);
+    else
+        yr::prefill_attn_kernel<64, true>
+            <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<64>(), st>>>(pp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("prefill_attn_kernel launch", e);
     return YR_OK;
@@ -763,41 +751,6 @@ extern "C" int yr_prefill_attend_block(const void *q, float *o, float *lse, int 
     return launch_attend(q, nullptr, lse, nullptr, B, Hq, Hkv, T, d, qs, os, tab, causal, window,
                          sinks_here, workspace_planes(workspace, B, Hkv, Tk, d),
                          static_cast<cudaStream_t>(stream), Tk, q_pos0 - k_pos0, k_pos0, o);
-}
-
-extern "C" int yr_prefill_attend_block_merge(const void *q, float *o_acc, float *lse_acc,
-                                             void *o_out, int init, int B, int Hq, int Hkv, int T,
-                                             int Tk, int d, const int64_t *q_strides,
-                                             const yr_rope_table *tab, int causal, int window,
-                                             int n_sink, int q_pos0, int k_pos0,
-                                             const void *workspace, size_t workspace_bytes,
-                                             void *stream) {
-    set_error("");
-    const std::string f("yr_prefill_attend_block_merge");
-    if (!o_acc || !lse_acc) return fail(YR_EINVAL, f + ": o_acc and lse_acc must be non-NULL");
-    if (init != 0 && init != 1) return fail(YR_EINVAL, f + ": init must be 0 or 1");
-    if (!aligned(o_acc, 16) || (o_out && !aligned(o_out, 16)) || !aligned(lse_acc, 4))
-        return fail(YR_EINVAL, f + ": o_acc and o_out must be 16-byte aligned, lse_acc 4-byte");
-    if (Tk < 1) return fail(YR_EINVAL, f + ": Tk must be >= 1");
-    if (q_pos0 < 0 || k_pos0 < 0 || static_cast<long long>(q_pos0) + T > (1ll << 30) ||
-        static_cast<long long>(k_pos0) + Tk > (1ll << 30))
-        return fail(YR_EINVAL, f + ": positions must be >= 0 and end below 2^30");
-    if (causal && q_pos0 < k_pos0)
-        return fail(YR_EINVAL, f + ": causal blocks need q_pos0 >= k_pos0 (a block wholly in the "
-                                   "future has no visible key; skip it)");
-    long long qs[3], os[3];
-    int rc = check_attend(q, o_acc, lse_acc, nullptr, B, Hq, Hkv, T, d, q_strides, nullptr, tab,
-                          causal, window, n_sink, workspace, workspace_bytes, f.c_str(), qs, os);
-    if (rc != YR_OK) return rc;
-    rc = check_common(f.c_str(), B, Hkv, Tk, d, tab, workspace, workspace_bytes);
-    if (rc != YR_OK) return rc;
-    rc = prepare_device(nullptr);
-    if (rc != YR_OK) return rc;
-    const int sinks_here = n_sink > k_pos0 ? n_sink - k_pos0 : 0;
-    return launch_attend(q, nullptr, lse_acc, nullptr, B, Hq, Hkv, T, d, qs, os, tab, causal,
-                         window, sinks_here, workspace_planes(workspace, B, Hkv, Tk, d),
-                         static_cast<cudaStream_t>(stream), Tk, q_pos0 - k_pos0, k_pos0, o_acc,
-                         1, true, init, static_cast<__nv_bfloat16 *>(o_out));
 }
 
 extern "C" int yr_attn_merge(const float *o_part, const float *lse_part, float *o_acc,

@@ -67,18 +67,6 @@ def block_visible(q_block: int, k_block: int, C: int, causal: bool, window: int,
     return nearest < window or k_block * C < n_sink
 
 
-def _attend_into(ops, q, block, Hkv, Tk, table, q_pos0, k_pos0, causal, window, n_sink, acc,
-                 first, last):
-    """One ring step's attention folded into the running result: the fused block kernel
-    when `ops` has one, else attend then merge."""
-    if hasattr(ops, "attend_into"):
-        ops.attend_into(q, block, Hkv, Tk, table, q_pos0, k_pos0, causal, window, n_sink, acc,
-                        first, last)
-    else:
-        o_p, lse_p = ops.attend(q, block, Hkv, Tk, table, q_pos0, k_pos0, causal, window, n_sink)
-        ops.merge(o_p, lse_p, acc, first, last)
-
-
 class BlockOps:
     """The three block operations of a ring step, on this package's CUDA kernels."""
 
@@ -102,14 +90,6 @@ class BlockOps:
     def merge(self, o_part, lse_part, acc, first: bool, last: bool):
         o_acc, lse_acc, out = acc
         api.attn_merge(o_part, lse_part, o_acc, lse_acc, out=out if last else None, init=first)
-
-    def attend_into(self, q, block, Hkv: int, Tk: int, table, q_pos0: int, k_pos0: int,
-                    causal: bool, window: int, n_sink: int, acc, first: bool, last: bool):
-        """attend + merge in one kernel (the block's fp32 partial is never written)."""
-        o_acc, lse_acc, out = acc
-        api.prefill_attend_block_merge(q, Hkv, Tk, table, block, q_pos0, k_pos0, o_acc, lse_acc,
-                                       causal, window, n_sink, out=out if last else None,
-                                       init=first)
 
     def result(self, acc):
         return acc[2], acc[1]
@@ -146,8 +126,9 @@ def ring_prefill(q, k, v, table, group=None, causal: bool = True, window: int = 
                 dist.P2POp(dist.isend, block, peer_next, group),
                 dist.P2POp(dist.irecv, spare, peer_prev, group)])
         if vis:
-            _attend_into(ops, q, block, Hkv, C, table, rank * C, src * C, causal, window,
-                         n_sink, acc, first, step == last_visible)
+            o_p, lse_p = ops.attend(q, block, Hkv, C, table, rank * C, src * C, causal, window,
+                                    n_sink)
+            ops.merge(o_p, lse_p, acc, first, step == last_visible)
             first = False
         for r in reqs:
             r.wait()
@@ -195,8 +176,9 @@ def _ring_prefill_zigzag(q, k, v, table, group, causal, window, n_sink, ops):
                             dist.P2POp(dist.irecv, spares[b], peer_prev, group)]
             reqs = dist.batch_isend_irecv(ops_p2p)
         for a, b in pairs:
-            _attend_into(ops, q_ch[a], blocks[b], Hkv, c, table, mine[a] * c, theirs[b] * c,
-                         causal, window, n_sink, accs[a], first[a], last.get(a) == (step, b))
+            o_p, lse_p = ops.attend(q_ch[a], blocks[b], Hkv, c, table, mine[a] * c,
+                                    theirs[b] * c, causal, window, n_sink)
+            ops.merge(o_p, lse_p, accs[a], first[a], last.get(a) == (step, b))
             first[a] = False
         for r in reqs:
             r.wait()
@@ -237,9 +219,9 @@ def ring_prefill_emulated(q, k, v, table, world: int, causal: bool = True, windo
             first = [True, True]
             for step, src, theirs, pairs in plan:
                 for a, b in pairs:
-                    _attend_into(ops, q_ch[a], chunk_blocks[theirs[b]], Hkv, c, table,
-                                 mine[a] * c, theirs[b] * c, causal, window, n_sink, accs[a],
-                                 first[a], last.get(a) == (step, b))
+                    o_p, lse_p = ops.attend(q_ch[a], chunk_blocks[theirs[b]], Hkv, c, table,
+                                            mine[a] * c, theirs[b] * c, causal, window, n_sink)
+                    ops.merge(o_p, lse_p, accs[a], first[a], last.get(a) == (step, b))
                     first[a] = False
             res = [ops.result(accs[a]) for a in (0, 1)]
             outs.append((torch.cat([res[0][0], res[1][0]], dim=2),
@@ -259,7 +241,8 @@ def ring_prefill_emulated(q, k, v, table, world: int, causal: bool = True, windo
                  if block_visible(rank, src, C, causal, window, n_sink)]
         acc = ops.new_acc(q_r)
         for n, (_, src) in enumerate(steps):
-            _attend_into(ops, q_r, blocks[src], Hkv, C, table, rank * C, src * C, causal,
-                         window, n_sink, acc, n == 0, n == len(steps) - 1)
+            o_p, lse_p = ops.attend(q_r, blocks[src], Hkv, C, table, rank * C, src * C, causal,
+                                    window, n_sink)
+            ops.merge(o_p, lse_p, acc, n == 0, n == len(steps) - 1)
         outs.append(ops.result(acc))
     return outs
