@@ -347,10 +347,10 @@ def decode_bench(w, steps, warmup, stream):
     return step, lens.tolist()
 
 
-def workload_prefill(w, steps, stream, dist, peak_t):
+def workload_prefill(w, steps, stream, dist, peak_t, warmup=2):
     """Prefill of one more workload: attention-kernel TFLOP/s with causal (and window/sink)
     FLOPs counted, and the whole step (rotated-key pass + attention)."""
-    step, keep = prefill_bench(w, steps, 2, stream)
+    step, keep = prefill_bench(w, steps, warmup, stream)
     flops = metrics.prefill_flops(w.B, w.Hq, w.T, w.d, w.causal, w.window, w.n_sink)
     dist.barrier()
     total_ms, (prep_ms, attn_ms) = time_events(step, steps, stream)
@@ -589,6 +589,13 @@ def main():
                 "tflops": r["call_tflops"], "frac": r["frac_of_peak"],
                 "rank_work_max_over_mean": r["rank_work_max_over_mean"]}
             torch.cuda.empty_cache()
+        # the largest single-GPU prefill: 2^20 tokens, ~8 s a step, against the sustained peak
+        w1m = synth.LLAMA3_1M
+        r = workload_prefill(w1m, 1, stream, dist, peaks["bf16_tflops_sustained"], warmup=1)
+        others["prefill_1m"] = {"tflops": r["attn_kernel_tflops"], "step_tflops": r["step_tflops"],
+                                "frac_of_sustained": r["frac_of_peak"],
+                                "ms": r["attn_kernel_ms"]}
+        torch.cuda.empty_cache()
         w16 = synth.LLAMA2_16K
         r = workload_prefill(w16, max(args.other_steps, 20), stream, dist, peak_burst)
         prefill_16k = {"workload": w16.name, "step_tflops": r["step_tflops"],

@@ -36,7 +36,8 @@ def _tables(w):
 
 
 def test_million_token_prefill_sampled_rows():
-    w = dataclasses.replace(synth.LLAMA3_128K, T=T_MILLION)
+    w = synth.LLAMA3_1M
+    assert w.T == T_MILLION
     q, k, v = synth.prefill_inputs(w, "cuda")
     tab, th, ss = _tables(w)
     lse = torch.empty(q.shape[:3], device="cuda")

@@ -57,6 +57,9 @@ DECODE = Workload("decode_b8_gqa_128k", "decode", 3, 8, 32, 8, 128, 131073, "yar
 # The last 4096 tokens of a 128K Llama-3-8B-shaped prompt, after a cached 124K prefix.
 CHUNK = Workload("chunk_llama3_8b_124k_plus_4k", "chunk", 5, 1, 32, 8, 128, 131072, "yarn",
                  500000.0, 8192, 16.0, P0=126976, Tq=4096)
+# The same heads and table at 2^20 tokens: the largest single-GPU prefill of the path.
+LLAMA3_1M = Workload("llama3_8b_1m_gqa_prefill", "prefill", 6, 1, 32, 8, 128, 1 << 20, "yarn",
+                     500000.0, 8192, 16.0)
 
 
 def sweep(method: str, windowed: bool) -> Workload:
@@ -67,7 +70,7 @@ def sweep(method: str, windowed: bool) -> Workload:
 
 
 SWEEP = [sweep(m, w) for m in ("rope", "pi", "ntk", "yarn") for w in (False, True)]
-ALL = {w.name: w for w in [TINY, LLAMA2_16K, LLAMA3_128K, DECODE, CHUNK] + SWEEP}
+ALL = {w.name: w for w in [TINY, LLAMA2_16K, LLAMA3_128K, DECODE, CHUNK, LLAMA3_1M] + SWEEP}
 
 
 def _gen(seed: int, device) -> torch.Generator:
