@@ -10,8 +10,9 @@ This module only marshals numpy arrays into it.  Inputs are bf16 bit patterns
 (``uint16``), widened exactly to double inside the C code.
 
 Parity status (see the header of ``yarn_oracle.c``): every function is pinned
-by a test in ``tests/test_oracle_pins.py`` except the interior of the YaRN
-ramp, which is a reading of the pages ("parity unpinned" there).
+by a test in ``tests/test_oracle_pins.py``.  The interior of the YaRN ramp is a
+reading of the pages (linear in r, where they print no value); the oracle is
+pinned to that reading's closed form at constructed points.
 """
 from __future__ import annotations
 

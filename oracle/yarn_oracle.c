@@ -34,8 +34,12 @@
  *
  * Parity status per function:
  *   oracle_rope_theta   pinned (closed forms, s=1 reductions, NTK worked
- *                       number, band endpoints); the YaRN ramp INTERIOR is
- *                       a reading of the pages: parity unpinned there.
+ *                       number, band endpoints).  The YaRN ramp interior is
+ *                       a reading of the pages (they print no value inside
+ *                       it); the oracle's ramp is pinned to that reading's
+ *                       closed form at constructed points (a base that puts a
+ *                       pair at r = alpha + f (beta - alpha) must give
+ *                       f theta + (1 - f) theta / s).
  *   oracle_rope_theta_ext  dynamic NTK pinned (RoPE at or below L_train, equal
  *                       to NTK at L_cur = s L_train, the page's ~82,000 base);
  *                       dimension-ramp YaRN pinned outside its ramp and at the

@@ -742,3 +742,19 @@ def test_kv_cache_bytes_worked_numbers(golden):
             assert got / 1e9 == pytest.approx(row["printed_gb"], rel=row["rel_tol"])
         else:
             assert got / 2 ** 30 == pytest.approx(row["printed_gib"], rel=row["rel_tol"])
+
+
+@pytest.mark.parametrize("i0", [5, 20, 40])
+@pytest.mark.parametrize("f", [0.0, 0.25, 0.5, 0.75, 1.0])
+def test_yarn_ramp_interior_at_constructed_points(i0, f):
+    # Inside YaRN's ramp the reading is linear in r = L_train / lambda_i.  Choose the base
+    # so that pair i0 sits at r = alpha + f (beta - alpha): its frequency must then be the
+    # plain mix f theta + (1 - f) theta / s.  A ramp in log r or in the pair index, a
+    # swapped mix, or swapped band edges all miss these values.
+    d, L, s, alpha, beta = 128, 4096, 16.0, 1.0, 32.0
+    r = alpha + f * (beta - alpha)
+    base = (L / (2.0 * math.pi * r)) ** (d / (2.0 * i0))
+    th, _, _ = oracle.rope_theta(d, base, L, s, "yarn", alpha, beta)
+    rope, _, _ = oracle.rope_theta(d, base, L, 1.0, "rope")
+    assert rope[i0] * L / (2.0 * math.pi) == pytest.approx(r, rel=1e-12)
+    assert th[i0] / rope[i0] == pytest.approx(f + (1.0 - f) / s, rel=1e-12)
