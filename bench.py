@@ -302,10 +302,11 @@ def reference_arm(args, dist: Dist):
 
 
 # ------------------------------------------------------------------- GPU arm
-def prefill_bench(w, steps, warmup, stream):
+def prefill_bench(w, steps, warmup, stream, pairs="interleaved"):
     from yarn_position_scaling_b200 import api
     q, k, v = synth.prefill_inputs(w, "cuda")
-    tab = api.rope_freq_table(w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta)
+    tab = api.rope_freq_table(w.d, w.base, w.L_train, w.scale, w.method, w.alpha, w.beta,
+                              pairs=pairs)
     ws = torch.empty(api.attn_prefill_workspace_bytes(w.B, w.Hkv, w.T, w.d), dtype=torch.uint8,
                      device="cuda")
     o = torch.empty_like(q)
@@ -347,10 +348,10 @@ def decode_bench(w, steps, warmup, stream):
     return step, lens.tolist()
 
 
-def workload_prefill(w, steps, stream, dist, peak_t, warmup=2):
+def workload_prefill(w, steps, stream, dist, peak_t, warmup=2, pairs="interleaved"):
     """Prefill of one more workload: attention-kernel TFLOP/s with causal (and window/sink)
     FLOPs counted, and the whole step (rotated-key pass + attention)."""
-    step, keep = prefill_bench(w, steps, warmup, stream)
+    step, keep = prefill_bench(w, steps, warmup, stream, pairs)
     flops = metrics.prefill_flops(w.B, w.Hq, w.T, w.d, w.causal, w.window, w.n_sink)
     dist.barrier()
     total_ms, (prep_ms, attn_ms) = time_events(step, steps, stream)
@@ -575,6 +576,15 @@ def main():
                 "tflops": r["attn_kernel_tflops"], "step_tflops": r["step_tflops"],
                 "frac": r["frac_of_peak"]}
             torch.cuda.empty_cache()
+        # the half-split pair layout (i, i + d/2), a kernel instantiation of its own
+        w = synth.sweep("yarn", False)
+        flops_w = metrics.prefill_flops(w.B, w.Hq, w.T, w.d, w.causal, w.window, w.n_sink)
+        r = workload_prefill(w, max(args.other_steps, int(1e14 / flops_w)), stream, dist,
+                             peak_burst, pairs="half")
+        others["yarn_dense_half_pairs"] = {"tflops": r["attn_kernel_tflops"],
+                                           "step_tflops": r["step_tflops"],
+                                           "frac": r["frac_of_peak"]}
+        torch.cuda.empty_cache()
         r = chunk_bench(synth.CHUNK, args.other_steps, stream, dist, peak_burst)
         others["chunk_124k_plus_4k"] = {"tflops": r["call_tflops"], "frac": r["frac_of_peak"],
                                         "ms": r["call_ms"]}
