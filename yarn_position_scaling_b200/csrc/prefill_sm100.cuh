@@ -7,6 +7,7 @@
 //   warp 9      MMA issuer: S_t = Q_t K~^T and O_t += P_t V with tcgen05.mma,
 //               accumulators in tensor memory (TMEM); the whole warp runs the
 //               loop and one elected lane issues
+//   warps 10-11 build the per-lane rotation table for the Q prologue
 //   warps 0-3   softmax for Q0, warps 4-7 softmax for Q1: each thread owns one
 //               query row (= one TMEM lane), so row max and row sum need no
 //               shuffles; P is written back over S in TMEM as fp16
@@ -33,9 +34,12 @@
 // Rotation ("Arch_03_Long_Context", RoPE slide): pair (2i, 2i+1) of the query
 // at position m turns by m * theta'_i (or pair (i, i + d/2) in the half-split
 // layout, a separate instantiation of the kernel).  Each softmax warp reduces the angle of
-// every pair at its first row in fp64 (turns minus the nearest integer); a row
-// adds lane * theta'_i / (2 pi) in fp32 and takes fp32 sin/cos.  A rotated value
-// that does not fit fp16 sets the range bit of the device status word.  Rarely run
+// every pair at its first row in fp64 (turns minus the nearest integer) and takes its
+// fp32 sin/cos; a row at lane l of the warp adds l * theta'_i by angle addition with
+// (cos, sin)(l * theta'_i) from a table the two idle warps of the load/MMA warpgroup
+// build once per CTA, so the prologue takes one sin/cos per pair and warp instead of
+// one per element.  A rotated value that does not fit fp16 sets the range bit of the
+// device status word.  Rarely run
 // paths are kept small (rolled loops, compact masks): their instructions are
 // fetched cold.
 //
@@ -108,12 +112,14 @@ struct PrefillSmem {
     uint8_t k[kKStages][kSub][kSubTileBytes];
     uint8_t v[kVStages][kSub][kSubTileBytes];
     uint64_t q_full[kQTiles], q_ready[kQTiles];
+    uint64_t lanes_ready;
     uint64_t k_full[kKStages], k_empty[kKStages];
     uint64_t v_full[kVStages], v_empty[kVStages];
     uint64_t s_full[kQTiles], p_full[kQTiles], o_done[kQTiles];
     // Q rotation: per softmax warp, the angle (turns, reduced) of each pair at the
     // warp's first row, and the pair's rotations per position in fp32.
-    float q_base[8][kMaxPairs], q_turn[8][kMaxPairs];
+    float2 q_cs0[8][kMaxPairs];       // per softmax warp: (cos, sin) of pair i at its first row
+    float2 lane_cs[kMaxPairs][32];    // (cos, sin) of lane * theta'_i, lane 0..31
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort;
@@ -282,6 +288,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             mbar_init(&sm->v_empty[s], 1);
         }
         mbar_init(&sm->mma_done, 1);
+        mbar_init(&sm->lanes_ready, 2);  // warps 10 and 11
         sm->abort = 0;
         fence_mbar_init();
     }
@@ -301,9 +308,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     volatile int *abort = &sm->abort;
 
     if (warp >= 8) {
-      // load/MMA warpgroup (warps 8-11; 10 and 11 have no role): shrink first
+      // load/MMA warpgroup (warps 8-11; 10 and 11 build the rotation table): shrink first
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
-      if (warp == 8) {
+      if (warp >= 10) {
+        // ------------------------------------------ per-lane rotation table
+        // (cos, sin) of lane * theta'_i for lane 0..31: angle reduced in fp64 (turns
+        // minus the nearest integer), one fp32 sin/cos per entry, for all CTAs' rows.
+        for (int e = (warp - 10) * 32 + lane; e < (HD / 2) * 32; e += 64) {
+            const int i = e >> 5, l = e & 31;
+            const double tr = static_cast<double>(l) * p.turns[i];
+            float sn, cs;
+            __sincosf(static_cast<float>((tr - rint(tr)) * 6.283185307179586), &sn, &cs);
+            sm->lane_cs[i][l] = make_float2(cs, sn);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm->lanes_ready);
+      } else if (warp == 8) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint64_t pol_q = l2_policy_evict_first();
@@ -488,25 +508,26 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 float *dbg = (p.q_dbg != nullptr && row < p.T)
                                  ? p.q_dbg + ((static_cast<long long>(b) * p.Hq + h) * p.T + row) * HD
                                  : nullptr;
-                // Angle of pair i at this row, in turns: the warp's first row reduced in
-                // fp64 (turns minus the nearest integer) plus lane * turns_i in fp32
-                // (lane <= 31, so the sum stays below 6 turns: ~3e-7 turns of rounding).
-                float *qb = sm->q_base[warp], *qt = sm->q_turn[warp];
+                // Angle of pair i at this row = the warp's first row's angle plus
+                // lane * theta'_i: (cos, sin) of the first (fp64-reduced, fp32 sin/cos, once
+                // per warp and pair) times (cos, sin) of the lane's offset (a table built
+                // once per CTA), by angle addition.
+                float2 *cs0 = sm->q_cs0[warp];
                 const int pos0 = pos - lane;
                 for (int i = lane; i < HD / 2; i += 32) {
                     const double tr = static_cast<double>(pos0 + p.k_pos0) * p.turns[i];
-                    qb[i] = static_cast<float>(tr - rint(tr));
-                    qt[i] = static_cast<float>(p.turns[i]);
+                    float sn, cs;
+                    __sincosf(static_cast<float>((tr - rint(tr)) * 6.283185307179586), &sn, &cs);
+                    cs0[i] = make_float2(cs, sn);
                 }
                 __syncwarp();
-                const float lanef = static_cast<float>(lane);
+                ok = __all_sync(0xffffffffu, mbar_wait(&sm->lanes_ready, 0, abort, p.timeout_ns));
                 bool bad = false;  // a rotated value of this row does not fit fp16
                 // sin/cos of pair i's angle at this row
                 auto pair_sincos = [&](int i, float &sn, float &cs) {
-                    const float turns = fmaf(lanef, qt[i], qb[i]);
-                    // nearest integer by the 1.5 * 2^23 rounding trick (|turns| < 6)
-                    const float near = (turns + 12582912.0f) - 12582912.0f;
-                    __sincosf((turns - near) * 6.2831853071795865f, &sn, &cs);
+                    const float2 a = cs0[i], l = sm->lane_cs[i][lane];
+                    cs = fmaf(a.x, l.x, -a.y * l.y);
+                    sn = fmaf(a.y, l.x, a.x * l.y);
                 };
                 // 16-byte chunk g (elements 8g .. 8g+7) of this row in the swizzled tile
                 auto q_chunk = [&](int g) {
