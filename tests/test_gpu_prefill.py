@@ -85,6 +85,18 @@ def test_window_and_sinks(T, window, n_sink):
     run_full(synth.LLAMA3_128K, T, window=window, n_sink=n_sink)
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,T,d,window,n_sink", [
+    (1, 4, 2, 129, 128, 64, 0),      # two heads per CTA, one row past a tile
+    (2, 8, 1, 1000, 64, 300, 4),     # eight query heads on one KV head, batch 2
+    (1, 16, 2, 777, 128, 128, 130),  # sinks reaching past the first key tile
+    (1, 6, 2, 700, 128, 200, 4),     # a group of three: one head per CTA
+])
+def test_window_head_pairs(B, Hq, Hkv, T, d, window, n_sink):
+    """Windowed calls with an even number of query heads per KV head run two heads of one
+    group at the same 128 rows in a CTA (odd groups keep 256 rows of one head)."""
+    run_full(synth.LLAMA3_128K, T, B=B, d=d, Hq=Hq, Hkv=Hkv, window=window, n_sink=n_sink)
+
+
 @pytest.mark.parametrize("T,d", [(200, 64), (300, 128)])
 def test_non_causal(T, d):
     run_full(synth.TINY, T, causal=False, d=d)

@@ -1,8 +1,11 @@
 // prefill_sm100.cuh -- causal / windowed GQA attention prefill for sm_100a with
 // rotary position embedding applied to Q inside the kernel.
 //
-// One CTA owns two 128-row query tiles (Q0, Q1) of one (batch, head) and walks
-// the key/value tiles those rows can see:
+// One CTA owns two 128-row query tiles (Q0, Q1) and walks the key/value tiles
+// their rows can see.  Q0 and Q1 are rows [0, 128) and [128, 256) of a 256-row block
+// of one (batch, head), or (head pairs, for windowed calls with an even number of
+// query heads per KV head) the same 128 rows of two query heads of one KV group, which
+// see exactly the same key tiles.  Roles:
 //   warp 8      TMA producer: Q tiles once, then K~/V tiles through a 2-stage ring
 //   warp 9      MMA issuer: S_t = Q_t K~^T and O_t += P_t V with tcgen05.mma,
 //               accumulators in tensor memory (TMEM); the whole warp runs the
@@ -89,6 +92,10 @@ struct alignas(64) PrefillParams {
     int causal, window, n_sink;
     int n_qblocks;
     int kv_major;  // CTA order: 1 = by KV head first (grouped heads), 0 = by query block
+    // 1: the CTA's two query tiles are heads h and h + 1 of one KV group at the same 128
+    // rows (so both see exactly the same key tiles); 0: rows [0, 128) and [128, 256) of one
+    // head.  n_qblocks counts 128-row blocks with head pairs, 256-row blocks without.
+    int head_pair;
     int alibi;     // 1: add the ALiBi bias -m_h (i - j) to the logits
     // Split-KV: each (batch, head, query block) item is cut into n_split CTAs that take
     // equal shares of its key tiles; CTA s writes its normalised fp32 partial to
@@ -181,6 +188,12 @@ __device__ __forceinline__ bool tile_full(const PrefillParams &p, int r_lo, int 
     return true;
 }
 
+// Query head of tile t of a CTA whose tile 0 has head h.  (Evaluated where it is used: a
+// variable held across the softmax loop costs the d = 64 kernel a spill.)
+__device__ __forceinline__ int tile_head(const PrefillParams &p, int h, int t) {
+    return t == 0 ? h : h + p.head_pair;
+}
+
 // Bits 0..min(c, 31) set (0 for c < 0): columns at or below c of a 32-column word.
 __device__ __forceinline__ uint32_t cols_upto(int c) {
     if (c < 0) return 0u;
@@ -235,17 +248,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int split = p.n_split > 1 ? static_cast<int>(blockIdx.x) % p.n_split : 0;
     const int item = p.n_split > 1 ? static_cast<int>(blockIdx.x) / p.n_split
                                    : static_cast<int>(blockIdx.x);
-    int qb, b, h;
+    int qb, b, h;  // h: the head of query tile 0 (tile 1's is h + head_pair)
     if (p.kv_major) {
         // Grouped heads: one (batch, KV head) after another, its query blocks
-        // heaviest first and the query heads of its group adjacent, so the CTAs
-        // resident at any time read the K/V of one or two KV heads, which stay in L2.
-        const int per_kv = p.n_qblocks * p.group;
+        // heaviest first and the query heads (or head pairs) of its group adjacent, so
+        // the CTAs resident at any time read the K/V of one or two KV heads, which stay
+        // in L2.
+        const int units = p.head_pair ? p.group / 2 : p.group;  // head units per KV head
+        const int per_kv = p.n_qblocks * units;
         const int bk = item / per_kv;
         const int rem = item % per_kv;
-        qb = p.n_qblocks - 1 - rem / p.group;
+        qb = p.n_qblocks - 1 - rem / units;
         b = bk / p.Hkv;
-        h = (bk % p.Hkv) * p.group + rem % p.group;
+        h = (bk % p.Hkv) * p.group + (rem % units) * (p.head_pair ? 2 : 1);
     } else {
         // Heaviest causal blocks first, the heads of one query block adjacent.
         const int bh_count = p.B * p.Hq;
@@ -256,8 +271,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
     const int kvh = h / p.group;
     // Query tiles by position: row r of the query tensor sits at position q_off + r.
-    const int q0 = p.q_off + qb * (kQTiles * kBlockM);
-    const int last_pos = min(q0 + kQTiles * kBlockM - 1, p.q_off + p.T - 1);
+    const int block_rows = p.head_pair ? kBlockM : kQTiles * kBlockM;
+    const int q0 = p.q_off + qb * block_rows;
+    const int last_pos = min(q0 + block_rows - 1, p.q_off + p.T - 1);
     TilePlan tp = plan_tiles(p, q0, last_pos);
     if (p.n_split > 1) {
         const int per = (tp.n + p.n_split - 1) / p.n_split;
@@ -267,7 +283,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     int r_lo[kQTiles], r_hi[kQTiles];
 #pragma unroll
     for (int t = 0; t < kQTiles; ++t) {
-        r_lo[t] = q0 + t * kBlockM;
+        r_lo[t] = p.head_pair ? q0 : q0 + t * kBlockM;
         r_hi[t] = min(r_lo[t] + kBlockM - 1, last_pos);
     }
 
@@ -333,8 +349,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 if (r_lo[t] > r_hi[t]) continue;
                 mbar_arrive_expect_tx(&sm->q_full[t], kSub * kSubTileBytes);
                 for (int s = 0; s < kSub; ++s)
-                    tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64, r_lo[t] - p.q_off, h,
-                                b, pol_q);
+                    tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64, r_lo[t] - p.q_off,
+                                tile_head(p, h, t), b, pol_q);
             }
             const int kv_plane = b * p.Hkv + kvh;
             int issued_k[kKStages] = {}, issued_v[kVStages] = {};
@@ -506,7 +522,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
                 float *dbg = (p.q_dbg != nullptr && row < p.T)
-                                 ? p.q_dbg + ((static_cast<long long>(b) * p.Hq + h) * p.T + row) * HD
+                                 ? p.q_dbg + ((static_cast<long long>(b) * p.Hq + tile_head(p, h, t)) * p.T +
+                                              row) * HD
                                  : nullptr;
                 // Angle of pair i at this row = the warp's first row's angle plus
                 // lane * theta'_i: (cos, sin) of the first (fp64-reduced, fp32 sin/cos, once
@@ -605,7 +622,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
         // ALiBi slope of this head, m_h = 2^(-8 (h+1) / Hq), over the softmax scale.
         const float alibi_coef =
-            p.alibi ? exp2f(-8.0f * static_cast<float>(h + 1) / static_cast<float>(p.Hq)) *
+            p.alibi ? exp2f(-8.0f * static_cast<float>(tile_head(p, h, t) + 1) /
+                            static_cast<float>(p.Hq)) *
                           1.4426950408889634f / p.sl2
                     : 0.0f;
         float m_run = -INFINITY;  // reference max of this row, log2 units (score * sl2)
@@ -746,14 +764,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         // Epilogue: O / l -> bf16 (or fp32), and the log-sum-exp in natural-log units.
         const long long orow_idx =
-            (static_cast<long long>(b) * p.Hq + h) * p.T + row + split * p.split_rows;
+            (static_cast<long long>(b) * p.Hq + tile_head(p, h, t)) * p.T + row + split * p.split_rows;
         if (ok && tile_live && it > 0) {
             ok = mbar_wait(&sm->o_done[t], (it - 1) & 1, abort, p.timeout_ns);
             ok = __all_sync(0xffffffffu, ok);
             if (ok) {
                 tc_fence_after();
                 const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
-                __nv_bfloat16 *orow = p.o + b * p.osb + h * p.osh + static_cast<long long>(row) * p.ost;
+                __nv_bfloat16 *orow = p.o + b * p.osb + tile_head(p, h, t) * p.osh +
+                                      static_cast<long long>(row) * p.ost;
                 uint32_t raw[32];
 #pragma unroll
                 for (int c = 0; c < HD / 32; ++c) {
@@ -799,7 +818,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll 1
                 for (int c = 0; c < HD / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
             } else {
-                __nv_bfloat16 *orow = p.o + b * p.osb + h * p.osh + static_cast<long long>(row) * p.ost;
+                __nv_bfloat16 *orow = p.o + b * p.osb + tile_head(p, h, t) * p.osh +
+                                      static_cast<long long>(row) * p.ost;
 #pragma unroll 1
                 for (int c = 0; c < HD / 8; ++c)
                     *reinterpret_cast<uint4 *>(orow + c * 8) = make_uint4(0u, 0u, 0u, 0u);

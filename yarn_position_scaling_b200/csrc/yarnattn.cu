@@ -375,6 +375,21 @@ KvPlanes workspace_planes(const void *workspace, int B, int Hkv, int Tk, int d) 
     return {k16, k16 + static_cast<size_t>(B) * Hkv * Tk * d, Tk};
 }
 
+// Does the attention kernel pair two query heads per CTA, and how many (batch, head unit,
+// query block) items does a call of T rows have?  Pairs need an even number of query heads
+// per KV head.  They pay off with a window, where a CTA's key tiles are few and the two
+// tiles a 256-row block has for one of its halves alone (the window's first, the
+// diagonal's last) are a large share of them: +1-4% on the windowed 64K GQA workloads,
+// -0.4% / -1% on the dense 128K / 64K ones (four alternating rounds on one B200).
+int attend_head_pair(int Hq, int Hkv, int window) {
+    return window > 0 && (Hq / Hkv) % 2 == 0 ? 1 : 0;
+}
+long long attend_items(int B, int Hq, int Hkv, int T, int window) {
+    return attend_head_pair(Hq, Hkv, window)
+               ? static_cast<long long>(B) * (Hq / 2) * ((T + 127) / 128)
+               : static_cast<long long>(B) * Hq * ((T + 255) / 256);
+}
+
 // T query rows against the Tk keys of `kv`.  Key n sits at position k_pos0 + n and
 // query row r at k_pos0 + q_off + r; masks use the offsets relative to key 0.
 int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, int Hq, int Hkv,
@@ -420,7 +435,10 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     pp.B = B; pp.Hq = Hq; pp.Hkv = Hkv; pp.T = T; pp.group = Hq / Hkv;
     pp.Tk = Tk; pp.q_off = q_off; pp.k_pos0 = k_pos0;
     pp.causal = causal; pp.window = window; pp.n_sink = n_sink;
-    pp.n_qblocks = (T + 255) / 256;
+    // Windowed calls with an even number of query heads per KV head: a CTA takes two heads of
+    // one group at the same 128 rows, so both query tiles see the same key tiles.
+    pp.head_pair = attend_head_pair(Hq, Hkv, window);
+    pp.n_qblocks = pp.head_pair ? (T + 127) / 128 : (T + 255) / 256;
     pp.n_split = n_split;
     pp.split_rows = static_cast<long long>(B) * Hq * T;
     // Grouped query heads read each K/V tile several times: order the CTAs by KV head
@@ -439,7 +457,7 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
 #endif
     for (int i = 0; i < d / 2; ++i) pp.turns[i] = tab->turns[i];
     const unsigned grid =
-        static_cast<unsigned>(static_cast<long long>(B) * Hq * pp.n_qblocks * n_split);
+        static_cast<unsigned>(attend_items(B, Hq, Hkv, T, window) * n_split);
     if (d == 128 && !half)
         yr::prefill_attn_kernel<128, false>
             <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<128>(), st>>>(pp);
@@ -539,12 +557,13 @@ size_t split_share_bytes(long long B, long long Hq, long long Tq, long long d) {
 // waves x (tiles per share + 5) wins.  Each share keeps at least 4 key tiles; at most kMaxSplit shares
 // and at most what the split workspace holds.
 constexpr int kMaxSplit = 16;
-int choose_split(int sm_count, int B, int Hq, int Tq, int P0, int window, size_t ws_bytes,
-                 size_t share_bytes) {
-    const long long items = static_cast<long long>(B) * Hq * ((Tq + 255) / 256);
+int choose_split(int sm_count, int B, int Hq, int Hkv, int Tq, int P0, int window,
+                 size_t ws_bytes, size_t share_bytes) {
+    const long long items = attend_items(B, Hq, Hkv, Tq, window);
     if (items >= 2ll * sm_count || share_bytes == 0) return 1;
-    int keys = P0 + (Tq < 256 ? Tq : 256);  // the first query block's keys (the fewest)
-    if (window > 0 && window < keys) keys = window + 256;
+    const int rows = attend_head_pair(Hq, Hkv, window) ? 128 : 256;  // query rows per CTA
+    int keys = P0 + (Tq < rows ? Tq : rows);  // the first query block's keys (the fewest)
+    if (window > 0 && window < keys) keys = window + rows;
     const int tiles = (keys + 127) / 128;
     long long s_max = kMaxSplit;
     if (s_max > tiles / 4) s_max = tiles / 4;
@@ -616,7 +635,7 @@ int chunk_call(const char *fn, const void *q, const void *k_new, const void *v_n
         if (e != cudaSuccess) return cuda_fail("chunk_prep_kernel launch", e);
     }
     const size_t share = split_share_bytes(B, Hq, Tq, d);
-    const int n_split = split_ws ? choose_split(sm_count, B, Hq, Tq, P0, window, split_ws_bytes,
+    const int n_split = split_ws ? choose_split(sm_count, B, Hq, Hkv, Tq, P0, window, split_ws_bytes,
                                                 share)
                                  : 1;
     const KvPlanes kv{k16, v16, ld16};
