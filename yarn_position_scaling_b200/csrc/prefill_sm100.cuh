@@ -96,6 +96,9 @@ struct alignas(64) PrefillParams {
     // rows (so both see exactly the same key tiles); 0: rows [0, 128) and [128, 256) of one
     // head.  n_qblocks counts 128-row blocks with head pairs, 256-row blocks without.
     int head_pair;
+    // > 0: each CTA's producer prefetches into L2 the Q tiles of CTA blockIdx + this stride
+    // (the SM count: about the CTA that will start next on some SM).
+    int q_prefetch_stride;
     int alibi;     // 1: add the ALiBi bias -m_h (i - j) to the logits
     // Split-KV: each (batch, head, query block) item is cut into n_split CTAs that take
     // equal shares of its key tiles; CTA s writes its normalised fp32 partial to
@@ -186,6 +189,27 @@ __device__ __forceinline__ bool tile_full(const PrefillParams &p, int r_lo, int 
     if (p.causal && k_hi > r_lo) return false;
     if (p.window > 0 && !(r_hi - k_lo < p.window || k_hi < p.n_sink)) return false;
     return true;
+}
+
+// Query block, batch and first query head of CTA `cta` (the kernel's own decode, for the
+// L2 prefetch of a later CTA's Q tiles).
+__device__ __forceinline__ void cta_q_coords(const PrefillParams &p, int cta, int &qb, int &b,
+                                             int &h) {
+    const int item = p.n_split > 1 ? cta / p.n_split : cta;
+    if (p.kv_major) {
+        const int units = p.head_pair ? p.group / 2 : p.group;
+        const int per_kv = p.n_qblocks * units;
+        const int bk = item / per_kv, rem = item % per_kv;
+        qb = p.n_qblocks - 1 - rem / units;
+        b = bk / p.Hkv;
+        h = (bk % p.Hkv) * p.group + (rem % units) * (p.head_pair ? 2 : 1);
+    } else {
+        const int bh_count = p.B * p.Hq;
+        qb = p.n_qblocks - 1 - item / bh_count;
+        const int rem = item % bh_count;
+        b = rem / p.Hq;
+        h = rem % p.Hq;
+    }
 }
 
 // Query head of tile t of a CTA whose tile 0 has head h.  (Evaluated where it is used: a
@@ -351,6 +375,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 for (int s = 0; s < kSub; ++s)
                     tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64, r_lo[t] - p.q_off,
                                 tile_head(p, h, t), b, pol_q);
+            }
+            if (p.q_prefetch_stride > 0 &&
+                blockIdx.x + static_cast<unsigned>(p.q_prefetch_stride) < gridDim.x) {
+                int nqb, nb, nh;
+                cta_q_coords(p, static_cast<int>(blockIdx.x) + p.q_prefetch_stride, nqb, nb, nh);
+                const int rows = p.head_pair ? kBlockM : kQTiles * kBlockM;
+                for (int t = 0; t < kQTiles; ++t) {
+                    const int r0 = nqb * rows + (p.head_pair ? 0 : t * kBlockM);
+                    if (r0 >= p.T) continue;
+                    for (int s = 0; s < kSub; ++s)
+                        tma_prefetch_4d(&p.tm_q, s * 64, r0, nh + (p.head_pair ? t : 0), nb);
+                }
             }
             const int kv_plane = b * p.Hkv + kvh;
             int issued_k[kKStages] = {}, issued_v[kVStages] = {};

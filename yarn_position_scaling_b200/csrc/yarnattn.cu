@@ -438,6 +438,9 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     // Windowed calls with an even number of query heads per KV head: a CTA takes two heads of
     // one group at the same 128 rows, so both query tiles see the same key tiles.
     pp.head_pair = attend_head_pair(Hq, Hkv, window);
+    // The CTA one wave later (about the next to start on some SM) gets its Q tiles into L2
+    // while this one runs.
+    pp.q_prefetch_stride = ds.sm_count;
     pp.n_qblocks = pp.head_pair ? (T + 127) / 128 : (T + 255) / 256;
     pp.n_split = n_split;
     pp.split_rows = static_cast<long long>(B) * Hq * T;
