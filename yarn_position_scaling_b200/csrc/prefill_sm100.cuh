@@ -354,7 +354,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // ------------------------------------------ per-lane rotation table
         // (cos, sin) of lane * theta'_i for lane 0..31: angle reduced in fp64 (turns
         // minus the nearest integer), one fp32 sin/cos per entry, for all CTAs' rows.
-        for (int e = (warp - 10) * 32 + lane; e < (HD / 2) * 32; e += 64) {
+        // Unrolled so that independent entries overlap: one entry is a chain of fp64
+        // operations, a sin/cos and a store, and run one after another the table held
+        // up the Q rotation (a timing-only copy without it ran 5% faster at 16K and on
+        // the windowed 64K workloads).
+#pragma unroll 8
+        for (int k = 0; k < (HD / 2) * 32 / 64; ++k) {
+            const int e = (warp - 10) * 32 + lane + 64 * k;
             const int i = e >> 5, l = e & 31;
             const double tr = static_cast<double>(l) * p.turns[i];
             float sn, cs;
