@@ -573,7 +573,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 // once per CTA), by angle addition.
                 float2 *cs0 = sm->q_cs0[warp];
                 const int pos0 = pos - lane;
-                for (int i = lane; i < HD / 2; i += 32) {
+#pragma unroll
+                for (int k = 0; k < HD / 64; ++k) {
+                    const int i = lane + 32 * k;
                     const double tr = static_cast<double>(pos0 + p.k_pos0) * p.turns[i];
                     float sn, cs;
                     __sincosf(static_cast<float>((tr - rint(tr)) * 6.283185307179586), &sn, &cs);
@@ -588,7 +590,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     cs = fmaf(a.x, l.x, -a.y * l.y);
                     sn = fmaf(a.y, l.x, a.x * l.y);
                 };
-                // 16-byte chunk g (elements 8g .. 8g+7) of this row in the swizzled tile
+                // 16-byte chunk g (elements 8g .. 8g+7) of this row in the swizzled tile.  The
+                // chunk loops below are unrolled so that the chunks' loads and rotations
+                // overlap: the rotation sits on the path to the CTA's first S (measured +3-9%
+                // at 16K and +2-7% on the windowed 64K workloads against one chunk at a time).
                 auto q_chunk = [&](int g) {
                     return reinterpret_cast<uint4 *>(sm->q[t][g >> 3] + r * 128 +
                                                      (((g & 7) ^ (r & 7)) << 4));
@@ -596,7 +601,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 if constexpr (kHalfPairs) {
                     // Pairs (i, i + d/2): chunk c holds the first elements of pairs
                     // 8c .. 8c+7, chunk c + d/16 their second elements.
-#pragma unroll 1
+#pragma unroll
                     for (int c = 0; c < HD / 16; ++c) {
                         uint4 *plo = q_chunk(c), *phi = q_chunk(c + HD / 16);
                         const uint4 rlo = *plo, rhi = *phi;
@@ -629,7 +634,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     }
                 } else {
                     // Pairs (2i, 2i+1): chunk c holds pairs 4c .. 4c+3.
-#pragma unroll 1
+#pragma unroll
                     for (int c = 0; c < HD / 8; ++c) {
                         uint4 *ptr = q_chunk(c);
                         const uint4 raw = *ptr;
