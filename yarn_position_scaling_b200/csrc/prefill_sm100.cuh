@@ -311,7 +311,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         r_hi[t] = min(r_lo[t] + kBlockM - 1, last_pos);
     }
 
-    if (threadIdx.x == 0) {
+    // The TMA producer thread sets up the barriers and issues the Q tiles' loads at once,
+    // so that they overlap the TMEM allocation and the CTA-wide barrier below.
+    if (warp == 8 && lane == 0) {
+        prefetch_tensormap(&p.tm_q);
         for (int t = 0; t < kQTiles; ++t) {
             mbar_init(&sm->q_full[t], 1);
             mbar_init(&sm->q_ready[t], kBlockM / 32);  // one arrival per softmax warp
@@ -331,15 +334,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         mbar_init(&sm->lanes_ready, 2);  // warps 10 and 11
         sm->abort = 0;
         fence_mbar_init();
+        const uint64_t pol_q = l2_policy_evict_first();
+        for (int t = 0; t < kQTiles; ++t) {
+            if (r_lo[t] > r_hi[t]) continue;
+            mbar_arrive_expect_tx(&sm->q_full[t], kSub * kSubTileBytes);
+            for (int s = 0; s < kSub; ++s)
+                tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64, r_lo[t] - p.q_off,
+                            tile_head(p, h, t), b, pol_q);
+        }
+        prefetch_tensormap(&p.tm_k);
+        prefetch_tensormap(&p.tm_v);
     }
     if (warp == 9) {
         tmem_alloc(&sm->tmem_base, kTmemCols);
         tmem_relinquish();
-    }
-    if (warp == 8 && lane == 0) {
-        prefetch_tensormap(&p.tm_q);
-        prefetch_tensormap(&p.tm_k);
-        prefetch_tensormap(&p.tm_v);
     }
     tc_fence_before();
     __syncthreads();
@@ -372,16 +380,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       } else if (warp == 8) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
-            const uint64_t pol_q = l2_policy_evict_first();
+            // (the Q tiles' loads were issued with the barrier set-up)
             const uint64_t pol_kv = l2_policy_evict_last();
             bool ok = true;
-            for (int t = 0; t < kQTiles; ++t) {
-                if (r_lo[t] > r_hi[t]) continue;
-                mbar_arrive_expect_tx(&sm->q_full[t], kSub * kSubTileBytes);
-                for (int s = 0; s < kSub; ++s)
-                    tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64, r_lo[t] - p.q_off,
-                                tile_head(p, h, t), b, pol_q);
-            }
             if (p.q_prefetch_stride > 0 &&
                 blockIdx.x + static_cast<unsigned>(p.q_prefetch_stride) < gridDim.x) {
                 int nqb, nb, nh;
