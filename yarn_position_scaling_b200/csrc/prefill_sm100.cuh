@@ -77,6 +77,7 @@ struct alignas(64) PrefillParams {
     CUtensorMap tm_q;  // bf16 [B][Hq][T][d] (4-D, caller strides)
     CUtensorMap tm_k;  // fp16 [B*Hkv][T][d] rotated keys (workspace)
     CUtensorMap tm_v;  // fp16 [B*Hkv][T][d] values (workspace)
+    CUtensorMap tm_o;  // bf16 [B][Hq][T][d] output (caller strides), when o_tma is set
     __nv_bfloat16 *o;
     long long osb, osh, ost;
     float *o32;  // if set: O as fp32 [B][Hq][T][d] (contiguous) instead of o
@@ -92,6 +93,7 @@ struct alignas(64) PrefillParams {
     int causal, window, n_sink;
     int n_qblocks;
     int kv_major;  // CTA order: 1 = by KV head first (grouped heads), 0 = by query block
+    int o_tma;     // 1: the bf16 output leaves through shared memory and tm_o (TMA stores)
     // 1: the CTA's two query tiles are heads h and h + 1 of one KV group at the same 128
     // rows (so both see exactly the same key tiles); 0: rows [0, 128) and [128, 256) of one
     // head.  n_qblocks counts 128-row blocks with head pairs, 256-row blocks without.
@@ -126,6 +128,7 @@ struct PrefillSmem {
     uint64_t k_full[kKStages], k_empty[kKStages];
     uint64_t v_full[kVStages], v_empty[kVStages];
     uint64_t s_full[kQTiles], p_full[kQTiles], o_done[kQTiles];
+    uint64_t o_staged[kQTiles];  // the tile's softmax warps have written O into its Q buffer
     // Q rotation: per softmax warp, the angle (turns, reduced) of each pair at the
     // warp's first row, and the pair's rotations per position in fp32.
     float2 q_cs0[8][kMaxPairs];       // per softmax warp: (cos, sin) of pair i at its first row
@@ -257,7 +260,13 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
         : "memory");
 }
 
-template <int HD, bool kHalfPairs>
+// kShort: the instantiation for calls whose CTAs are short (a window, or up to 128 key
+// tiles each), where a CTA's start and end are a large share of its time: the barriers
+// are set up and the Q tiles requested before the CTA-wide barrier, the Q tiles of a CTA
+// one wave later are prefetched into L2, and the output leaves through shared memory by
+// TMA stores.  Long CTAs take the other instantiation: there these changes gain nothing
+// and cost the steady state 0.3-0.8% (code layout).
+template <int HD, bool kHalfPairs, bool kShort>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_attn_kernel(const __grid_constant__ PrefillParams p) {
     using Smem = PrefillSmem<HD>;
@@ -311,16 +320,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         r_hi[t] = min(r_lo[t] + kBlockM - 1, last_pos);
     }
 
-    // The TMA producer thread sets up the barriers and issues the Q tiles' loads at once,
-    // so that they overlap the TMEM allocation and the CTA-wide barrier below.
-    if (warp == 8 && lane == 0) {
-        prefetch_tensormap(&p.tm_q);
+    // Short CTAs: the TMA producer thread sets up the barriers and issues the Q tiles' loads
+    // at once, so that they overlap the TMEM allocation and the CTA-wide barrier below.
+    if (kShort ? (warp == 8 && lane == 0) : (threadIdx.x == 0)) {
+        if constexpr (kShort) prefetch_tensormap(&p.tm_q);
         for (int t = 0; t < kQTiles; ++t) {
             mbar_init(&sm->q_full[t], 1);
             mbar_init(&sm->q_ready[t], kBlockM / 32);  // one arrival per softmax warp
             mbar_init(&sm->s_full[t], 1);
             mbar_init(&sm->p_full[t], kBlockM / 32);
             mbar_init(&sm->o_done[t], 1);
+            mbar_init(&sm->o_staged[t], kBlockM / 32);
         }
         for (int s = 0; s < kKStages; ++s) {
             mbar_init(&sm->k_full[s], 1);
@@ -334,20 +344,29 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         mbar_init(&sm->lanes_ready, 2);  // warps 10 and 11
         sm->abort = 0;
         fence_mbar_init();
-        const uint64_t pol_q = l2_policy_evict_first();
-        for (int t = 0; t < kQTiles; ++t) {
-            if (r_lo[t] > r_hi[t]) continue;
-            mbar_arrive_expect_tx(&sm->q_full[t], kSub * kSubTileBytes);
-            for (int s = 0; s < kSub; ++s)
-                tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64, r_lo[t] - p.q_off,
-                            tile_head(p, h, t), b, pol_q);
+        if constexpr (kShort) {
+            const uint64_t pol_q = l2_policy_evict_first();
+            for (int t = 0; t < kQTiles; ++t) {
+                if (r_lo[t] > r_hi[t]) continue;
+                mbar_arrive_expect_tx(&sm->q_full[t], kSub * kSubTileBytes);
+                for (int s = 0; s < kSub; ++s)
+                    tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64, r_lo[t] - p.q_off,
+                                tile_head(p, h, t), b, pol_q);
+            }
+            prefetch_tensormap(&p.tm_k);
+            prefetch_tensormap(&p.tm_v);
         }
-        prefetch_tensormap(&p.tm_k);
-        prefetch_tensormap(&p.tm_v);
     }
     if (warp == 9) {
         tmem_alloc(&sm->tmem_base, kTmemCols);
         tmem_relinquish();
+    }
+    if constexpr (!kShort) {
+        if (warp == 8 && lane == 0) {
+            prefetch_tensormap(&p.tm_q);
+            prefetch_tensormap(&p.tm_k);
+            prefetch_tensormap(&p.tm_v);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -380,10 +399,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       } else if (warp == 8) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
-            // (the Q tiles' loads were issued with the barrier set-up)
+            // (short CTAs: the Q tiles' loads were issued with the barrier set-up)
             const uint64_t pol_kv = l2_policy_evict_last();
             bool ok = true;
-            if (p.q_prefetch_stride > 0 &&
+            if constexpr (!kShort) {
+                const uint64_t pol_q = l2_policy_evict_first();
+                for (int t = 0; t < kQTiles; ++t) {
+                    if (r_lo[t] > r_hi[t]) continue;
+                    mbar_arrive_expect_tx(&sm->q_full[t], kSub * kSubTileBytes);
+                    for (int s = 0; s < kSub; ++s)
+                        tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64,
+                                    r_lo[t] - p.q_off, tile_head(p, h, t), b, pol_q);
+                }
+            }
+            if (kShort && p.q_prefetch_stride > 0 &&
                 blockIdx.x + static_cast<unsigned>(p.q_prefetch_stride) < gridDim.x) {
                 int nqb, nb, nh;
                 cta_q_coords(p, static_cast<int>(blockIdx.x) + p.q_prefetch_stride, nqb, nb, nh);
@@ -833,7 +862,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                                                   __uint_as_float(raw[4 * q4 + 1]) * inv_l,
                                                   __uint_as_float(raw[4 * q4 + 2]) * inv_l,
                                                   __uint_as_float(raw[4 * q4 + 3]) * inv_l);
-                    } else if (row < p.T) {
+                    } else if ((kShort && p.o_tma) || row < p.T) {
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4) {
                             uint32_t pk[4];
@@ -844,8 +873,36 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                                     __uint_as_float(raw[q4 * 8 + 2 * e + 1]) * inv_l);
                                 pk[e] = *reinterpret_cast<uint32_t *>(&v2);
                             }
-                            *reinterpret_cast<uint4 *>(orow + c * 32 + q4 * 8) =
-                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            const uint4 v4 = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            if (kShort && p.o_tma) {
+                                // 16-byte chunk g of row r in this tile's Q buffer, in the
+                                // swizzled layout TMA reads (the buffer is free: the tile's
+                                // last S completed before its last PV)
+                                const int g = c * 4 + q4;
+                                *reinterpret_cast<uint4 *>(sm->q[t][g >> 3] + r * 128 +
+                                                           (((g & 7) ^ (r & 7)) << 4)) = v4;
+                            } else {
+                                *reinterpret_cast<uint4 *>(orow + c * 32 + q4 * 8) = v4;
+                            }
+                        }
+                    }
+                }
+                if (kShort && p.o_tma) {
+                    // The tile's rows leave by TMA: coalesced lines instead of one 16-byte
+                    // piece of 32 rows per store instruction; rows past T are not written.
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm->o_staged[t]);
+                    if ((warp & 3) == 0 && lane == 0) {
+                        if (mbar_wait(&sm->o_staged[t], 0, abort, p.timeout_ns)) {
+                            for (int s = 0; s < kSub; ++s)
+                                tma_store_4d(&p.tm_o, sm->q[t][s], s * 64, my_lo - p.q_off,
+                                             tile_head(p, h, t), b);
+                            bulk_commit_group();
+                            bulk_wait_group_read0();
+                        } else {
+                            raise_status(kStatusTimeoutSoftmax);
+                            sm->abort = 1;
                         }
                     }
                 }
