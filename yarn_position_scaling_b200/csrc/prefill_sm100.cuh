@@ -264,8 +264,8 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
 // tiles each), where a CTA's start and end are a large share of its time: the barriers
 // are set up and the Q tiles requested before the CTA-wide barrier, the Q tiles of a CTA
 // one wave later are prefetched into L2, and the output leaves through shared memory by
-// TMA stores.  Long CTAs take the other instantiation: there these changes gain nothing
-// and cost the steady state 0.3-0.8% (code layout).
+// TMA stores.  Long CTAs take the other instantiation: there these changes gain nothing,
+// and the prefetched Q tiles wait in L2 long enough to be evicted and read twice.
 template <int HD, bool kHalfPairs, bool kShort>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_attn_kernel(const __grid_constant__ PrefillParams p) {

@@ -445,9 +445,9 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     pp.osb = os[0]; pp.osh = os[1]; pp.ost = os[2];
     pp.head_pair = attend_head_pair(Hq, Hkv, window);
     // Short CTAs (a window, or up to 128 key tiles each) take the kernel instantiation that
-    // overlaps a CTA's start and end with its neighbours' work (Q prefetch of the next wave,
-    // early Q loads, TMA-store epilogue): +15-25% at 16K, +5-10% on the windowed 64K
-    // workloads; with long CTAs that gains nothing, and the prefetched tiles wait in L2 so
+    // shortens a CTA's start and end (Q prefetch of the next wave, early Q loads, TMA-store
+    // epilogue; measured one at a time: +12-17% at 16K, +3-8% on the windowed 64K
+    // workloads).  With long CTAs that gains nothing, and the prefetched tiles wait in L2 so
     // long that some are evicted and read twice (+0.7 GB of DRAM reads at 128K).
     bool short_ctas;
     {
