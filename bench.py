@@ -72,7 +72,7 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {
-    "prefill_attn_kernel<128, false, false>": ["prefill_sm100.cuh"],
+    "prefill_attn_kernel<128, false>": ["prefill_sm100.cuh"],
     "kv_prep_kernel<false>": ["kvprep_sm100.cuh"],
     "decode_split_kernel<128, 1>": ["decode_sm100.cuh"],
 }
@@ -654,14 +654,14 @@ def main():
         "vs_baseline": None, "dtype": "fp16",
         "data": "synthetic: seeded i.i.d. N(0,1) inputs rounded to bf16",
         "config": workload_config(wp, n),
-        "roofline": {"bound": "tensor", "kernel": "prefill_attn_kernel<128, false, false>",
+        "roofline": {"bound": "tensor", "kernel": "prefill_attn_kernel<128, false>",
                      "achieved": attn_tflops, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": attn_tflops / peak_t,
                      "peak_source": f"{peak_src} bf16 "
                                     f"{'sustained' if long_step else 'burst'} (of {peak_src}; "
                                     "the fp16 tensor rate equals bf16)",
                      "frac_of_burst": attn_tflops / peak_burst, "peak_burst": peak_burst,
-                     "traffic": ncu_traffic("prefill_attn_kernel<128, false, false>"),
+                     "traffic": ncu_traffic("prefill_attn_kernel<128, false>"),
                      "algorithmic_flops_per_launch": flops_step,
                      "kernel_ms": attn_ms_max / steps,
                      "kv_prep_ms": prep_ms_max / steps},

@@ -156,26 +156,6 @@ def test_strided_inputs_and_outputs_match_contiguous():
     assert torch.equal(out, ref)
 
 
-def test_short_and_long_cta_kernels_agree():
-    """A causal call of 32512 rows runs the short-CTA kernel instantiation (Q loads issued
-    with the barrier set-up, the next wave's Q prefetched, the output stored by TMA from
-    shared memory); one of 32768 rows runs the long-CTA one (at most 128 key tiles per CTA
-    is the boundary).  Causal rows see only earlier keys, so the first 32512 rows of the
-    two calls, and their log-sum-exp, must agree bit for bit."""
-    w = dataclasses.replace(synth.LLAMA3_128K, Hq=8, Hkv=2)
-    T_long, T_short = 32768, 32512
-    q, k, v = synth.prefill_inputs(w, "cuda", T=T_long)
-    tab = _table(w)
-    lse_l = torch.empty(q.shape[:3], device="cuda")
-    o_l = api.attn_prefill(q, k, v, tab, lse=lse_l)
-    qs, ks, vs = q[:, :, :T_short], k[:, :, :T_short], v[:, :, :T_short]
-    lse_s = torch.empty(qs.shape[:3], device="cuda")
-    o_s = api.attn_prefill(qs, ks, vs, tab, lse=lse_s)
-    api.device_status()
-    assert torch.equal(o_s, o_l[:, :, :T_short])
-    assert torch.equal(lse_s, lse_l[:, :, :T_short])
-
-
 def test_rotated_key_cache_output():
     w = synth.LLAMA2_16K
     T = 260

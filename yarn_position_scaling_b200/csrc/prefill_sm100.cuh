@@ -77,7 +77,6 @@ struct alignas(64) PrefillParams {
     CUtensorMap tm_q;  // bf16 [B][Hq][T][d] (4-D, caller strides)
     CUtensorMap tm_k;  // fp16 [B*Hkv][T][d] rotated keys (workspace)
     CUtensorMap tm_v;  // fp16 [B*Hkv][T][d] values (workspace)
-    CUtensorMap tm_o;  // bf16 [B][Hq][T][d] output (caller strides), when o_tma is set
     __nv_bfloat16 *o;
     long long osb, osh, ost;
     float *o32;  // if set: O as fp32 [B][Hq][T][d] (contiguous) instead of o
@@ -93,14 +92,10 @@ struct alignas(64) PrefillParams {
     int causal, window, n_sink;
     int n_qblocks;
     int kv_major;  // CTA order: 1 = by KV head first (grouped heads), 0 = by query block
-    int o_tma;     // 1: the bf16 output leaves through shared memory and tm_o (TMA stores)
     // 1: the CTA's two query tiles are heads h and h + 1 of one KV group at the same 128
     // rows (so both see exactly the same key tiles); 0: rows [0, 128) and [128, 256) of one
     // head.  n_qblocks counts 128-row blocks with head pairs, 256-row blocks without.
     int head_pair;
-    // > 0: each CTA's producer prefetches into L2 the Q tiles of CTA blockIdx + this stride
-    // (the SM count: about the CTA that will start next on some SM).
-    int q_prefetch_stride;
     int alibi;     // 1: add the ALiBi bias -m_h (i - j) to the logits
     // Split-KV: each (batch, head, query block) item is cut into n_split CTAs that take
     // equal shares of its key tiles; CTA s writes its normalised fp32 partial to
@@ -128,7 +123,6 @@ struct PrefillSmem {
     uint64_t k_full[kKStages], k_empty[kKStages];
     uint64_t v_full[kVStages], v_empty[kVStages];
     uint64_t s_full[kQTiles], p_full[kQTiles], o_done[kQTiles];
-    uint64_t o_staged[kQTiles];  // the tile's softmax warps have written O into its Q buffer
     // Q rotation: per softmax warp, the angle (turns, reduced) of each pair at the
     // warp's first row, and the pair's rotations per position in fp32.
     float2 q_cs0[8][kMaxPairs];       // per softmax warp: (cos, sin) of pair i at its first row
@@ -194,27 +188,6 @@ __device__ __forceinline__ bool tile_full(const PrefillParams &p, int r_lo, int 
     return true;
 }
 
-// Query block, batch and first query head of CTA `cta` (the kernel's own decode, for the
-// L2 prefetch of a later CTA's Q tiles).
-__device__ __forceinline__ void cta_q_coords(const PrefillParams &p, int cta, int &qb, int &b,
-                                             int &h) {
-    const int item = p.n_split > 1 ? cta / p.n_split : cta;
-    if (p.kv_major) {
-        const int units = p.head_pair ? p.group / 2 : p.group;
-        const int per_kv = p.n_qblocks * units;
-        const int bk = item / per_kv, rem = item % per_kv;
-        qb = p.n_qblocks - 1 - rem / units;
-        b = bk / p.Hkv;
-        h = (bk % p.Hkv) * p.group + (rem % units) * (p.head_pair ? 2 : 1);
-    } else {
-        const int bh_count = p.B * p.Hq;
-        qb = p.n_qblocks - 1 - item / bh_count;
-        const int rem = item % bh_count;
-        b = rem / p.Hq;
-        h = rem % p.Hq;
-    }
-}
-
 // Query head of tile t of a CTA whose tile 0 has head h.  (Evaluated where it is used: a
 // variable held across the softmax loop costs the d = 64 kernel a spill.)
 __device__ __forceinline__ int tile_head(const PrefillParams &p, int h, int t) {
@@ -260,13 +233,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
         : "memory");
 }
 
-// kShort: the instantiation for calls whose CTAs are short (a window, or up to 128 key
-// tiles each), where a CTA's start and end are a large share of its time: the barriers
-// are set up and the Q tiles requested before the CTA-wide barrier, the Q tiles of a CTA
-// one wave later are prefetched into L2, and the output leaves through shared memory by
-// TMA stores.  Long CTAs take the other instantiation: there these changes gain nothing,
-// and the prefetched Q tiles wait in L2 long enough to be evicted and read twice.
-template <int HD, bool kHalfPairs, bool kShort>
+template <int HD, bool kHalfPairs>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_attn_kernel(const __grid_constant__ PrefillParams p) {
     using Smem = PrefillSmem<HD>;
@@ -320,17 +287,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         r_hi[t] = min(r_lo[t] + kBlockM - 1, last_pos);
     }
 
-    // Short CTAs: the TMA producer thread sets up the barriers and issues the Q tiles' loads
-    // at once, so that they overlap the TMEM allocation and the CTA-wide barrier below.
-    if (kShort ? (warp == 8 && lane == 0) : (threadIdx.x == 0)) {
-        if constexpr (kShort) prefetch_tensormap(&p.tm_q);
+    if (threadIdx.x == 0) {
         for (int t = 0; t < kQTiles; ++t) {
             mbar_init(&sm->q_full[t], 1);
             mbar_init(&sm->q_ready[t], kBlockM / 32);  // one arrival per softmax warp
             mbar_init(&sm->s_full[t], 1);
             mbar_init(&sm->p_full[t], kBlockM / 32);
             mbar_init(&sm->o_done[t], 1);
-            mbar_init(&sm->o_staged[t], kBlockM / 32);
         }
         for (int s = 0; s < kKStages; ++s) {
             mbar_init(&sm->k_full[s], 1);
@@ -344,29 +307,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         mbar_init(&sm->lanes_ready, 2);  // warps 10 and 11
         sm->abort = 0;
         fence_mbar_init();
-        if constexpr (kShort) {
-            const uint64_t pol_q = l2_policy_evict_first();
-            for (int t = 0; t < kQTiles; ++t) {
-                if (r_lo[t] > r_hi[t]) continue;
-                mbar_arrive_expect_tx(&sm->q_full[t], kSub * kSubTileBytes);
-                for (int s = 0; s < kSub; ++s)
-                    tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64, r_lo[t] - p.q_off,
-                                tile_head(p, h, t), b, pol_q);
-            }
-            prefetch_tensormap(&p.tm_k);
-            prefetch_tensormap(&p.tm_v);
-        }
     }
     if (warp == 9) {
         tmem_alloc(&sm->tmem_base, kTmemCols);
         tmem_relinquish();
     }
-    if constexpr (!kShort) {
-        if (warp == 8 && lane == 0) {
-            prefetch_tensormap(&p.tm_q);
-            prefetch_tensormap(&p.tm_k);
-            prefetch_tensormap(&p.tm_v);
-        }
+    if (warp == 8 && lane == 0) {
+        prefetch_tensormap(&p.tm_q);
+        prefetch_tensormap(&p.tm_k);
+        prefetch_tensormap(&p.tm_v);
     }
     tc_fence_before();
     __syncthreads();
@@ -381,13 +330,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // ------------------------------------------ per-lane rotation table
         // (cos, sin) of lane * theta'_i for lane 0..31: angle reduced in fp64 (turns
         // minus the nearest integer), one fp32 sin/cos per entry, for all CTAs' rows.
-        // Unrolled so that independent entries overlap: one entry is a chain of fp64
-        // operations, a sin/cos and a store, and run one after another the table held
-        // up the Q rotation (a timing-only copy without it ran 5% faster at 16K and on
-        // the windowed 64K workloads).
-#pragma unroll 8
-        for (int k = 0; k < (HD / 2) * 32 / 64; ++k) {
-            const int e = (warp - 10) * 32 + lane + 64 * k;
+        for (int e = (warp - 10) * 32 + lane; e < (HD / 2) * 32; e += 64) {
             const int i = e >> 5, l = e & 31;
             const double tr = static_cast<double>(l) * p.turns[i];
             float sn, cs;
@@ -399,30 +342,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       } else if (warp == 8) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
-            // (short CTAs: the Q tiles' loads were issued with the barrier set-up)
+            const uint64_t pol_q = l2_policy_evict_first();
             const uint64_t pol_kv = l2_policy_evict_last();
             bool ok = true;
-            if constexpr (!kShort) {
-                const uint64_t pol_q = l2_policy_evict_first();
-                for (int t = 0; t < kQTiles; ++t) {
-                    if (r_lo[t] > r_hi[t]) continue;
-                    mbar_arrive_expect_tx(&sm->q_full[t], kSub * kSubTileBytes);
-                    for (int s = 0; s < kSub; ++s)
-                        tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64,
-                                    r_lo[t] - p.q_off, tile_head(p, h, t), b, pol_q);
-                }
-            }
-            if (kShort && p.q_prefetch_stride > 0 &&
-                blockIdx.x + static_cast<unsigned>(p.q_prefetch_stride) < gridDim.x) {
-                int nqb, nb, nh;
-                cta_q_coords(p, static_cast<int>(blockIdx.x) + p.q_prefetch_stride, nqb, nb, nh);
-                const int rows = p.head_pair ? kBlockM : kQTiles * kBlockM;
-                for (int t = 0; t < kQTiles; ++t) {
-                    const int r0 = nqb * rows + (p.head_pair ? 0 : t * kBlockM);
-                    if (r0 >= p.T) continue;
-                    for (int s = 0; s < kSub; ++s)
-                        tma_prefetch_4d(&p.tm_q, s * 64, r0, nh + (p.head_pair ? t : 0), nb);
-                }
+            for (int t = 0; t < kQTiles; ++t) {
+                if (r_lo[t] > r_hi[t]) continue;
+                mbar_arrive_expect_tx(&sm->q_full[t], kSub * kSubTileBytes);
+                for (int s = 0; s < kSub; ++s)
+                    tma_load_4d(sm->q[t][s], &p.tm_q, &sm->q_full[t], s * 64, r_lo[t] - p.q_off,
+                                tile_head(p, h, t), b, pol_q);
             }
             const int kv_plane = b * p.Hkv + kvh;
             int issued_k[kKStages] = {}, issued_v[kVStages] = {};
@@ -603,9 +531,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 // once per CTA), by angle addition.
                 float2 *cs0 = sm->q_cs0[warp];
                 const int pos0 = pos - lane;
-#pragma unroll
-                for (int k = 0; k < HD / 64; ++k) {
-                    const int i = lane + 32 * k;
+                for (int i = lane; i < HD / 2; i += 32) {
                     const double tr = static_cast<double>(pos0 + p.k_pos0) * p.turns[i];
                     float sn, cs;
                     __sincosf(static_cast<float>((tr - rint(tr)) * 6.283185307179586), &sn, &cs);
@@ -620,10 +546,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     cs = fmaf(a.x, l.x, -a.y * l.y);
                     sn = fmaf(a.y, l.x, a.x * l.y);
                 };
-                // 16-byte chunk g (elements 8g .. 8g+7) of this row in the swizzled tile.  The
-                // chunk loops below are unrolled so that the chunks' loads and rotations
-                // overlap: the rotation sits on the path to the CTA's first S (measured +3-9%
-                // at 16K and +2-7% on the windowed 64K workloads against one chunk at a time).
+                // 16-byte chunk g (elements 8g .. 8g+7) of this row in the swizzled tile
                 auto q_chunk = [&](int g) {
                     return reinterpret_cast<uint4 *>(sm->q[t][g >> 3] + r * 128 +
                                                      (((g & 7) ^ (r & 7)) << 4));
@@ -631,7 +554,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 if constexpr (kHalfPairs) {
                     // Pairs (i, i + d/2): chunk c holds the first elements of pairs
                     // 8c .. 8c+7, chunk c + d/16 their second elements.
-#pragma unroll
+#pragma unroll 1
                     for (int c = 0; c < HD / 16; ++c) {
                         uint4 *plo = q_chunk(c), *phi = q_chunk(c + HD / 16);
                         const uint4 rlo = *plo, rhi = *phi;
@@ -664,7 +587,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     }
                 } else {
                     // Pairs (2i, 2i+1): chunk c holds pairs 4c .. 4c+3.
-#pragma unroll
+#pragma unroll 1
                     for (int c = 0; c < HD / 8; ++c) {
                         uint4 *ptr = q_chunk(c);
                         const uint4 raw = *ptr;
@@ -862,7 +785,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                                                   __uint_as_float(raw[4 * q4 + 1]) * inv_l,
                                                   __uint_as_float(raw[4 * q4 + 2]) * inv_l,
                                                   __uint_as_float(raw[4 * q4 + 3]) * inv_l);
-                    } else if ((kShort && p.o_tma) || row < p.T) {
+                    } else if (row < p.T) {
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4) {
                             uint32_t pk[4];
@@ -873,36 +796,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                                     __uint_as_float(raw[q4 * 8 + 2 * e + 1]) * inv_l);
                                 pk[e] = *reinterpret_cast<uint32_t *>(&v2);
                             }
-                            const uint4 v4 = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                            if (kShort && p.o_tma) {
-                                // 16-byte chunk g of row r in this tile's Q buffer, in the
-                                // swizzled layout TMA reads (the buffer is free: the tile's
-                                // last S completed before its last PV)
-                                const int g = c * 4 + q4;
-                                *reinterpret_cast<uint4 *>(sm->q[t][g >> 3] + r * 128 +
-                                                           (((g & 7) ^ (r & 7)) << 4)) = v4;
-                            } else {
-                                *reinterpret_cast<uint4 *>(orow + c * 32 + q4 * 8) = v4;
-                            }
-                        }
-                    }
-                }
-                if (kShort && p.o_tma) {
-                    // The tile's rows leave by TMA: coalesced lines instead of one 16-byte
-                    // piece of 32 rows per store instruction; rows past T are not written.
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm->o_staged[t]);
-                    if ((warp & 3) == 0 && lane == 0) {
-                        if (mbar_wait(&sm->o_staged[t], 0, abort, p.timeout_ns)) {
-                            for (int s = 0; s < kSub; ++s)
-                                tma_store_4d(&p.tm_o, sm->q[t][s], s * 64, my_lo - p.q_off,
-                                             tile_head(p, h, t), b);
-                            bulk_commit_group();
-                            bulk_wait_group_read0();
-                        } else {
-                            raise_status(kStatusTimeoutSoftmax);
-                            sm->abort = 1;
+                            *reinterpret_cast<uint4 *>(orow + c * 32 + q4 * 8) =
+                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         }
                     }
                 }

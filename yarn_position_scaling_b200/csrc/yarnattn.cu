@@ -4,7 +4,6 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include <algorithm>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -135,21 +134,13 @@ int prepare_device(int *sm_count, DeviceState *out = nullptr) {
                 const void *fn;
                 size_t bytes;
             } attrs[] = {
-                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, false, false>),
+                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, false>),
                  yr::prefill_smem_bytes<128>()},
-                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, true, false>),
+                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, true>),
                  yr::prefill_smem_bytes<128>()},
-                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, false, false>),
+                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, false>),
                  yr::prefill_smem_bytes<64>()},
-                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, true, false>),
-                 yr::prefill_smem_bytes<64>()},
-                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, false, true>),
-                 yr::prefill_smem_bytes<128>()},
-                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, true, true>),
-                 yr::prefill_smem_bytes<128>()},
-                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, false, true>),
-                 yr::prefill_smem_bytes<64>()},
-                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, true, true>),
+                {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, true>),
                  yr::prefill_smem_bytes<64>()},
                 {reinterpret_cast<const void *>(&yr::decode_split_kernel<128, 1>),
                  yr::decode_smem_bytes<128>()},
@@ -168,15 +159,10 @@ int prepare_device(int *sm_count, DeviceState *out = nullptr) {
             // The prefill kernel re-splits its registers between warpgroups
             // (setmaxnreg); that only works if the launch reserves enough of them.
             st.prefill_regs_ok = true;
-            for (const void *fn :
-                 {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, false, false>),
-                  reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, true, false>),
-                  reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, false, false>),
-                  reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, true, false>),
-                  reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, false, true>),
-                  reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, true, true>),
-                  reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, false, true>),
-                  reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, true, true>)}) {
+            for (const void *fn : {reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, false>),
+                                   reinterpret_cast<const void *>(&yr::prefill_attn_kernel<128, true>),
+                                   reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, false>),
+                                   reinterpret_cast<const void *>(&yr::prefill_attn_kernel<64, true>)}) {
                 cudaFuncAttributes fa;
                 e = cudaFuncGetAttributes(&fa, fn);
                 if (e != cudaSuccess) return cuda_fail("cudaFuncGetAttributes", e);
@@ -443,33 +429,6 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     }
     pp.o = static_cast<__nv_bfloat16 *>(o);
     pp.osb = os[0]; pp.osh = os[1]; pp.ost = os[2];
-    pp.head_pair = attend_head_pair(Hq, Hkv, window);
-    // Short CTAs (a window, or up to 128 key tiles each) take the kernel instantiation that
-    // shortens a CTA's start and end (Q prefetch of the next wave, early Q loads, TMA-store
-    // epilogue; measured one at a time: +12-17% at 16K, +3-8% on the windowed 64K
-    // workloads).  With long CTAs that gains nothing, and the prefetched tiles wait in L2 so
-    // long that some are evicted and read twice (+0.7 GB of DRAM reads at 128K).
-    bool short_ctas;
-    {
-        const long long rows = pp.head_pair ? yr::kBlockM : yr::kQTiles * yr::kBlockM;
-        long long keys = window > 0 ? std::min<long long>(window + rows, Tk)
-                                    : (causal ? (Tk + rows) / 2 : Tk);
-        keys /= n_split;
-        short_ctas = keys <= 128ll * yr::kBlockN;
-    }
-    // A bf16 output whose strides TMA can take is written by TMA stores from shared memory.
-    pp.o_tma = 0;
-    if (short_ctas && o != nullptr && o32 == nullptr && strides_ok(os)) {
-        const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(T),
-                                    static_cast<cuuint64_t>(Hq), static_cast<cuuint64_t>(B)};
-        const cuuint64_t strides[3] = {static_cast<cuuint64_t>(os[2] * 2),
-                                       static_cast<cuuint64_t>(os[1] * 2),
-                                       static_cast<cuuint64_t>(os[0] * 2)};
-        const cuuint32_t box[4] = {64, 128, 1, 1};
-        rc = encode(&pp.tm_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, o, dims, strides, box, "o");
-        if (rc != YR_OK) return rc;
-        pp.o_tma = 1;
-    }
     pp.o32 = o32;
     pp.lse = lse;
     pp.q_dbg = q_rot_dbg;
@@ -478,9 +437,7 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     pp.causal = causal; pp.window = window; pp.n_sink = n_sink;
     // Windowed calls with an even number of query heads per KV head: a CTA takes two heads of
     // one group at the same 128 rows, so both query tiles see the same key tiles.
-    // The CTA one wave later (about the next to start on some SM) gets its Q tiles into L2
-    // while this one runs.
-    pp.q_prefetch_stride = short_ctas ? ds.sm_count : 0;
+    pp.head_pair = attend_head_pair(Hq, Hkv, window);
     pp.n_qblocks = pp.head_pair ? (T + 127) / 128 : (T + 255) / 256;
     pp.n_split = n_split;
     pp.split_rows = static_cast<long long>(B) * Hq * T;
@@ -501,22 +458,18 @@ int launch_attend(const void *q, void *o, float *lse, float *q_rot_dbg, int B, i
     for (int i = 0; i < d / 2; ++i) pp.turns[i] = tab->turns[i];
     const unsigned grid =
         static_cast<unsigned>(attend_items(B, Hq, Hkv, T, window) * n_split);
-    auto launch = [&](auto kern, size_t smem) {
-        kern<<<grid, yr::kPrefillThreads, smem, st>>>(pp);
-    };
-    const size_t smem128 = yr::prefill_smem_bytes<128>(), smem64 = yr::prefill_smem_bytes<64>();
     if (d == 128 && !half)
-        short_ctas ? launch(yr::prefill_attn_kernel<128, false, true>, smem128)
-                   : launch(yr::prefill_attn_kernel<128, false, false>, smem128);
+        yr::prefill_attn_kernel<128, false>
+            <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<128>(), st>>>(pp);
     else if (d == 128)
-        short_ctas ? launch(yr::prefill_attn_kernel<128, true, true>, smem128)
-                   : launch(yr::prefill_attn_kernel<128, true, false>, smem128);
+        yr::prefill_attn_kernel<128, true>
+            <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<128>(), st>>>(pp);
     else if (!half)
-        short_ctas ? launch(yr::prefill_attn_kernel<64, false, true>, smem64)
-                   : launch(yr::prefill_attn_kernel<64, false, false>, smem64);
+        yr::prefill_attn_kernel<64, false>
+            <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<64>(), st>>>(pp);
     else
-        short_ctas ? launch(yr::prefill_attn_kernel<64, true, true>, smem64)
-                   : launch(yr::prefill_attn_kernel<64, true, false>, smem64);
+        yr::prefill_attn_kernel<64, true>
+            <<<grid, yr::kPrefillThreads, yr::prefill_smem_bytes<64>(), st>>>(pp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("prefill_attn_kernel launch", e);
     return YR_OK;
