@@ -132,11 +132,17 @@ struct PrefillSmem {
     int abort;
 };
 
-// Key tiles one CTA visits: of the item's sequence -- the sink tiles [0, sink_end)
-// that precede the window, then the tiles from lo on -- the n starting at position
-// `first` (0, or the start of this CTA's share under split-KV).
+// Key tiles one CTA visits, the n starting at position `first` (0, or the start of this
+// CTA's share under split-KV) of the item's sequence.  Without a window the sequence is
+// the tiles from lo on.  With a window it is the window's tiles after its first (fully
+// visible to every row of a head-paired CTA), then the window's first tile, then the sink
+// tiles [0, sink_end): a row's first tile is then a full one, on which reference 0 is
+// normally kept, and the masked tiles (diagonal, window edge, sinks) come last and in a
+// row (order-balanced A/B, 20 rounds: +1.7% / +2.7% on the windowed 64K YaRN / RoPE
+// workloads; the online softmax takes its tiles in any order).
 struct TilePlan {
     int sink_end, lo, n, first;
+    int n_win;  // tiles of the window (lo .. lo + n_win - 1) when windowed, else 0
 };
 
 // q0 and last_row are query positions.
@@ -157,10 +163,15 @@ __device__ __forceinline__ TilePlan plan_tiles(const PrefillParams &p, int q0, i
     }
     tp.n = tp.sink_end + max(0, hi - tp.lo + 1);
     tp.first = 0;
+    tp.n_win = p.window > 0 ? tp.n - tp.sink_end : 0;
     return tp;
 }
 __device__ __forceinline__ int tile_at(const TilePlan &tp, int idx) {
     const int g = tp.first + idx;
+    if (tp.n_win > 0) {
+        if (g < tp.n_win - 1) return tp.lo + 1 + g;
+        return g == tp.n_win - 1 ? tp.lo : g - tp.n_win;
+    }
     return g < tp.sink_end ? g : tp.lo + (g - tp.sink_end);
 }
 
